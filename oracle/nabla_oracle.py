@@ -1,0 +1,258 @@
+"""fp64 CPU oracle for the NABLA hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, links or runs
+this module; only the tests, the package smoke check and the benchmark's CPU
+baseline leg use it.  It shares no code with the CUDA library: it is a slow,
+plain restatement of what the method computes, so that the kernels can be
+compared against it element by element.
+
+Sources (the paper "∇NABLA: Neighborhood Adaptive Block-Level Attention",
+arXiv 2507.13546v1):
+
+* Algorithm 1 "NABLA Sparse Mask Generation" (§3.1.2): block average pooling
+  of Q and K, the reduced attention map softmax(Qa Ka^T / sqrt(D)), row-wise
+  ascending sort, cumulative sum, binarisation cvals >= 1 - thr and the
+  restoration of the original order.
+* §3.1.3: the final mask is the union of the NABLA mask and the STA mask.
+* §2.2, Eq. 4: masked attention softmax(QK^T / sqrt(D) + M) V with
+  M in {-inf, 0}; §2.1, Eq. 2-3: dense attention.
+* §2.2: the STA window is a fixed 3D window of tiles centred on the query tile.
+
+Readings where the paper is silent (listed with reasons in the design notes):
+
+* sort direction: ascending, so that cvals >= 1 - thr keeps the largest
+  entries and thr = 1 keeps every block;
+* ties in the sort: stable (lower block index first);
+* 1 - thr is formed in fp64 from the float32 value of thr;
+* a partial last block (S not a multiple of 64) is averaged over its valid
+  tokens, and its missing key positions are excluded from attention;
+* STA window: |dt| <= wT // 2, |dy| <= wH // 2, |dx| <= wW // 2 in tile units,
+  truncated at the grid edge (no shifting of the window);
+* the mask is a constant of the backward pass (no gradient through pooling).
+
+Every function here is pinned by the CPU tests in tests/test_oracle_*.py
+against values the paper fixes (Table 1 STA sparsities), closed forms,
+library routines on special cases and brute force on tiny inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 64
+
+
+def num_blocks(S: int, N: int = BLOCK) -> int:
+    return -(-S // N)
+
+
+def as_f64(x) -> np.ndarray:
+    """Exact fp64 copy of a numpy array or torch tensor (bf16 and fp32 values
+    are exactly representable in fp64)."""
+    if hasattr(x, "detach"):
+        x = x.detach().float().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------- Algorithm 1
+
+def block_pool(X: np.ndarray, N: int = BLOCK) -> np.ndarray:
+    """Block averaging of Algorithm 1: view the S tokens as S/N blocks of N
+    tokens and take the mean over each block.  X: [..., S, D] -> [..., nb, D].
+    A partial last block is averaged over its valid tokens only."""
+    S = X.shape[-2]
+    nb = num_blocks(S, N)
+    out = np.empty(X.shape[:-2] + (nb, X.shape[-1]), dtype=np.float64)
+    for i in range(nb):
+        lo, hi = i * N, min(i * N + N, S)
+        out[..., i, :] = X[..., lo:hi, :].sum(axis=-2) / (hi - lo)
+    return out
+
+
+def reduced_scores(Qa: np.ndarray, Ka: np.ndarray) -> np.ndarray:
+    """Logits of the reduced attention map of Algorithm 1: Qa Ka^T / sqrt(D),
+    with D the head dimension.  [..., nb, D] x [..., nb, D] -> [..., nb, nb]."""
+    D = Qa.shape[-1]
+    return np.matmul(Qa, np.swapaxes(Ka, -1, -2)) / np.sqrt(D)
+
+
+def row_softmax(L: np.ndarray) -> np.ndarray:
+    """Softmax along the last dimension (max-subtracted)."""
+    z = L - L.max(axis=-1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def cdf_binarize(A: np.ndarray, thr: float):
+    """Binarisation via the CDF (Algorithm 1): sort every row ascending, take
+    the cumulative sum, keep the sorted positions whose cumulative value is
+    >= 1 - thr, and put the decisions back in the original column order.
+
+    Returns (M, C): the boolean mask and, at each original position, the
+    cumulative mass its sorted position reached (used for the tolerance band
+    around the threshold)."""
+    one_minus = 1.0 - float(np.float32(thr))
+    order = np.argsort(A, axis=-1, kind="stable")
+    vals = np.take_along_axis(A, order, axis=-1)
+    cvals = np.cumsum(vals, axis=-1)
+    keep_sorted = cvals >= one_minus
+    M = np.zeros(A.shape, dtype=bool)
+    C = np.zeros(A.shape, dtype=np.float64)
+    np.put_along_axis(M, order, keep_sorted, axis=-1)
+    np.put_along_axis(C, order, cvals, axis=-1)
+    return M, C
+
+
+def sta_mask(coords: np.ndarray, window) -> np.ndarray:
+    """Sliding-tile mask on block tile coordinates (§2.2, §3.1.3): block j is
+    visible from block i iff every tile-coordinate difference lies inside the
+    window centred on i.  coords: int [nb, 3] (t, y, x); window (wT, wH, wW)."""
+    c = np.asarray(coords, dtype=np.int64)
+    r = np.array([w // 2 for w in window], dtype=np.int64)
+    d = np.abs(c[:, None, :] - c[None, :, :])
+    return np.all(d <= r[None, None, :], axis=-1)
+
+
+def sta_grid_coords(T: int, Hy: int, Wx: int) -> np.ndarray:
+    """All tile coordinates of a T x Hy x Wx tile grid, time-major."""
+    t, y, x = np.meshgrid(np.arange(T), np.arange(Hy), np.arange(Wx), indexing="ij")
+    return np.stack([t.ravel(), y.ravel(), x.ravel()], 1)
+
+
+def nabla_mask(Q, K, thr: float, coords=None, window=None, N: int = BLOCK):
+    """Full mask builder for Q, K [B, H, S, D]: returns (M, C, P) with
+    M bool [B, H, nb, nb] = M_nabla OR M_STA (STA only if window is given),
+    C the cumulative mass of each entry in its sorted row and P the reduced
+    attention map."""
+    Qa = block_pool(as_f64(Q), N)
+    Ka = block_pool(as_f64(K), N)
+    P = row_softmax(reduced_scores(Qa, Ka))
+    M, C = cdf_binarize(P, thr)
+    if window is not None:
+        M = M | sta_mask(coords, window)[None, None]
+    return M, C, P
+
+
+def band_mask(C: np.ndarray, thr: float, band: float = 1e-5) -> np.ndarray:
+    """Entries whose cumulative mass lies within `band` of 1 - thr; there the
+    decision depends on rounding and a compared implementation may differ."""
+    return np.abs(C - (1.0 - float(np.float32(thr)))) <= band
+
+
+# --------------------------------------------------- mask -> index structures
+
+def mask_to_bits(M: np.ndarray) -> np.ndarray:
+    """Bool [..., nb, nb] -> uint32 [..., nb, ceil(nb/32)], bit (j % 32) of
+    word j // 32 set iff block j is kept."""
+    nb = M.shape[-1]
+    W = -(-nb // 32)
+    pad = np.zeros(M.shape[:-1] + (W * 32,), dtype=np.uint64)
+    pad[..., :nb] = M
+    pad = pad.reshape(M.shape[:-1] + (W, 32))
+    w = (pad << np.arange(32, dtype=np.uint64)).sum(axis=-1)
+    return w.astype(np.uint32)
+
+
+def bits_to_mask(bits: np.ndarray, nb: int) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint64)[..., :, None] >> np.arange(32, dtype=np.uint64)
+    return (b & 1).astype(bool).reshape(bits.shape[:-1] + (-1,))[..., :nb]
+
+
+# ------------------------------------------------------------------ attention
+
+def _allowed_keys(M_row: np.ndarray, S: int, N: int = BLOCK) -> np.ndarray:
+    """Token indices of the keys inside the kept blocks of one mask row."""
+    blocks = np.nonzero(M_row)[0]
+    if blocks.size == 0:
+        return np.zeros(0, dtype=np.int64)
+    return np.concatenate([np.arange(j * N, min(j * N + N, S)) for j in blocks])
+
+
+def masked_attention(Q, K, V, M: np.ndarray, N: int = BLOCK):
+    """Eq. 4 with a block mask: for every query token, softmax over the keys of
+    the kept blocks of its block row (all other keys get -inf), then the
+    weighted sum of values.  Q, K, V [B, H, S, D]; M bool [B, H, nb, nb].
+    Returns (O [B, H, S, D], LSE [B, H, S]) in fp64, LSE = log sum exp of the
+    scaled logits over the allowed keys."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    B, H, S, D = Q.shape
+    nb = num_blocks(S, N)
+    O = np.zeros_like(Q)
+    LSE = np.full((B, H, S), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                rows = slice(i * N, min(i * N + N, S))
+                keys = _allowed_keys(M[b, h, i], S, N)
+                if keys.size == 0:
+                    continue
+                logit = Q[b, h, rows] @ K[b, h, keys].T / np.sqrt(D)
+                mx = logit.max(axis=-1, keepdims=True)
+                e = np.exp(logit - mx)
+                s = e.sum(axis=-1, keepdims=True)
+                O[b, h, rows] = (e / s) @ V[b, h, keys]
+                LSE[b, h, rows] = (mx + np.log(s))[:, 0]
+    return O, LSE
+
+
+def masked_attention_rows(Q, K, V, M: np.ndarray, b: int, h: int, rows, N: int = BLOCK):
+    """Same as masked_attention for a few query tokens of one (b, h); returns
+    (O [len(rows), D], LSE [len(rows)])."""
+    Qh, Kh, Vh = as_f64(Q[b, h]), as_f64(K[b, h]), as_f64(V[b, h])
+    S, D = Qh.shape
+    rows = np.asarray(rows)
+    O = np.zeros((rows.size, D))
+    LSE = np.full(rows.size, -np.inf)
+    for n, s in enumerate(rows):
+        keys = _allowed_keys(M[b, h, s // N], S, N)
+        if keys.size == 0:
+            continue
+        logit = Kh[keys] @ Qh[s] / np.sqrt(D)
+        mx = logit.max()
+        e = np.exp(logit - mx)
+        O[n] = e @ Vh[keys] / e.sum()
+        LSE[n] = mx + np.log(e.sum())
+    return O, LSE
+
+
+def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK):
+    """Gradients of masked_attention with the mask held constant: with
+    P = softmax(Q K_sel^T / sqrt(D)) per query block,
+      dV_sel += P^T dO,  dP = dO V_sel^T,  dS = P * (dP - rowsum(P * dP)),
+      dQ = dS K_sel / sqrt(D),  dK_sel += dS^T Q / sqrt(D).
+    Returns (dQ, dK, dV) fp64 [B, H, S, D]."""
+    Q, K, V, dO = as_f64(Q), as_f64(K), as_f64(V), as_f64(dO)
+    B, H, S, D = Q.shape
+    nb = num_blocks(S, N)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    scale = 1.0 / np.sqrt(D)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                rows = slice(i * N, min(i * N + N, S))
+                keys = _allowed_keys(M[b, h, i], S, N)
+                if keys.size == 0:
+                    continue
+                logit = Q[b, h, rows] @ K[b, h, keys].T * scale
+                e = np.exp(logit - logit.max(axis=-1, keepdims=True))
+                P = e / e.sum(axis=-1, keepdims=True)
+                g = dO[b, h, rows]
+                dV[b, h, keys] += P.T @ g
+                dP = g @ V[b, h, keys].T
+                dS = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+                dQ[b, h, rows] = dS @ K[b, h, keys] * scale
+                dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
+    return dQ, dK, dV
+
+
+# ------------------------------------------------------------ error metrics
+
+def max_abs(x, ref) -> float:
+    x, ref = as_f64(x), as_f64(ref)
+    return float(np.max(np.abs(x - ref))) if ref.size else 0.0
+
+
+def mean_rel(x, ref) -> float:
+    """mean |x - ref| / mean |ref| (a ratio of means, robust near zero)."""
+    x, ref = as_f64(x), as_f64(ref)
+    den = float(np.mean(np.abs(ref)))
+    return float(np.mean(np.abs(x - ref))) / den if den > 0 else float(np.mean(np.abs(x)))

@@ -1,0 +1,128 @@
+"""Plants plausible mistakes in the oracle (CPU only) and checks that the pins
+in test_oracle_pins.py catch every one of them: a wrong sort direction, a
+strict comparison, an exclusive cumulative sum, thr for 1 - thr, a missing
+order restoration, a tail block divided by 64, transposed or unscaled scores,
+softmax over the wrong axis, a wrong STA half-width, a transposed block mask
+and a dropped term in the backward pass."""
+import numpy as np
+import pytest
+
+from oracle import nabla_oracle as orc
+from tests import test_oracle_pins as pins
+
+_ORIG_ATTN = orc.masked_attention
+
+
+def _all_pins():
+    checks = []
+    for case in pins._read_golden("cdf_select_cases.txt"):
+        checks.append(lambda c=case: pins.test_cdf_hand_cases(c))
+    for case in pins._read_golden("sta_table1.txt"):
+        checks.append(lambda c=case: pins.test_sta_reproduces_table1_sparsity(c))
+    for name in dir(pins):
+        fn = getattr(pins, name)
+        if name.startswith("test_") and callable(fn) and name not in (
+                "test_cdf_hand_cases", "test_sta_reproduces_table1_sparsity"):
+            checks.append(fn)
+    return checks
+
+
+def _some_pin_fails():
+    for check in _all_pins():
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+def _cdf_variant(descending=False, strict=False, exclusive=False, use_thr=False, no_reorder=False):
+    def f(A, thr):
+        lim = float(np.float32(thr)) if use_thr else 1.0 - float(np.float32(thr))
+        order = np.argsort(-A if descending else A, axis=-1, kind="stable")
+        vals = np.take_along_axis(A, order, axis=-1)
+        c = np.cumsum(vals, axis=-1)
+        if exclusive:
+            c = c - vals
+        keep = c > lim if strict else c >= lim
+        M = np.zeros(A.shape, dtype=bool)
+        C = np.zeros(A.shape)
+        if no_reorder:
+            M[...] = keep
+            C[...] = c
+        else:
+            np.put_along_axis(M, order, keep, axis=-1)
+            np.put_along_axis(C, order, c, axis=-1)
+        return M, C
+    return f
+
+
+def _pool_div64(X, N=64):
+    S = X.shape[-2]
+    nb = orc.num_blocks(S, N)
+    return np.stack([X[..., i * N:min(i * N + N, S), :].sum(-2) / N for i in range(nb)], -2)
+
+
+def _sta_full_width(coords, window):
+    c = np.asarray(coords, dtype=np.int64)
+    d = np.abs(c[:, None, :] - c[None, :, :])
+    return np.all(d <= np.array(window)[None, None, :], axis=-1)
+
+
+def _attn_unscaled(Q, K, V, M, N=64):
+    D = np.asarray(orc.as_f64(Q)).shape[-1]
+    return _ORIG_ATTN(orc.as_f64(Q) * np.sqrt(D), K, V, M, N)
+
+
+def _attn_transposed_mask(Q, K, V, M, N=64):
+    return _ORIG_ATTN(Q, K, V, np.swapaxes(M, -1, -2), N)
+
+
+def _bwd_no_rowsum(Q, K, V, dO, M, N=64):
+    Q, K, V, dO = (orc.as_f64(x) for x in (Q, K, V, dO))
+    B, H, S, D = Q.shape
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for b in range(B):
+        for h in range(H):
+            for i in range(orc.num_blocks(S, N)):
+                rows = slice(i * N, min(i * N + N, S))
+                keys = orc._allowed_keys(M[b, h, i], S, N)
+                lg = Q[b, h, rows] @ K[b, h, keys].T / np.sqrt(D)
+                e = np.exp(lg - lg.max(-1, keepdims=True))
+                P = e / e.sum(-1, keepdims=True)
+                dV[b, h, keys] += P.T @ dO[b, h, rows]
+                dS = P * (dO[b, h, rows] @ V[b, h, keys].T)
+                dQ[b, h, rows] = dS @ K[b, h, keys] / np.sqrt(D)
+                dK[b, h, keys] += dS.T @ Q[b, h, rows] / np.sqrt(D)
+    return dQ, dK, dV
+
+
+MUTANTS = {
+    "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
+    "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
+    "exclusive_cumsum": ("cdf_binarize", _cdf_variant(exclusive=True)),
+    "thr_not_one_minus_thr": ("cdf_binarize", _cdf_variant(use_thr=True)),
+    "no_order_restoration": ("cdf_binarize", _cdf_variant(no_reorder=True)),
+    "tail_divided_by_64": ("block_pool", _pool_div64),
+    "scores_transposed": ("reduced_scores",
+                          lambda Qa, Ka: np.matmul(Ka, np.swapaxes(Qa, -1, -2)) / np.sqrt(Qa.shape[-1])),
+    "scores_scaled_by_D": ("reduced_scores",
+                           lambda Qa, Ka: np.matmul(Qa, np.swapaxes(Ka, -1, -2)) / Qa.shape[-1]),
+    "softmax_wrong_axis": ("row_softmax",
+                           lambda L: np.exp(L - L.max(-2, keepdims=True)) / np.exp(L - L.max(-2, keepdims=True)).sum(-2, keepdims=True)),
+    "sta_full_width": ("sta_mask", _sta_full_width),
+    "attention_unscaled": ("masked_attention", _attn_unscaled),
+    "attention_mask_transposed": ("masked_attention", _attn_transposed_mask),
+    "backward_no_rowsum": ("masked_attention_bwd", _bwd_no_rowsum),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    assert _some_pin_fails(), f"no pin caught the planted mistake {name}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert not _some_pin_fails()

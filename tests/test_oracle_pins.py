@@ -1,0 +1,286 @@
+"""Pins of the fp64 oracle against things other than itself: hand-worked
+cases of Algorithm 1, Table 1's STA sparsities, closed forms, brute force on
+tiny rows, library routines on special cases and finite differences.
+
+Source: "∇NABLA: Neighborhood Adaptive Block-Level Attention"
+(arXiv 2507.13546v1): §3.1.2 Algorithm 1, §3.1.3, §2.1 Eq. 2-3, §2.2 Eq. 4-5,
+§4.1 Table 1.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nabla_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append([part.split() for part in line.split(";")])
+    return rows
+
+
+# ------------------------------------------------------------ selection rule
+
+@pytest.mark.parametrize("case", _read_golden("cdf_select_cases.txt"))
+def test_cdf_hand_cases(case):
+    thr = float(case[0][0])
+    P = np.array([float(x) for x in case[1]])
+    want = np.array([bool(int(x)) for x in case[2]])
+    M, C = orc.cdf_binarize(P[None, :], thr)
+    assert (M[0] == want).all(), (M[0], want)
+
+
+def _brute_force_keep(P, thr):
+    """Minimal set of blocks whose mass exceeds thr; among sets of that size,
+    the one with the largest mass (the definition the selection is meant to
+    realise, searched exhaustively)."""
+    n = P.size
+    best = None
+    for k in range(1, n + 1):
+        for sub in itertools.combinations(range(n), k):
+            m = P[list(sub)].sum()
+            if m > thr and (best is None or m > best[0]):
+                best = (m, sub)
+        if best is not None:
+            break
+    keep = np.zeros(n, dtype=bool)
+    keep[list(best[1])] = True
+    return keep
+
+
+def test_cdf_matches_brute_force_on_tiny_rows():
+    rng = np.random.default_rng(7)
+    checked = 0
+    for trial in range(400):
+        n = int(rng.integers(1, 10))
+        P = rng.dirichlet(np.full(n, rng.uniform(0.2, 3.0)))
+        thr = float(np.float32(rng.uniform(0.05, 0.999)))
+        M, C = orc.cdf_binarize(P[None, :], thr)
+        if np.any(np.abs(C - (1 - thr)) < 1e-12):
+            continue
+        assert (M[0] == _brute_force_keep(P, thr)).all()
+        checked += 1
+    assert checked > 350
+
+
+def test_cdf_invariants_random_rows():
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = int(rng.integers(1, 300))
+        P = orc.row_softmax(rng.normal(0, rng.uniform(0.1, 6), size=(4, n)))
+        thrs = sorted(float(np.float32(t)) for t in rng.uniform(0.01, 1.0, size=3))
+        prev = None
+        for thr in thrs + [1.0]:
+            M, C = orc.cdf_binarize(P, thr)
+            for r in range(P.shape[0]):
+                kept, drop = P[r][M[r]], P[r][~M[r]]
+                assert kept.size >= 1
+                assert kept.sum() >= thr - 1e-12
+                assert kept.sum() - kept.min() <= thr + 1e-12 or thr == 1.0
+                if drop.size:
+                    assert kept.min() >= drop.max()
+            if prev is not None:
+                assert (prev <= M).all()  # monotone in thr
+            prev = M
+        assert prev.all()  # thr = 1 keeps every block
+
+
+def test_band_mask_marks_near_threshold_entries():
+    P = np.array([[0.1, 0.2, 0.3, 0.4]])
+    M, C = orc.cdf_binarize(P, 0.7)   # 1 - thr = 0.3 (float32 0.7) ~ c of the 0.2 entry
+    band = orc.band_mask(C, 0.7)
+    assert band[0].tolist() == [False, True, False, False]
+
+
+# ------------------------------------------------ pooling, scores, softmax
+
+def test_block_pool_closed_form_with_ragged_tail():
+    S, D = 70, 2
+    X = np.zeros((S, D))
+    X[:, 0] = np.arange(S)
+    X[:, 1] = 1.0
+    Xa = orc.block_pool(X)
+    assert Xa.shape == (2, 2)
+    assert Xa[0].tolist() == [31.5, 1.0]          # mean of 0..63
+    assert Xa[1].tolist() == [66.5, 1.0]          # mean of 64..69 (6 valid tokens)
+
+
+def test_block_pool_constant_blocks_exact():
+    rng = np.random.default_rng(3)
+    vals = rng.integers(-1000, 1000, size=(5, 16)) / 8.0   # sums stay exact in fp64
+    X = np.repeat(vals, 64, axis=0)[:300]          # last block has 44 tokens
+    assert np.array_equal(orc.block_pool(X), vals)
+
+
+def test_reduced_scores_and_softmax_closed_form():
+    Qa = np.array([[1.0, 1.0, 0.0, 0.0], [0.0, 2.0, 0.0, 0.0]])
+    Ka = np.array([[2.0, 0.0, 0.0, 0.0], [0.0, 3.0, 0.0, 0.0]])
+    L = orc.reduced_scores(Qa, Ka)                 # / sqrt(4) = / 2
+    assert np.allclose(L, [[1.0, 1.5], [0.0, 3.0]], rtol=0, atol=1e-15)
+    P = orc.row_softmax(L)
+    s0 = 1 / (1 + math.exp(0.5))
+    s1 = 1 / (1 + math.exp(3.0))
+    assert np.allclose(P, [[s0, 1 - s0], [s1, 1 - s1]], rtol=0, atol=1e-15)
+
+
+def test_nabla_mask_on_block_constant_inputs():
+    # Two blocks of D=4 tokens with the pooled vectors of the closed-form
+    # case above: P = [[.378, .622], [.047, .953]].  thr = 0.5: row 0 keeps
+    # only block 1 (mass .622 > .5), row 1 keeps only block 1.
+    # thr = 0.7: row 0 needs both blocks, row 1 still only block 1.
+    Qa = np.array([[1.0, 1.0, 0.0, 0.0], [0.0, 2.0, 0.0, 0.0]])
+    Ka = np.array([[2.0, 0.0, 0.0, 0.0], [0.0, 3.0, 0.0, 0.0]])
+    Q = np.repeat(Qa, 64, axis=0)[None, None]
+    K = np.repeat(Ka, 64, axis=0)[None, None]
+    M, C, P = orc.nabla_mask(Q, K, 0.5)
+    assert M[0, 0].tolist() == [[False, True], [False, True]]
+    M, C, P = orc.nabla_mask(Q, K, 0.7)
+    assert M[0, 0].tolist() == [[True, True], [False, True]]
+
+
+# ---------------------------------------------------------------------- STA
+
+@pytest.mark.parametrize("case", _read_golden("sta_table1.txt"))
+def test_sta_reproduces_table1_sparsity(case):
+    grid = tuple(int(x) for x in case[0])
+    window = tuple(int(x) for x in case[1])
+    want = float(case[2][0])
+    M = orc.sta_mask(orc.sta_grid_coords(*grid), window)
+    sparsity = 100.0 * (1.0 - M.mean())
+    assert round(sparsity, 2) == want
+
+
+def test_sta_eq5_bound_and_interior_count():
+    # Eq. 5: dense blocks = prod(W/B) * prod(L/B); with odd windows every
+    # interior tile sees exactly wT*wH*wW tiles and the total cannot exceed Eq. 5.
+    grid, window = (9, 9, 9), (3, 5, 3)
+    c = orc.sta_grid_coords(*grid)
+    M = orc.sta_mask(c, window)
+    assert M.sum() <= np.prod(window) * np.prod(grid)
+    centre = np.ravel_multi_index((4, 4, 4), grid)
+    assert M[centre].sum() == 3 * 5 * 3
+    assert (M == M.T).all() and M.diagonal().all()
+
+
+def test_mask_bits_roundtrip():
+    rng = np.random.default_rng(5)
+    M = rng.random((2, 3, 70, 70)) < 0.3
+    bits = orc.mask_to_bits(M)
+    assert bits.shape == (2, 3, 70, 3) and bits.dtype == np.uint32
+    assert (orc.bits_to_mask(bits, 70) == M).all()
+    # bit j % 32 of word j // 32
+    one = np.zeros((1, 40), dtype=bool)
+    one[0, 33] = True
+    assert orc.mask_to_bits(one)[0].tolist() == [0, 2]
+
+
+# ---------------------------------------------------------------- attention
+
+def _sdpa(Q, K, V, token_mask=None):
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x)) for x in (Q, K, V))
+    m = None if token_mask is None else torch.from_numpy(token_mask)
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m).numpy()
+
+
+def _token_mask(M, S):
+    blk = np.arange(S) // 64
+    return M[..., blk[:, None], blk[None, :]]
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).normal(size=shape)
+
+
+def test_attention_all_blocks_equals_dense_sdpa():
+    B, H, S, D = 1, 2, 150, 16
+    Q, K, V = (_rand((B, H, S, D), s) for s in (1, 2, 3))
+    M = np.ones((B, H, 3, 3), dtype=bool)
+    O, LSE = orc.masked_attention(Q, K, V, M)
+    assert np.abs(O - _sdpa(Q, K, V)).max() < 1e-12
+    logits = np.einsum("bhsd,bhtd->bhst", Q, K) / math.sqrt(D)
+    assert np.abs(LSE - np.log(np.exp(logits).sum(-1))).max() < 1e-12
+
+
+def test_attention_block_mask_equals_sdpa_with_token_mask():
+    B, H, S, D = 2, 2, 200, 8                      # 4 blocks, last has 8 tokens
+    Q, K, V = (_rand((B, H, S, D), s) for s in (4, 5, 6))
+    rng = np.random.default_rng(9)
+    M = rng.random((B, H, 4, 4)) < 0.5
+    M[..., np.arange(4), rng.integers(0, 4, size=4)] = True   # every row keeps one
+    O, _ = orc.masked_attention(Q, K, V, M)
+    assert np.abs(O - _sdpa(Q, K, V, _token_mask(M, S))).max() < 1e-12
+
+
+def test_attention_closed_forms():
+    B, H, S, D = 1, 1, 130, 8
+    rng = np.random.default_rng(2)
+    K, V = rng.normal(size=(B, H, S, D)), rng.normal(size=(B, H, S, D))
+    M = np.array([[[[True, False, True], [False, True, False], [True, True, True]]]])
+    # Q = 0: uniform weights over the allowed keys, LSE = log(#keys)
+    O, LSE = orc.masked_attention(np.zeros((B, H, S, D)), K, V, M)
+    keys0 = np.r_[0:64, 128:130]
+    assert np.allclose(O[0, 0, 5], V[0, 0, keys0].mean(0), atol=1e-13)
+    assert abs(LSE[0, 0, 5] - math.log(keys0.size)) < 1e-13
+    assert np.allclose(O[0, 0, 129], V[0, 0].mean(0), atol=1e-13)
+    # constant V: output is that constant whatever the weights
+    Q = rng.normal(size=(B, H, S, D))
+    O, _ = orc.masked_attention(Q, K, np.full((B, H, S, D), 3.25), M)
+    assert np.abs(O - 3.25).max() < 1e-13
+
+
+def test_attention_rows_agree_with_full():
+    B, H, S, D = 1, 2, 190, 8
+    Q, K, V = (_rand((B, H, S, D), s) for s in (7, 8, 9))
+    M = np.random.default_rng(1).random((B, H, 3, 3)) < 0.6
+    M[..., np.arange(3), np.arange(3)] = True
+    O, LSE = orc.masked_attention(Q, K, V, M)
+    rows = [0, 63, 64, 150, 189]
+    Or, Lr = orc.masked_attention_rows(Q, K, V, M, 0, 1, rows)
+    assert np.abs(Or - O[0, 1, rows]).max() < 1e-13
+    assert np.abs(Lr - LSE[0, 1, rows]).max() < 1e-13
+
+
+def test_backward_matches_torch_autograd_and_finite_differences():
+    B, H, S, D = 1, 2, 128 + 40, 8
+    Q, K, V, dO = (_rand((B, H, S, D), s) for s in (10, 11, 12, 13))
+    M = np.array([[[True, False, True], [True, True, False], [False, True, True]],
+                  [[True, True, True], [False, True, False], [True, False, True]]])[None]
+    dQ, dK, dV = orc.masked_attention_bwd(Q, K, V, dO, M)
+    q, k, v = (torch.from_numpy(x.copy()).requires_grad_() for x in (Q, K, V))
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=torch.from_numpy(_token_mask(M, S)))
+    out.backward(torch.from_numpy(dO))
+    for mine, ref in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        assert np.abs(mine - ref.numpy()).max() < 1e-11
+    # central finite differences of <O, dO> on a few coordinates
+    def f(Qx, Kx, Vx):
+        return float((orc.masked_attention(Qx, Kx, Vx, M)[0] * dO).sum())
+    h = 1e-6
+    rng = np.random.default_rng(0)
+    for which, grad in ((0, dQ), (1, dK), (2, dV)):
+        for _ in range(4):
+            idx = (0, int(rng.integers(2)), int(rng.integers(S)), int(rng.integers(D)))
+            args = [Q.copy(), K.copy(), V.copy()]
+            args[which][idx] += h
+            fp = f(*args)
+            args[which][idx] -= 2 * h
+            fm = f(*args)
+            assert abs((fp - fm) / (2 * h) - grad[idx]) < 1e-6
+
+
+def test_error_metrics():
+    ref = np.array([1.0, -2.0, 4.0])
+    x = ref + np.array([0.1, 0.0, -0.2])
+    assert abs(orc.max_abs(x, ref) - 0.2) < 1e-15
+    assert abs(orc.mean_rel(x, ref) - (0.3 / 3) / (7 / 3)) < 1e-15
