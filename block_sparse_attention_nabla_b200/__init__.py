@@ -1,0 +1,247 @@
+"""NABLA adaptive block-sparse attention for B200 (sm_100a).
+
+Python binding of libnabla.so (include/nabla.h).  This module only marshals
+arguments: it checks tensor shapes and dtypes, allocates outputs with torch
+and passes raw device pointers and the current CUDA stream to the C ABI.  Every
+step of the computation runs in the library's CUDA kernels; if the library is
+missing or fails to load, every call raises NablaError.
+
+    mask = build_mask(q, k, thr=0.8)            # Algorithm 1 (+ optional STA)
+    o, lse = attn_fwd(q, k, v, mask)            # Eq. 4 over the kept tiles
+    dq, dk, dv = attn_bwd(q, k, v, o, do, lse, mask)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
+           "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
+           "BLOCK", "BF16", "FP32"]
+
+BLOCK = 64
+BF16, FP32 = 0, 1
+_DTYPES = {torch.bfloat16: BF16, torch.float32: FP32}
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so")
+
+# Exported symbols, in the order include/nabla.h declares them.
+SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_mask_from_bits", "nabla_attn_fwd",
+           "nabla_attn_bwd", "nabla_workspace_status", "nabla_set_wait_limit_ns",
+           "nabla_last_error", "nabla_abi_version"]
+
+
+class NablaError(RuntimeError):
+    pass
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("block", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class _Sta(ctypes.Structure):
+    _fields_ = [("block_coords", ctypes.c_void_p), ("wT", ctypes.c_int32),
+                ("wH", ctypes.c_int32), ("wW", ctypes.c_int32)]
+
+
+class _Mask(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_void_p), ("cnt", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+                ("cnt_t", ctypes.c_void_p), ("idx_t", ctypes.c_void_p), ("work", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libnabla.so (once) and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise NablaError(f"{LIB_PATH} is missing; build it with "
+                         "`python -m block_sparse_attention_nabla_b200.build`")
+    try:
+        L = ctypes.CDLL(LIB_PATH)
+    except OSError as e:
+        raise NablaError(f"cannot load {LIB_PATH}: {e}") from e
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    SH, ST, MK = ctypes.POINTER(_Shape), ctypes.POINTER(_Sta), ctypes.POINTER(_Mask)
+    L.nabla_workspace_size.argtypes, L.nabla_workspace_size.restype = [SH, I32], SZ
+    L.nabla_build_mask.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P, SZ, P]
+    L.nabla_mask_from_bits.argtypes = [SH, P, MK, P, SZ, P]
+    L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
+    L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
+    L.nabla_workspace_status.argtypes = [P, ctypes.POINTER(I32), P]
+    L.nabla_set_wait_limit_ns.argtypes, L.nabla_set_wait_limit_ns.restype = [ctypes.c_uint64], None
+    L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
+    L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
+    for name in ("nabla_build_mask", "nabla_mask_from_bits", "nabla_attn_fwd", "nabla_attn_bwd",
+                 "nabla_workspace_status"):
+        getattr(L, name).restype = I32
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        msg = lib().nabla_last_error().decode(errors="replace")
+        raise NablaError(f"{what} failed with status {status}: {msg}")
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _shape_of(q: torch.Tensor) -> _Shape:
+    if q.dim() != 4:
+        raise NablaError(f"expected [B, H, S, D], got shape {tuple(q.shape)}")
+    if q.dtype not in _DTYPES:
+        raise NablaError(f"dtype must be bfloat16 or float32, got {q.dtype}")
+    if not q.is_cuda:
+        raise NablaError("tensors must be CUDA tensors")
+    B, H, S, D = q.shape
+    return _Shape(B, H, S, D, BLOCK, _DTYPES[q.dtype])
+
+
+def _same(ref: torch.Tensor, *ts: torch.Tensor) -> None:
+    for t in ts:
+        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise NablaError(f"tensor {tuple(t.shape)} {t.dtype} does not match {tuple(ref.shape)} {ref.dtype}")
+        if not t.is_contiguous():
+            raise NablaError("tensors must be contiguous")
+
+
+def num_blocks(S: int) -> int:
+    return -(-S // BLOCK)
+
+
+@dataclass
+class Mask:
+    """Device-side mask of one problem (layout in include/nabla.h)."""
+    bits: torch.Tensor           # uint32 words as int32 [B, H, nb, W]
+    cnt: torch.Tensor            # int32 [B, H, nb]
+    idx: torch.Tensor            # int32 [B, H, nb, nb]
+    work: torch.Tensor           # int32 [B * H * npairs, 2]
+    cnt_t: torch.Tensor | None = None
+    idx_t: torch.Tensor | None = None
+
+    def as_struct(self) -> _Mask:
+        return _Mask(_ptr(self.bits), _ptr(self.cnt), _ptr(self.idx), _ptr(self.cnt_t),
+                     _ptr(self.idx_t), _ptr(self.work))
+
+    @staticmethod
+    def empty(B: int, H: int, S: int, device, transpose: bool = True) -> "Mask":
+        nb = num_blocks(S)
+        W, npairs = -(-nb // 32), -(-nb // 2)
+        i32 = dict(dtype=torch.int32, device=device)
+        return Mask(bits=torch.empty(B, H, nb, W, **i32), cnt=torch.empty(B, H, nb, **i32),
+                    idx=torch.empty(B, H, nb, nb, **i32), work=torch.empty(B * H * npairs, 2, **i32),
+                    cnt_t=torch.empty(B, H, nb, **i32) if transpose else None,
+                    idx_t=torch.empty(B, H, nb, nb, **i32) if transpose else None)
+
+    def dense(self) -> torch.Tensor:
+        """bool [B, H, nb, nb] view of the bitmask (host-side convenience)."""
+        nb = self.cnt.shape[-1]
+        b = self.bits.to(torch.int64) & 0xFFFFFFFF
+        shifts = torch.arange(32, device=b.device)
+        m = ((b[..., None] >> shifts) & 1).bool()
+        return m.flatten(-2)[..., :nb]
+
+
+def workspace_size(q_shape, dtype=torch.bfloat16, want_bwd: bool = False) -> int:
+    B, H, S, D = q_shape
+    sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    n = lib().nabla_workspace_size(ctypes.byref(sh), int(want_bwd))
+    if n == 0:
+        raise NablaError(f"invalid shape {tuple(q_shape)}")
+    return n
+
+
+def workspace(q: torch.Tensor, want_bwd: bool = False) -> torch.Tensor:
+    n = workspace_size(tuple(q.shape), q.dtype, want_bwd)
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def build_mask(q: torch.Tensor, k: torch.Tensor, thr: float, sta_coords: torch.Tensor | None = None,
+               sta_window: tuple | None = None, out: Mask | None = None, ws: torch.Tensor | None = None,
+               transpose: bool = True) -> Mask:
+    """NABLA mask (Algorithm 1, plus the STA union when sta_coords/sta_window are given)."""
+    sh = _shape_of(q)
+    _same(q, k)
+    out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
+    ws = ws if ws is not None else workspace(q)
+    sta = None
+    if sta_coords is not None:
+        if sta_window is None:
+            raise NablaError("sta_window is required with sta_coords")
+        if sta_coords.dtype != torch.int32 or not sta_coords.is_cuda or not sta_coords.is_contiguous():
+            raise NablaError("sta_coords must be a contiguous int32 CUDA tensor [nb, 3]")
+        sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    ms = out.as_struct()
+    _check(lib().nabla_build_mask(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), ctypes.c_float(thr),
+                                  ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
+                                  ws.data_ptr(), ws.numel(), _stream()), "nabla_build_mask")
+    return out
+
+
+def mask_from_bits(bits: torch.Tensor, q_shape, dtype=torch.bfloat16, out: Mask | None = None,
+                   ws: torch.Tensor | None = None, transpose: bool = True) -> Mask:
+    """Index lists and work list for an externally supplied bitmask [B, H, nb, W]."""
+    B, H, S, D = q_shape
+    sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    bits = bits.to(torch.int32).contiguous()
+    out = out or Mask.empty(B, H, S, bits.device, transpose)
+    out.bits = bits
+    if ws is None:
+        ws = torch.empty(workspace_size(q_shape, dtype), dtype=torch.uint8, device=bits.device)
+    ms = out.as_struct()
+    _check(lib().nabla_mask_from_bits(ctypes.byref(sh), bits.data_ptr(), ctypes.byref(ms),
+                                      ws.data_ptr(), ws.numel(), _stream()), "nabla_mask_from_bits")
+    return out
+
+
+def attn_fwd(q, k, v, mask: Mask, o=None, lse=None, ws=None):
+    """Block-sparse attention forward; returns (o, lse)."""
+    sh = _shape_of(q)
+    _same(q, k, v)
+    o = o if o is not None else torch.empty_like(q)
+    lse = lse if lse is not None else torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ws = ws if ws is not None else workspace(q)
+    ms = mask.as_struct()
+    _check(lib().nabla_attn_fwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                ctypes.byref(ms), o.data_ptr(), lse.data_ptr(), ws.data_ptr(),
+                                ws.numel(), _stream()), "nabla_attn_fwd")
+    return o, lse
+
+
+def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None):
+    """Backward of attn_fwd under the same mask; returns (dq, dk, dv)."""
+    sh = _shape_of(q)
+    _same(q, k, v, o, do)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = ws if ws is not None else workspace(q, want_bwd=True)
+    ms = mask.as_struct()
+    _check(lib().nabla_attn_bwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                o.data_ptr(), do.data_ptr(), lse.data_ptr(), ctypes.byref(ms),
+                                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                ws.numel(), _stream()), "nabla_attn_bwd")
+    return dq, dk, dv
+
+
+def workspace_status(ws: torch.Tensor) -> int:
+    """Device status word of a workspace (0 = ok, 4 = a bounded wait ran out)."""
+    out = ctypes.c_int32(-1)
+    _check(lib().nabla_workspace_status(ws.data_ptr(), ctypes.byref(out), _stream()),
+           "nabla_workspace_status")
+    return out.value
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().nabla_set_wait_limit_ns(int(ns))

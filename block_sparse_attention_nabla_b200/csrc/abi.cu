@@ -1,0 +1,249 @@
+// extern "C" entry points of libnabla.so: argument validation, workspace
+// layout, kernel dispatch and error reporting.  Declarations and the contract
+// of every call are in include/nabla.h.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "internal.cuh"
+
+namespace nabla {
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_wait_limit_ns{0};
+
+nabla_status fail(nabla_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+nabla_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NABLA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+nabla_status check_shape(const nabla_shape* s) {
+  if (!s) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->H < 1 || s->S < 1 || s->D < 1)
+    return fail(NABLA_ERR_INVALID_ARG, "B, H, S, D must be >= 1 (got %d, %d, %d, %d)", s->B, s->H,
+                s->S, s->D);
+  if (s->block != kBlock)
+    return fail(NABLA_ERR_UNSUPPORTED, "block must be %d (got %d)", kBlock, s->block);
+  if (s->dtype != NABLA_BF16 && s->dtype != NABLA_FP32)
+    return fail(NABLA_ERR_INVALID_ARG, "dtype must be NABLA_BF16 or NABLA_FP32 (got %d)", s->dtype);
+  if (s->D != 64 && s->D != 128)
+    return fail(NABLA_ERR_UNSUPPORTED, "head dimension D must be 64 or 128 (got %d)", s->D);
+  const long long nb = (s->S + kBlock - 1) / kBlock;
+  if (nb > kMaxBlocks)
+    return fail(NABLA_ERR_UNSUPPORTED, "S = %d gives %lld blocks; at most %d are supported", s->S,
+                nb, kMaxBlocks);
+  if ((long long)s->B * s->H > (1ll << 30))
+    return fail(NABLA_ERR_UNSUPPORTED, "B * H too large");
+  return NABLA_OK;
+}
+
+nabla_status check_tensor(const void* p, const char* name) {
+  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 16)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return NABLA_OK;
+}
+
+nabla_status check_i32(const void* p, const char* name) {
+  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 4)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);
+  return NABLA_OK;
+}
+
+nabla_status check_ws(const Dims& d, bool bwd, const void* ws, size_t bytes) {
+  const size_t need = ws_layout(d, bwd).total;
+  if (!ws) return fail(NABLA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (!aligned(ws, 256)) return fail(NABLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (bytes < need)
+    return fail(NABLA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", bytes, need);
+  return NABLA_OK;
+}
+
+#define NABLA_TRY(expr)                   \
+  do {                                    \
+    nabla_status _s = (expr);             \
+    if (_s != NABLA_OK) return _s;        \
+  } while (0)
+
+#define NABLA_CUDA(expr, what)                      \
+  do {                                              \
+    cudaError_t _e = (expr);                        \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+// Builds cnt / idx is done by the caller; this adds the transposed lists and
+// the work list, which both derive from the bitmask.
+nabla_status emit_derived(const Dims& d, const uint32_t* bits, const nabla_mask* out,
+                          cudaStream_t st) {
+  if (out->cnt_t || out->idx_t) {
+    NABLA_TRY(check_i32(out->cnt_t, "mask.cnt_t"));
+    NABLA_TRY(check_i32(out->idx_t, "mask.idx_t"));
+    NABLA_CUDA(launch_transpose_lists(d, bits, out->cnt_t, out->idx_t, st), "transpose lists");
+  }
+  NABLA_CUDA(launch_work_list(d, bits, out->work, st), "work list");
+  return NABLA_OK;
+}
+
+nabla_status check_mask_out(const nabla_mask* m, bool need_bits) {
+  if (!m) return fail(NABLA_ERR_INVALID_ARG, "mask is NULL");
+  if (need_bits) NABLA_TRY(check_i32(m->bits, "mask.bits"));
+  NABLA_TRY(check_i32(m->cnt, "mask.cnt"));
+  NABLA_TRY(check_i32(m->idx, "mask.idx"));
+  NABLA_TRY(check_i32(m->work, "mask.work"));
+  if ((m->cnt_t == nullptr) != (m->idx_t == nullptr))
+    return fail(NABLA_ERR_INVALID_ARG, "mask.cnt_t and mask.idx_t must both be set or both NULL");
+  return NABLA_OK;
+}
+
+nabla_status reset_status(void* ws, cudaStream_t st) {
+  NABLA_CUDA(cudaMemsetAsync(ws, 0, 256, st), "clear workspace header");
+  return NABLA_OK;
+}
+
+}  // namespace
+
+uint64_t wait_limit_ns() {
+  const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v ? v : 2000000000ull;
+}
+
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" {
+
+int32_t nabla_abi_version(void) { return NABLA_ABI_VERSION; }
+
+const char* nabla_last_error(void) { return g_last_error.c_str(); }
+
+void nabla_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns, std::memory_order_relaxed); }
+
+size_t nabla_workspace_size(const nabla_shape* shape, int32_t want_bwd) {
+  if (check_shape(shape) != NABLA_OK) return 0;
+  return ws_layout(make_dims(*shape), want_bwd != 0).total;
+}
+
+nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const void* k, float thr,
+                              const nabla_sta* sta, const nabla_mask* out, void* workspace,
+                              size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_tensor(q, "q"));
+  NABLA_TRY(check_tensor(k, "k"));
+  if (!(thr > 0.f && thr <= 1.f))
+    return fail(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1] (got %g)", (double)thr);
+  if (sta && sta->block_coords) {
+    NABLA_TRY(check_i32(sta->block_coords, "sta.block_coords"));
+    if (sta->wT < 1 || sta->wH < 1 || sta->wW < 1)
+      return fail(NABLA_ERR_INVALID_ARG, "STA window sizes must be >= 1 (got %d, %d, %d)", sta->wT,
+                  sta->wH, sta->wW);
+  }
+  NABLA_TRY(check_mask_out(out, true));
+  NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsLayout L = ws_layout(d, false);
+  char* ws = (char*)workspace;
+  float* qa = (float*)(ws + L.qa);
+  float* ka = (float*)(ws + L.ka);
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_pool(d, q, k, qa, ka, st), "pooling kernel");
+  NABLA_CUDA(launch_select(d, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st), "select kernel");
+  return emit_derived(d, out->bits, out, st);
+}
+
+nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits,
+                                  const nabla_mask* out, void* workspace, size_t workspace_bytes,
+                                  nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_i32(bits, "bits"));
+  NABLA_TRY(check_mask_out(out, false));
+  NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_lists_from_bits(d, bits, out->cnt, out->idx, st), "lists kernel");
+  return emit_derived(d, bits, out, st);
+}
+
+nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                            const nabla_mask* mask, void* o, float* lse, void* workspace,
+                            size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_tensor(q, "q"));
+  NABLA_TRY(check_tensor(k, "k"));
+  NABLA_TRY(check_tensor(v, "v"));
+  NABLA_TRY(check_tensor(o, "o"));
+  if (lse && !aligned(lse, 4)) return fail(NABLA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  NABLA_TRY(check_mask_out(mask, false));
+  NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_TRY(reset_status(workspace, st));
+  if (d.dtype == NABLA_BF16)
+    NABLA_CUDA(launch_attn_fwd_tc(d, q, k, v, mask->cnt, mask->idx, mask->work, o, lse,
+                                  (int32_t*)workspace, st),
+               "tensor-core attention forward");
+  else
+    NABLA_CUDA(launch_attn_fwd_simt(d, q, k, v, mask->cnt, mask->idx, o, lse, st),
+               "fp32 attention forward");
+  return NABLA_OK;
+}
+
+nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                            const void* o, const void* dout, const float* lse,
+                            const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_tensor(q, "q"));
+  NABLA_TRY(check_tensor(k, "k"));
+  NABLA_TRY(check_tensor(v, "v"));
+  NABLA_TRY(check_tensor(o, "o"));
+  NABLA_TRY(check_tensor(dout, "dout"));
+  NABLA_TRY(check_tensor(dq, "dq"));
+  NABLA_TRY(check_tensor(dk, "dk"));
+  NABLA_TRY(check_tensor(dv, "dv"));
+  NABLA_TRY(check_i32(lse, "lse"));
+  NABLA_TRY(check_mask_out(mask, false));
+  if (!mask->cnt_t) return fail(NABLA_ERR_INVALID_ARG, "backward needs mask.cnt_t and mask.idx_t");
+  NABLA_TRY(check_ws(d, true, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsLayout L = ws_layout(d, true);
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
+                                  mask->idx_t, (float*)((char*)workspace + L.delta), dq, dk, dv, st),
+             "attention backward");
+  return NABLA_OK;
+}
+
+nabla_status nabla_workspace_status(const void* workspace, int32_t* host_status,
+                                    nabla_stream_t stream) {
+  g_last_error.clear();
+  if (!workspace || !host_status)
+    return fail(NABLA_ERR_INVALID_ARG, "workspace and host_status must not be NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_CUDA(cudaMemcpyAsync(host_status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, st),
+             "read status word");
+  NABLA_CUDA(cudaStreamSynchronize(st), "synchronise stream");
+  return NABLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// Internal declarations shared by the translation units of libnabla.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nabla.h"
+
+namespace nabla {
+
+constexpr int kBlock = 64;         // N of Algorithm 1: tokens per block
+constexpr int kMaxBlocks = 8192;   // nb limit (S <= 524,288); keeps per-row state on chip
+
+// Derived sizes of one problem.
+struct Dims {
+  int B, H, S, D, nb, W, npairs, dtype;
+  long long BH() const { return (long long)B * H; }
+};
+
+inline Dims make_dims(const nabla_shape& s) {
+  Dims d;
+  d.B = s.B; d.H = s.H; d.S = s.S; d.D = s.D; d.dtype = s.dtype;
+  d.nb = (s.S + kBlock - 1) / kBlock;
+  d.W = (d.nb + 31) / 32;
+  d.npairs = (d.nb + 1) / 2;
+  return d;
+}
+
+// Workspace layout: a 256-byte header (status word, scheduler counters), then
+// the pooled Qa / Ka (fp32 [B, H, nb, D]) and, for the backward, the per-row
+// Delta = rowsum(dO * O) (fp32 [B, H, S]).
+struct WsLayout {
+  size_t header = 0;
+  size_t qa = 0, ka = 0, delta = 0;
+  size_t total = 0;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
+  WsLayout w;
+  size_t off = 256;
+  size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(float);
+  w.qa = off; off = align256(off + pooled);
+  w.ka = off; off = align256(off + pooled);
+  if (want_bwd) { w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float)); }
+  w.total = off;
+  return w;
+}
+
+// Header words (int32 index into the workspace).
+enum : int { kWsStatus = 0, kWsTileCounter = 1 };
+
+uint64_t wait_limit_ns();
+
+// ---------------------------------------------------------------- launchers
+// Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
+
+cudaError_t launch_pool(const Dims& d, const void* q, const void* k, float* qa, float* ka,
+                        cudaStream_t st);
+cudaError_t launch_select(const Dims& d, const float* qa, const float* ka, float thr,
+                          const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                          cudaStream_t st);
+cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
+                                   int32_t* idx, cudaStream_t st);
+cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,
+                                   int32_t* idx_t, cudaStream_t st);
+cudaError_t launch_work_list(const Dims& d, const uint32_t* bits, int32_t* work, cudaStream_t st);
+
+cudaError_t launch_attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v,
+                                 const int32_t* cnt, const int32_t* idx, void* o, float* lse,
+                                 cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
+                                 const void* o, const void* dout, const float* lse,
+                                 const int32_t* cnt, const int32_t* idx, const int32_t* cnt_t,
+                                 const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
+                                 cudaStream_t st);
+cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
+                               const int32_t* cnt, const int32_t* idx, const int32_t* work,
+                               void* o, float* lse, int32_t* ws_header, cudaStream_t st);
+
+}  // namespace nabla

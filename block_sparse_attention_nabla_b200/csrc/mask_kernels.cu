@@ -1,0 +1,469 @@
+// Mask builder kernels: Algorithm 1 "NABLA Sparse Mask Generation" of
+// "∇NABLA: Neighborhood Adaptive Block-Level Attention" (§3.1.2), the STA
+// union of §3.1.3, and the index structures the attention kernels walk.
+//
+//   pool_kernel        block averaging of Q and K (reads Q and K once; the
+//                      HBM-bound part of the builder)
+//   select_kernel      reduced scores Qa Ka^T / sqrt(D), row softmax, CDF
+//                      binarisation, STA OR, bitmask + compact index lists
+//   lists_kernel       bitmask -> compact index lists (external masks)
+//   transpose_kernel   per key block, the query blocks that attend to it
+//   work_kernel        per (b, h): query-block pairs sorted by cost
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.cuh"
+
+namespace nabla {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void add_chunk(const uint4& u, float (&acc)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __bfloat1622float2(h[e]);
+    acc[2 * e] += f.x;
+    acc[2 * e + 1] += f.y;
+  }
+}
+
+__device__ __forceinline__ void add_chunk(const uint4& u, float (&acc)[4]) {
+  acc[0] += __uint_as_float(u.x);
+  acc[1] += __uint_as_float(u.y);
+  acc[2] += __uint_as_float(u.z);
+  acc[3] += __uint_as_float(u.w);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// ------------------------------------------------------------------ pooling
+// One 64-token block of Q or K per loop iteration: 256 threads issue 16-byte
+// loads covering the block (64 rows x D), each thread sums its rows in fp32,
+// lanes holding the same columns are combined by shuffles, warps through
+// shared memory.  The tail block divides by its number of valid tokens.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                   float* __restrict__ qa, float* __restrict__ ka,
+                                                   int S, int nb, long long per_tensor) {
+  constexpr int VE = 16 / sizeof(T);  // elements per 16-byte chunk
+  constexpr int CH = D / VE;          // chunks per row (8, 16 or 32)
+  constexpr int RP = 256 / CH;        // rows covered per pass
+  constexpr int NP = kBlock / RP;     // passes per block
+  __shared__ float red[8][D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid % CH, r0 = tid / CH;
+  for (long long item = blockIdx.x; item < 2 * per_tensor; item += gridDim.x) {
+    const bool isk = item >= per_tensor;
+    const long long it = isk ? item - per_tensor : item;  // (b * H + h) * nb + i
+    const long long bh = it / nb;
+    const int i = (int)(it - bh * nb);
+    const T* src = (isk ? k : q) + (bh * S + (long long)i * kBlock) * D;
+    const int valid = min(kBlock, S - i * kBlock);
+    uint4 v[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const int r = r0 + p * RP;
+      v[p] = r < valid ? ld_stream(src + (long long)r * D + c * VE) : make_uint4(0, 0, 0, 0);
+    }
+    float acc[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) add_chunk(v[p], acc);
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[e] += __shfl_xor_sync(kFull, acc[e], off);
+    if (lane < CH)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) red[warp][lane * VE + e] = acc[e];
+    __syncthreads();
+    if (tid < D) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[w][tid];
+      (isk ? ka : qa)[it * D + tid] = s / (float)valid;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------ index emission
+// Writes one mask row given, for t = 0 .. W-1, the kept flag of block
+// j = 32 t + lane.  Indices come out in ascending order.
+struct RowOut {
+  uint32_t* bits;  // row's W words (may be null)
+  int32_t* idx;    // row's nb slots
+  int32_t* cnt;    // row's count
+};
+
+// ------------------------------------------------------------ score + select
+// One CTA handles R query blocks of one (b, h).
+//   phase 1: L[r][j] = (Qa_r . Ka_j) * (1/sqrt(D)) in fp32, staged in shared
+//            memory (the map is never written to HBM);
+//   phase 2: one warp per row: max, e_j = exp(L_j - max), s = sum e_j; the
+//            kept set is {j : sum of e over entries above j <= thr * s},
+//            found as the smallest bit pattern u of a positive float with
+//            sum_{e_k > u} e_k <= thr * s (binary search over the float bits;
+//            positive floats order like their bit patterns); keep e_j >= u.
+//            That is Algorithm 1's ascending cumulative sum compared with
+//            1 - thr, expressed through the mass above each entry.
+//   then OR the STA window and emit bits / cnt / idx.
+template <int R, int D>
+__global__ void __launch_bounds__(256) select_kernel(
+    const float* __restrict__ qa, const float* __restrict__ ka, int nb, int W, int ldl, float thr,
+    float scale, const int32_t* __restrict__ coords, int hT, int hH, int hW,
+    uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
+  extern __shared__ float4 smem4[];
+  constexpr int LD = D + 4;  // padded Qa/Ka row: LD / 4 is odd -> conflict-free float4 rows
+  constexpr int KC = 64;     // Ka rows per chunk
+  constexpr int RG = R / 2;  // row pairs
+  constexpr int CT = 256 / RG;
+  constexpr int CPT = KC / CT;
+  float* Ls = reinterpret_cast<float*>(smem4);
+  float* Qs = Ls + R * ldl;
+  float* Ks = Qs + R * LD;
+  int* Ct = reinterpret_cast<int*>(Ks + KC * LD);
+  int* Cy = Ct + nb;
+  int* Cx = Cy + nb;
+  const bool use_sta = coords != nullptr;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long bh = blockIdx.y;
+  const int row0 = blockIdx.x * R;
+  const float* qa_h = qa + bh * nb * D;
+  const float* ka_h = ka + bh * nb * D;
+
+  for (int e = tid; e < R * (D / 4); e += 256) {
+    const int r = e / (D / 4), c4 = e % (D / 4);
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row0 + r < nb) val = *reinterpret_cast<const float4*>(qa_h + (long long)(row0 + r) * D + c4 * 4);
+    *reinterpret_cast<float4*>(Qs + r * LD + c4 * 4) = val;
+  }
+  if (use_sta)
+    for (int j = tid; j < nb; j += 256) {
+      Ct[j] = coords[3 * j];
+      Cy[j] = coords[3 * j + 1];
+      Cx[j] = coords[3 * j + 2];
+    }
+
+  const int tr = tid / CT, tc = tid % CT;
+  for (int c0 = 0; c0 < nb; c0 += KC) {
+    __syncthreads();
+    for (int e = tid; e < KC * (D / 4); e += 256) {
+      const int r = e / (D / 4), c4 = e % (D / 4);
+      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + r < nb) val = *reinterpret_cast<const float4*>(ka_h + (long long)(c0 + r) * D + c4 * 4);
+      *reinterpret_cast<float4*>(Ks + r * LD + c4 * 4) = val;
+    }
+    __syncthreads();
+    float acc0[CPT], acc1[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) acc0[j] = acc1[j] = 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < D; kk += 4) {
+      const float4 a0 = *reinterpret_cast<const float4*>(Qs + (2 * tr) * LD + kk);
+      const float4 a1 = *reinterpret_cast<const float4*>(Qs + (2 * tr + 1) * LD + kk);
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const float4 b = *reinterpret_cast<const float4*>(Ks + (tc + CT * j) * LD + kk);
+        acc0[j] = fmaf(a0.x, b.x, acc0[j]);
+        acc0[j] = fmaf(a0.y, b.y, acc0[j]);
+        acc0[j] = fmaf(a0.z, b.z, acc0[j]);
+        acc0[j] = fmaf(a0.w, b.w, acc0[j]);
+        acc1[j] = fmaf(a1.x, b.x, acc1[j]);
+        acc1[j] = fmaf(a1.y, b.y, acc1[j]);
+        acc1[j] = fmaf(a1.z, b.z, acc1[j]);
+        acc1[j] = fmaf(a1.w, b.w, acc1[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int col = c0 + tc + CT * j;
+      if (col < nb) {
+        Ls[(2 * tr) * ldl + col] = acc0[j] * scale;
+        Ls[(2 * tr + 1) * ldl + col] = acc1[j] * scale;
+      }
+    }
+  }
+  __syncthreads();
+
+  for (int r = warp; r < R; r += 8) {
+    const int row = row0 + r;
+    if (row >= nb) break;
+    float* Lr = Ls + r * ldl;
+    float mx = -INFINITY;
+    for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, Lr[j]);
+    mx = warp_max(mx);
+    float s = 0.f;
+    for (int j = lane; j < nb; j += 32) {
+      const float e = expf(Lr[j] - mx);
+      Lr[j] = e;
+      s += e;
+    }
+    s = warp_sum(s);
+    const float limit = thr * s;
+    // e_max = exp(0) = 1, so every entry's bit pattern is <= 0x3F800000 and
+    // the mass strictly above 0x3F800001 is 0 <= limit.
+    uint32_t lo = 0u, hi = 0x3F800001u;
+    while (lo < hi) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      float f = 0.f;
+      for (int j = lane; j < nb; j += 32) {
+        const float e = Lr[j];
+        f += __float_as_uint(e) > mid ? e : 0.f;
+      }
+      f = warp_sum(f);
+      if (f <= limit) hi = mid; else lo = mid + 1u;
+    }
+    const long long grow = bh * nb + row;
+    uint32_t* brow = bits + grow * W;
+    int32_t* irow = idx + grow * nb;
+    int running = 0;
+    const int ti = use_sta ? Ct[row] : 0, yi = use_sta ? Cy[row] : 0, xi = use_sta ? Cx[row] : 0;
+    for (int t = 0; t < W; ++t) {
+      const int j = t * 32 + lane;
+      bool keep = false;
+      if (j < nb) {
+        keep = __float_as_uint(Lr[j]) >= lo;
+        if (use_sta && !keep)
+          keep = abs(Ct[j] - ti) <= hT && abs(Cy[j] - yi) <= hH && abs(Cx[j] - xi) <= hW;
+      }
+      const uint32_t word = __ballot_sync(kFull, keep);
+      if (lane == 0) brow[t] = word;
+      if (keep) irow[running + __popc(word & lanemask_lt())] = j;
+      running += __popc(word);
+    }
+    if (lane == 0) cnt[grow] = running;
+  }
+}
+
+// ------------------------------------------------------ lists from a bitmask
+__global__ void __launch_bounds__(256) lists_kernel(const uint32_t* __restrict__ bits, long long rows,
+                                                    int nb, int W, int32_t* __restrict__ cnt,
+                                                    int32_t* __restrict__ idx) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint32_t* brow = bits + row * W;
+  int32_t* irow = idx + row * nb;
+  int running = 0;
+  for (int t = 0; t < W; ++t) {
+    const int j = t * 32 + lane;
+    uint32_t word = brow[t];
+    if (t == W - 1 && (nb & 31)) word &= (1u << (nb & 31)) - 1u;
+    if ((word >> lane) & 1u) irow[running + __popc(word & lanemask_lt())] = j;
+    running += __popc(word);
+  }
+  if (lane == 0) cnt[row] = running;
+}
+
+// --------------------------------------------------- transposed (CSC) lists
+__global__ void __launch_bounds__(256) transpose_kernel(const uint32_t* __restrict__ bits,
+                                                        long long cols, int nb, int W,
+                                                        int32_t* __restrict__ cnt_t,
+                                                        int32_t* __restrict__ idx_t) {
+  const long long gcol = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gcol >= cols) return;
+  const long long bh = gcol / nb;
+  const int j = (int)(gcol - bh * nb);
+  const uint32_t* bm = bits + bh * nb * W + (j >> 5);
+  int32_t* irow = idx_t + gcol * nb;
+  int running = 0;
+  for (int i0 = 0; i0 < nb; i0 += 32) {
+    const int i = i0 + lane;
+    const bool keep = i < nb && ((bm[(long long)i * W] >> (j & 31)) & 1u);
+    const uint32_t word = __ballot_sync(kFull, keep);
+    if (keep) irow[running + __popc(word & lanemask_lt())] = i;
+    running += __popc(word);
+  }
+  if (lane == 0) cnt_t[gcol] = running;
+}
+
+// ---------------------------------------------------------------- work list
+// One CTA per (b, h): cost of each query-block pair = popcount of the union of
+// its two rows; bitonic sort of (nb - cost, pair) ascending = cost descending,
+// pair ascending among equal costs.
+__global__ void __launch_bounds__(1024) work_kernel(const uint32_t* __restrict__ bits, int nb, int W,
+                                                    int npairs, int p2, int32_t* __restrict__ work) {
+  extern __shared__ unsigned long long keys[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const long long bh = blockIdx.x;
+  const uint32_t* rb = bits + bh * nb * W;
+  for (int p = warp; p < npairs; p += nwarp) {
+    int c = 0;
+    const bool has_b = 2 * p + 1 < nb;
+    for (int w = lane; w < W; w += 32) {
+      const uint32_t a = rb[(long long)(2 * p) * W + w];
+      const uint32_t b = has_b ? rb[(long long)(2 * p + 1) * W + w] : 0u;
+      c += __popc(a | b);
+    }
+    c = warp_sum_i(c);
+    if (lane == 0) keys[p] = ((unsigned long long)(nb - c) << 32) | (unsigned)p;
+  }
+  for (int p = npairs + tid; p < p2; p += blockDim.x) keys[p] = ~0ull;
+  __syncthreads();
+  for (int kk = 2; kk <= p2; kk <<= 1) {
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < p2; i += blockDim.x) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], b = keys[ixj];
+          const bool up = (i & kk) == 0;
+          if ((a > b) == up) { keys[i] = b; keys[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int r = tid; r < npairs; r += blockDim.x) {
+    const unsigned long long key = keys[r];
+    const int p = (int)(key & 0xffffffffu);
+    const int cost = nb - (int)(key >> 32);
+    work[(bh * npairs + r) * 2] = (int32_t)(bh * npairs + p);
+    work[(bh * npairs + r) * 2 + 1] = cost;
+  }
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern k, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+constexpr size_t kSmemLimit = 227 * 1024;
+
+template <int R, int D>
+size_t select_smem(int nb, int ldl) {
+  return sizeof(float) * ((size_t)R * ldl + (size_t)R * (D + 4) + 64 * (D + 4)) + 3 * sizeof(int) * nb;
+}
+
+template <int R, int D>
+cudaError_t run_select(const Dims& d, const float* qa, const float* ka, float thr,
+                       const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                       cudaStream_t st, int ldl) {
+  const size_t smem = select_smem<R, D>(d.nb, ldl);
+  auto kern = select_kernel<R, D>;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const bool use_sta = sta && sta->block_coords;
+  dim3 grid((d.nb + R - 1) / R, (unsigned)d.BH());
+  kern<<<grid, 256, smem, st>>>(qa, ka, d.nb, d.W, ldl, thr, 1.0f / sqrtf((float)d.D),
+                                use_sta ? sta->block_coords : nullptr, use_sta ? sta->wT / 2 : 0,
+                                use_sta ? sta->wH / 2 : 0, use_sta ? sta->wW / 2 : 0, bits, cnt, idx);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t select_d(const Dims& d, const float* qa, const float* ka, float thr,
+                     const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                     cudaStream_t st) {
+  const int ldl = (d.nb + 3) & ~3;
+  if (select_smem<32, D>(d.nb, ldl) <= kSmemLimit)
+    return run_select<32, D>(d, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
+  if (select_smem<16, D>(d.nb, ldl) <= kSmemLimit)
+    return run_select<16, D>(d, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
+  if (select_smem<8, D>(d.nb, ldl) <= kSmemLimit)
+    return run_select<8, D>(d, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Dims& d, const void* q, const void* k, float* qa, float* ka,
+                        cudaStream_t st) {
+  const long long per = d.BH() * d.nb;
+  const long long items = 2 * per;
+  const int grid = (int)std::min<long long>(items, (long long)num_sms() * 8);
+  if (d.dtype == NABLA_BF16) {
+    if (d.D == 128)
+      pool_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, d.S, d.nb, per);
+    else
+      pool_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, d.S, d.nb, per);
+  } else {
+    if (d.D == 128)
+      pool_kernel<float, 128><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, d.S, d.nb, per);
+    else
+      pool_kernel<float, 64><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, d.S, d.nb, per);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Dims& d, const float* qa, const float* ka, float thr,
+                          const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                          cudaStream_t st) {
+  if (d.D == 128) return select_d<128>(d, qa, ka, thr, sta, bits, cnt, idx, st);
+  return select_d<64>(d, qa, ka, thr, sta, bits, cnt, idx, st);
+}
+
+cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt, int32_t* idx,
+                                   cudaStream_t st) {
+  const long long rows = d.BH() * d.nb;
+  const long long blocks = (rows * 32 + 255) / 256;
+  lists_kernel<<<(unsigned)blocks, 256, 0, st>>>(bits, rows, d.nb, d.W, cnt, idx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,
+                                   int32_t* idx_t, cudaStream_t st) {
+  const long long cols = d.BH() * d.nb;
+  const long long blocks = (cols * 32 + 255) / 256;
+  transpose_kernel<<<(unsigned)blocks, 256, 0, st>>>(bits, cols, d.nb, d.W, cnt_t, idx_t);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_work_list(const Dims& d, const uint32_t* bits, int32_t* work, cudaStream_t st) {
+  int p2 = 1;
+  while (p2 < d.npairs) p2 <<= 1;
+  const size_t smem = sizeof(unsigned long long) * p2;
+  cudaError_t e = set_smem(work_kernel, smem);
+  if (e != cudaSuccess) return e;
+  work_kernel<<<(unsigned)d.BH(), 1024, smem, st>>>(bits, d.nb, d.W, d.npairs, p2, work);
+  return cudaGetLastError();
+}
+
+}  // namespace nabla

@@ -1,0 +1,179 @@
+/*
+ * nabla.h - C ABI of the NABLA block-sparse attention library for B200 (sm_100a).
+ *
+ * The library implements the data-parallel hot path of NABLA
+ * ("∇NABLA: Neighborhood Adaptive Block-Level Attention", arXiv 2507.13546v1):
+ *
+ *   1. the adaptive mask builder of §3.1.2, Algorithm 1 "NABLA Sparse Mask
+ *      Generation": average-pool Q and K over blocks of N = 64 tokens, form the
+ *      reduced attention map softmax(Qa Ka^T / sqrt(D)) per head, sort each row,
+ *      accumulate, keep the entries whose cumulative value reaches 1 - thr and
+ *      restore the original order; optionally OR-ed (§3.1.3) with the
+ *      sliding-tile (STA) window mask of §2.2;
+ *   2. block-sparse attention over the kept 64 x 64 tiles: Eq. 4 of §2.2,
+ *      softmax(Q K^T / sqrt(D) + M) V with M in {-inf, 0}, and its backward.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors Q, K, V, O, dO, dQ, dK, dV are dense, contiguous [B, H, S, D] in
+ *   the dtype named by the shape (bf16 or fp32), in device memory, with a
+ *   16-byte aligned base address.  S may be any value >= 1: the last 64-token
+ *   block may be partial (its pooled mean averages its valid tokens and its
+ *   missing keys are excluded from attention).
+ * - nb = ceil(S / 64) blocks per sequence; W = ceil(nb / 32) bitmask words per
+ *   mask row; npairs = ceil(nb / 2) query-block pairs per (b, h).
+ * - Every pointer argument is a device pointer unless stated otherwise.  The
+ *   caller owns every buffer, including the workspace; the library allocates no
+ *   device memory and keeps no global device state.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream).  A returned NABLA_OK means the arguments were valid and the work
+ *   was enqueued; device-side failures (a bounded wait that ran out) are
+ *   reported in the workspace status word, read with nabla_workspace_status().
+ * - On any error the call enqueues nothing (argument errors) or stops enqueuing
+ *   (launch errors), returns a status != NABLA_OK and records a message that
+ *   nabla_last_error() returns in the calling thread.
+ */
+#ifndef NABLA_H
+#define NABLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NABLA_API __attribute__((visibility("default")))
+#else
+#define NABLA_API
+#endif
+
+#define NABLA_ABI_VERSION 1
+#define NABLA_BLOCK 64
+
+typedef struct CUstream_st* nabla_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NABLA_OK = 0,
+  NABLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, thr outside (0, 1] */
+  NABLA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. D = 96) */
+  NABLA_ERR_CUDA = 3,         /* a CUDA runtime call failed; message in nabla_last_error() */
+  NABLA_ERR_TIMEOUT = 4,      /* device status only: a bounded wait inside a kernel ran out */
+  NABLA_ERR_WORKSPACE = 5     /* workspace pointer null or smaller than nabla_workspace_size() */
+} nabla_status;
+
+typedef enum { NABLA_BF16 = 0, NABLA_FP32 = 1 } nabla_dtype;
+
+/* Problem shape.  block must be 64 (N in Algorithm 1); D must be 64 or 128. */
+typedef struct {
+  int32_t B, H, S, D;
+  int32_t block;
+  int32_t dtype; /* nabla_dtype */
+} nabla_shape;
+
+/* Optional STA neighbourhood (§2.2, §3.1.3).  block_coords: device int32
+ * [nb][3], the (t, y, x) tile coordinate of every 64-token block (shared by
+ * all samples and heads).  Block j is visible from block i iff
+ * |t_i - t_j| <= wT / 2, |y_i - y_j| <= wH / 2 and |x_i - x_j| <= wW / 2
+ * (integer division; window centred on the query tile, cut at the grid edge).
+ * Window sizes are in tiles and must be >= 1. */
+typedef struct {
+  const int32_t* block_coords;
+  int32_t wT, wH, wW;
+} nabla_sta;
+
+/* Mask outputs (all device memory, written by the library).
+ *   bits  uint32 [B, H, nb, W]: bit (j % 32) of word j / 32 of row i is set
+ *         iff query block i attends to key block j.  Padding bits are zero.
+ *   cnt   int32 [B, H, nb]: number of kept key blocks of each query block.
+ *   idx   int32 [B, H, nb, nb]: row i holds its cnt[i] kept key-block indices
+ *         in ascending order; entries past cnt[i] are not written.
+ *   cnt_t, idx_t: the same lists transposed (per key block, the query blocks
+ *         that attend to it, ascending).  Needed only by nabla_attn_bwd; may be
+ *         NULL for forward-only use.
+ *   work  int32 [B * H * npairs][2]: the forward scheduler's work list, one
+ *         entry per pair of query blocks (2p, 2p + 1) of one (b, h):
+ *         { (b * H + h) * npairs + p, number of key blocks in the union of the
+ *         two rows }.  Entries are grouped by (b, h) in ascending order and
+ *         sorted by descending cost inside a group. */
+typedef struct {
+  uint32_t* bits;
+  int32_t* cnt;
+  int32_t* idx;
+  int32_t* cnt_t;
+  int32_t* idx_t;
+  int32_t* work;
+} nabla_mask;
+
+/* Bytes of device workspace the calls below need for `shape`.  want_bwd != 0
+ * adds what nabla_attn_bwd needs.  Returns 0 for an invalid shape. */
+NABLA_API size_t nabla_workspace_size(const nabla_shape* shape, int32_t want_bwd);
+
+/* Mask builder: Algorithm 1 of §3.1.2 plus the STA union of §3.1.3.
+ *   q, k   [B, H, S, D] in shape->dtype.
+ *   thr    binarisation threshold, 0 < thr <= 1 (thr = 1 keeps every block).
+ *          A row keeps block j iff the softmax mass of the entries ranked above
+ *          j (larger values) is <= thr; this is the ascending cumulative-sum
+ *          rule cvals >= 1 - thr of Algorithm 1 (entries tied with the cut-off
+ *          value are all kept).
+ *   sta    NULL or sta->block_coords NULL: no STA union.
+ *   out    bits, cnt, idx, work are required; cnt_t/idx_t are filled if not NULL.
+ * Pooling, scores and selection run in fp32 (the pooled vectors are fp32
+ * means of the inputs). */
+NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const void* k, float thr,
+                              const nabla_sta* sta, const nabla_mask* out, void* workspace,
+                              size_t workspace_bytes, nabla_stream_t stream);
+
+/* Builds cnt, idx, work (and cnt_t, idx_t if not NULL) of `out` from a
+ * caller-supplied bitmask `bits` [B, H, nb, W] (padding bits must be zero);
+ * out->bits is ignored.  Lets attention run under any externally computed
+ * block mask, e.g. a reference mask. */
+NABLA_API nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits,
+                                  const nabla_mask* out, void* workspace, size_t workspace_bytes,
+                                  nabla_stream_t stream);
+
+/* Block-sparse attention forward, Eq. 4 of §2.2 with M = -inf outside the kept
+ * tiles of `mask` (cnt, idx and work are read) and outside the sequence.
+ *   o    [B, H, S, D] output, shape->dtype.
+ *   lse  float [B, H, S]: natural-log log-sum-exp of the scaled logits
+ *        (Q K^T / sqrt(D)) over the attended keys, needed by the backward.
+ *        May be NULL.  A row with no kept block gets o = 0, lse = -inf.
+ * bf16 runs on the tensor cores (tcgen05, fp32 accumulation in TMEM); fp32 runs
+ * in fp32 on the CUDA cores. */
+NABLA_API nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                            const nabla_mask* mask, void* o, float* lse, void* workspace,
+                            size_t workspace_bytes, nabla_stream_t stream);
+
+/* Backward of nabla_attn_fwd with the mask held constant (no gradient flows
+ * into the mask builder).  o and lse are the forward's outputs, dout the
+ * upstream gradient; mask needs cnt, idx, cnt_t and idx_t.  Writes dq, dk, dv
+ * [B, H, S, D] in shape->dtype.  The result is deterministic (no atomics). */
+NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                            const void* o, const void* dout, const float* lse,
+                            const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, nabla_stream_t stream);
+
+/* Reads the device status word of `workspace` into *host_status (a host
+ * pointer): NABLA_OK, or NABLA_ERR_TIMEOUT if a bounded wait inside a kernel of
+ * the most recent call on this workspace ran out.  Synchronises `stream`. */
+NABLA_API nabla_status nabla_workspace_status(const void* workspace, int32_t* host_status,
+                                    nabla_stream_t stream);
+
+/* Sets the time limit, in nanoseconds, of every bounded spin-wait in the
+ * kernels launched after this call by the calling process (0 restores the
+ * default of 2 s).  A wait that runs out makes its kernel stop cleanly and set
+ * NABLA_ERR_TIMEOUT in the workspace status word. */
+NABLA_API void nabla_set_wait_limit_ns(uint64_t ns);
+
+/* Message of the last error recorded in the calling thread ("" if none). */
+NABLA_API const char* nabla_last_error(void);
+
+/* NABLA_ABI_VERSION of the loaded library. */
+NABLA_API int32_t nabla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NABLA_H */

@@ -1,0 +1,136 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/nabla.h declares, and its host-side logic (workspace sizing, argument
+validation) behaves as documented.  Every call here fails validation before
+any CUDA call is made, so no GPU is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_nabla_b200 as nabla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nabla.h")
+
+OK, INVALID, UNSUPPORTED, CUDA, TIMEOUT, WORKSPACE = range(6)
+FAKE = 1 << 20          # a non-null, 256-byte aligned address never dereferenced here
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"NABLA_API\s+[\w\s\*]+?\b(nabla_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(nabla.LIB_PATH):
+        from block_sparse_attention_nabla_b200 import build
+        build.build()
+    return nabla.lib()
+
+
+def shape(B=1, H=2, S=1000, D=128, block=64, dtype=0):
+    return nabla._Shape(B, H, S, D, block, dtype)
+
+
+def mask_struct(**kw):
+    m = dict(bits=FAKE, cnt=FAKE, idx=FAKE, cnt_t=None, idx_t=None, work=FAKE)
+    m.update(kw)
+    return nabla._Mask(m["bits"], m["cnt"], m["idx"], m["cnt_t"], m["idx_t"], m["work"])
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) == 9
+    assert sorted(nabla.SYMBOLS) == names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_abi_version(L):
+    assert L.nabla_abi_version() == 1
+
+
+def test_workspace_size_formula(L):
+    def align(x):
+        return (x + 255) // 256 * 256
+    for (B, H, S, D) in [(1, 2, 4096, 64), (1, 40, 75600, 128), (2, 16, 16384, 128), (1, 1, 1, 64)]:
+        nb = -(-S // 64)
+        pooled = align(B * H * nb * D * 4)
+        fwd = 256 + 2 * pooled
+        assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 0) == fwd
+        assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 1) == fwd + align(B * H * S * 4)
+
+
+def test_workspace_size_rejects_bad_shapes(L):
+    assert L.nabla_workspace_size(None, 0) == 0
+    assert L.nabla_workspace_size(ctypes.byref(shape(D=96)), 0) == 0
+    assert L.nabla_workspace_size(ctypes.byref(shape(block=32)), 0) == 0
+    assert L.nabla_workspace_size(ctypes.byref(shape(S=0)), 0) == 0
+    assert L.nabla_workspace_size(ctypes.byref(shape(S=64 * 8192 + 1)), 0) == 0
+
+
+def _build(L, sh=None, q=FAKE, k=FAKE, thr=0.5, sta=None, m=None, ws=FAKE, ws_bytes=1 << 40):
+    sh = sh or shape()
+    m = m or mask_struct()
+    return L.nabla_build_mask(ctypes.byref(sh), q, k, ctypes.c_float(thr),
+                              ctypes.byref(sta) if sta is not None else None, ctypes.byref(m), ws,
+                              ws_bytes, None)
+
+
+def test_build_mask_argument_errors(L):
+    assert _build(L, thr=0.0) == INVALID
+    assert b"thr" in L.nabla_last_error()
+    assert _build(L, thr=1.5) == INVALID
+    assert _build(L, thr=float("nan")) == INVALID
+    assert _build(L, q=None) == INVALID
+    assert b"q is NULL" in L.nabla_last_error()
+    assert _build(L, k=FAKE + 8) == INVALID            # not 16-byte aligned
+    assert b"aligned" in L.nabla_last_error()
+    assert _build(L, sh=shape(D=96)) == UNSUPPORTED
+    assert _build(L, sh=shape(block=128)) == UNSUPPORTED
+    assert _build(L, sh=shape(dtype=7)) == INVALID
+    assert _build(L, sh=shape(S=-5)) == INVALID
+    assert _build(L, m=mask_struct(work=None)) == INVALID
+    assert _build(L, m=mask_struct(cnt_t=FAKE)) == INVALID     # cnt_t without idx_t
+    assert _build(L, sta=nabla._Sta(FAKE, 3, 0, 3)) == INVALID
+    assert b"STA" in L.nabla_last_error()
+    assert _build(L, ws=None) == WORKSPACE
+    assert _build(L, ws_bytes=100) == WORKSPACE
+    assert b"needed" in L.nabla_last_error()
+    assert _build(L, ws=FAKE + 16) == WORKSPACE         # workspace must be 256-byte aligned
+
+
+def test_attention_argument_errors(L):
+    sh, m = shape(), mask_struct()
+    fwd = lambda **kw: L.nabla_attn_fwd(ctypes.byref(kw.get("sh", sh)), kw.get("q", FAKE), FAKE, FAKE,
+                                        ctypes.byref(kw.get("m", m)), kw.get("o", FAKE),
+                                        kw.get("lse", FAKE), kw.get("ws", FAKE), kw.get("wsb", 1 << 40), None)
+    assert fwd(o=None) == INVALID
+    assert fwd(lse=FAKE + 2) == INVALID
+    assert fwd(sh=shape(D=32)) == UNSUPPORTED
+    assert fwd(wsb=10) == WORKSPACE
+    bwd = lambda **kw: L.nabla_attn_bwd(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        ctypes.byref(kw.get("m", m)), FAKE, FAKE, kw.get("dv", FAKE),
+                                        FAKE, kw.get("wsb", 1 << 40), None)
+    assert bwd() == INVALID                              # forward-only mask: no transposed lists
+    assert b"cnt_t" in L.nabla_last_error()
+    full = mask_struct(cnt_t=FAKE, idx_t=FAKE)
+    assert bwd(m=full, dv=None) == INVALID
+    assert bwd(m=full, wsb=1000) == WORKSPACE
+
+
+def test_mask_from_bits_and_status_argument_errors(L):
+    sh = shape()
+    assert L.nabla_mask_from_bits(ctypes.byref(sh), None, ctypes.byref(mask_struct()), FAKE, 1 << 40, None) == INVALID
+    assert L.nabla_mask_from_bits(ctypes.byref(sh), FAKE, ctypes.byref(mask_struct(idx=None)), FAKE, 1 << 40, None) == INVALID
+    assert L.nabla_workspace_status(None, None, None) == INVALID
+
+
+def test_last_error_is_per_call(L):
+    assert _build(L, thr=0.0) == INVALID
+    assert L.nabla_last_error() != b""
+    assert L.nabla_workspace_size(ctypes.byref(shape()), 0) > 0   # does not touch the message
+    assert _build(L, q=None) == INVALID
+    assert b"thr" not in L.nabla_last_error()

@@ -1,0 +1,175 @@
+"""GPU parity of block-sparse attention (Eq. 4 of "∇NABLA: Neighborhood
+Adaptive Block-Level Attention", §2.2, over the kept tiles of the NABLA mask)
+against the fp64 oracle, computed under the oracle's own mask.
+
+Bar: max-abs 2e-2 and mean-rel 5e-3 for bf16 outputs, 1e-4 (both metrics)
+for fp32.  bf16 gradients dQ, dK, dV: elementwise |x - ref| <= 2e-2 + 2^-8 |ref|
+and mean-rel 5e-3 (see gpu_util.GRAD_REL for why the absolute bar scales)."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_nabla_b200 as nabla
+import synth
+from oracle import nabla_oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd_parity(x, M, kind):
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    ws = nabla.workspace(q)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    O, LSE = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, kind, "O")
+    rows = np.isfinite(LSE)
+    assert np.abs(lse.cpu().numpy()[rows] - LSE[rows]).max() < (1e-3 if kind == "bf16" else 1e-5)
+    return o, lse, mask
+
+
+def test_fwd_tiny_fp32_workload():
+    w = synth.WORKLOADS[1]
+    x = synth.make_inputs(w)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], w.thresholds[0])
+    _fwd_parity(x, M, "fp32")
+
+
+@pytest.mark.parametrize("S,D", [(1000, 128), (414, 128), (1000, 64), (130, 64), (64, 128), (37, 128)])
+@pytest.mark.parametrize("thr", [0.5, 0.9, 1.0])
+def test_fwd_small_bf16(S, D, thr):
+    x = synth.make_random_qkv(2, 2, S, D, "bf16", seed=3 * S + D)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], thr)
+    _fwd_parity(x, M, "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_fwd_edge_masks(dtype):
+    # empty rows, a full row, only the ragged tail block, a random pattern
+    S, nb = 64 * 9 + 7, 10
+    x = synth.make_random_qkv(1, 2, S, 128, dtype, seed=11)
+    rng = np.random.default_rng(4)
+    M = rng.random((1, 2, nb, nb)) < 0.3
+    M[0, 0, 3] = False
+    M[0, 0, 4] = False            # both rows of pair 2 empty
+    M[0, 1, 5] = True
+    M[0, 1, 9] = False
+    M[0, 1, 9, 9] = True
+    M[0, 1, 0] = False
+    M[0, 1, 0, 9] = True          # row 0 only sees the tail block
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    o, lse = nabla.attn_fwd(q, k, v, mask)
+    torch.cuda.synchronize()
+    O, LSE = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, dtype, "O")
+    empty = np.zeros((1, 2, S), dtype=bool)
+    empty[0, 0, 3 * 64:5 * 64] = True
+    assert (o.float().cpu().numpy()[empty] == 0).all()
+    assert np.isneginf(lse.cpu().numpy()[empty]).all()
+
+
+@pytest.mark.parametrize("wid,heads", [(2, [0, 21, 39]), (3, [0, 17, 39])])
+def test_fwd_full_size_sampled_rows(wid, heads):
+    """Full-size forward (the benchmark's launch configuration) under the
+    oracle's mask, checked on sampled rows of three heads."""
+    w = synth.WORKLOADS[wid]
+    x = synth.make_inputs(w)
+    thr = w.thresholds[0]
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], thr)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    ws = nabla.workspace(q)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    rng = np.random.default_rng(wid)
+    S = w.S
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128, S - 1, S - 2, S - 17],
+                                     rng.integers(0, S, size=40)]))
+    for h in heads:
+        Or, Lr = orc.masked_attention_rows(x["q"], x["k"], x["v"], M, 0, h, rows)
+        gu.assert_close(o[0, h, rows], Or, "bf16", f"head {h}")
+        assert np.abs(lse[0, h, rows].cpu().numpy() - Lr).max() < 1e-3
+    assert torch.isfinite(o.float()).all()
+
+
+def test_fwd_uses_gpu_built_mask_end_to_end():
+    w = synth.WORKLOADS[2].scaled(H=4)
+    x = synth.make_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = nabla.build_mask(q, k, 0.8)
+    o, lse = nabla.attn_fwd(q, k, v, mask)
+    torch.cuda.synchronize()
+    G = orc.bits_to_mask(gu.gpu_bits(mask), w.nb)
+    rows = np.arange(0, w.S, 997)
+    for h in range(4):
+        Or, _ = orc.masked_attention_rows(x["q"], x["k"], x["v"], G, 0, h, rows)
+        gu.assert_close(o[0, h, rows], Or, "bf16", f"head {h}")
+
+
+# ---------------------------------------------------------------- backward
+
+def _bwd_parity(x, M, kind, heads=None):
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    o, lse = nabla.attn_fwd(q, k, v, mask)
+    ws = nabla.workspace(q, want_bwd=True)
+    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    for (b, h) in ([(b, h) for b in range(q.shape[0]) for h in range(q.shape[1])] if heads is None else heads):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        dQ, dK, dV = orc.masked_attention_bwd(x["q"][sl], x["k"][sl], x["v"][sl], x["do"][sl], M[sl])
+        gu.assert_close(dq[sl], dQ, kind, f"dQ b{b} h{h}", grad=True)
+        gu.assert_close(dk[sl], dK, kind, f"dK b{b} h{h}", grad=True)
+        gu.assert_close(dv[sl], dV, kind, f"dV b{b} h{h}", grad=True)
+
+
+def test_bwd_tiny_fp32():
+    w = synth.WORKLOADS[1].scaled(with_grad=True)
+    x = synth.make_inputs(w)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], w.thresholds[0])
+    _bwd_parity(x, M, "fp32")
+
+
+@pytest.mark.parametrize("S,D", [(1000, 128), (414, 64), (130, 128)])
+def test_bwd_small_bf16(S, D):
+    x = synth.make_random_qkv(1, 2, S, D, "bf16", seed=S, with_grad=True)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
+    _bwd_parity(x, M, "bf16")
+
+
+def test_bwd_pretraining_workload_two_heads():
+    w = synth.WORKLOADS[4]
+    x = synth.make_inputs(w)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], w.thresholds[0])
+    _bwd_parity(x, M, "bf16", heads=[(0, 0), (1, 15)])
+
+
+# ------------------------------------------------------ bounded waits
+
+def test_wait_limit_reports_timeout_and_context_survives():
+    """A wait limit far below the time a tile takes makes the forward kernel's
+    bounded waits run out: the kernel stops, reports NABLA_ERR_TIMEOUT in the
+    workspace status word, and the next call with the default limit works."""
+    x = synth.make_random_qkv(1, 4, 4096, 128, "bf16", seed=5)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 1.0)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    ws = nabla.workspace(q)
+    try:
+        nabla.set_wait_limit_ns(1)
+        nabla.attn_fwd(q, k, v, mask, ws=ws)
+        torch.cuda.synchronize()
+        assert nabla.workspace_status(ws) == 4
+    finally:
+        nabla.set_wait_limit_ns(0)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    O, _ = orc.masked_attention(x["q"][:, :1], x["k"][:, :1], x["v"][:, :1], M[:, :1])
+    gu.assert_close(o[:, :1], O, "bf16", "O after timeout")
