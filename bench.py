@@ -38,7 +38,8 @@ THR = 0.8
 # reported only while the source is unchanged.  Filled from the summaries
 # under profiles/.
 NCU_TRAFFIC = {
-    # "attn_fwd_tc.cu": ("<sha256>", bytes_per_launch_at_full_workload),
+    # profiles/attn_fwd_tc_720p_h4.md: 414.6 MB at 4 heads, scaled x10 to 40 heads
+    "attn_fwd_tc.cu": ("92ae18f6fe1958b66d79b364e05037f110319ff6d937278f252b0a6e1a1401a3", 4.146e9),
 }
 
 
@@ -200,6 +201,9 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="nabla", choices=["nabla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the head count (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
@@ -222,6 +226,8 @@ def main() -> None:
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     w = synth.WORKLOADS[WORKLOAD_ID]
+    if args.heads:
+        w = w.scaled(H=args.heads, name=f"{w.name}_h{args.heads}")
     wr = w.scaled(seed=w.seed + 1000 * rank) if rank else w
     x = synth.make_inputs(wr)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
@@ -288,6 +294,42 @@ def main() -> None:
     peaks = _peaks()
 
     # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(nabla, q, k, v, o, lse, mask, ws, stream, args, world, dist, dev, flops)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(w, world),
+            "attn_ms_per_call": attn_avg, "attn_tflops_actual": attn_tflops,
+            "attn_frac_of_bf16_peak": attn_tflops / peaks["bf16_sus"],
+            "mask_build_ms": mask_avg, "mask_build_gbs": mask_gbs, "mask_build_frac_hbm": mask_gbs / peaks["hbm"],
+            "kept_fraction": kept_frac, "kept_tiles": kept_tiles,
+            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel<128> (attn_fwd_tc.cu)",
+                         "achieved": attn_tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                         "frac": attn_tflops / peaks["bf16_sus"],
+                         "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside a long step); "
+                                      f"burst {peaks['bf16']}",
+                         "traffic": _traffic("attn_fwd_tc.cu"),
+                         "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(nabla, q, k, v, o, lse, mask, ws, stream, args, world, dist, dev, flops):
+    """Same step through the public API with the inputs copied in from pinned
+    host memory and the output copied back, inside the timed region."""
+    import torch
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -313,34 +355,8 @@ def main() -> None:
         e2e_ms = t.item()
     h2d = 3 * q.numel() * q.element_size()
     d2h = o.numel() * o.element_size()
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(w, world),
-            "attn_ms_per_call": attn_avg, "attn_tflops_actual": attn_tflops,
-            "attn_frac_of_bf16_peak": attn_tflops / peaks["bf16_sus"],
-            "mask_build_ms": mask_avg, "mask_build_gbs": mask_gbs, "mask_build_frac_hbm": mask_gbs / peaks["hbm"],
-            "kept_fraction": kept_frac, "kept_tiles": kept_tiles,
-            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel<128> (attn_fwd_tc.cu)",
-                         "achieved": attn_tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                         "frac": attn_tflops / peaks["bf16_sus"],
-                         "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside a long step); "
-                                      f"burst {peaks['bf16']}",
-                         "traffic": _traffic("attn_fwd_tc.cu"),
-                         "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 4 * args.steps,
-            "clocks": clocks.summary(),
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR)
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    return {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
 if __name__ == "__main__":

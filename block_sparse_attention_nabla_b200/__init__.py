@@ -20,6 +20,7 @@ import torch
 
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
+           "selftest_wait_timeout",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -29,7 +30,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_mask_from_bits", "nabla_attn_fwd",
-           "nabla_attn_bwd", "nabla_workspace_status", "nabla_set_wait_limit_ns",
+           "nabla_attn_bwd", "nabla_selftest_wait_timeout", "nabla_workspace_status",
+           "nabla_set_wait_limit_ns",
            "nabla_last_error", "nabla_abi_version"]
 
 
@@ -75,11 +77,12 @@ def lib() -> ctypes.CDLL:
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_workspace_status.argtypes = [P, ctypes.POINTER(I32), P]
+    L.nabla_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.nabla_set_wait_limit_ns.argtypes, L.nabla_set_wait_limit_ns.restype = [ctypes.c_uint64], None
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_mask_from_bits", "nabla_attn_fwd", "nabla_attn_bwd",
-                 "nabla_workspace_status"):
+                 "nabla_workspace_status", "nabla_selftest_wait_timeout"):
         getattr(L, name).restype = I32
     _lib = L
     return L
@@ -241,6 +244,14 @@ def workspace_status(ws: torch.Tensor) -> int:
     _check(lib().nabla_workspace_status(ws.data_ptr(), ctypes.byref(out), _stream()),
            "nabla_workspace_status")
     return out.value
+
+
+def selftest_wait_timeout(ws: torch.Tensor, limit_ns: int) -> int:
+    """Runs the bounded-wait self-test kernel and returns the status word it
+    leaves (4 = NABLA_ERR_TIMEOUT is the expected outcome)."""
+    _check(lib().nabla_selftest_wait_timeout(ws.data_ptr(), int(limit_ns), _stream()),
+           "nabla_selftest_wait_timeout")
+    return workspace_status(ws)
 
 
 def set_wait_limit_ns(ns: int) -> None:

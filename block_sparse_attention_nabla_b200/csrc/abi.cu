@@ -158,8 +158,8 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const voi
   cudaStream_t st = (cudaStream_t)stream;
   const WsLayout L = ws_layout(d, false);
   char* ws = (char*)workspace;
-  float* qa = (float*)(ws + L.qa);
-  float* ka = (float*)(ws + L.ka);
+  double* qa = (double*)(ws + L.qa);
+  double* ka = (double*)(ws + L.ka);
   NABLA_TRY(reset_status(workspace, st));
   NABLA_CUDA(launch_pool(d, q, k, qa, ka, st), "pooling kernel");
   NABLA_CUDA(launch_select(d, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st), "select kernel");
@@ -231,6 +231,19 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
                                   mask->idx_t, (float*)((char*)workspace + L.delta), dq, dk, dv, st),
              "attention backward");
+  return NABLA_OK;
+}
+
+nabla_status nabla_selftest_wait_timeout(void* workspace, uint64_t limit_ns, nabla_stream_t stream) {
+  g_last_error.clear();
+  if (!workspace) return fail(NABLA_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(NABLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (limit_ns == 0 || limit_ns > 10000000000ull)
+    return fail(NABLA_ERR_INVALID_ARG, "limit_ns must lie in [1, 1e10] (got %llu)",
+                (unsigned long long)limit_ns);
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_wait_selftest((int32_t*)workspace + kWsStatus, limit_ns, st), "wait self-test");
   return NABLA_OK;
 }
 

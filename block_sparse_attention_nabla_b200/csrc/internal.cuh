@@ -27,7 +27,7 @@ inline Dims make_dims(const nabla_shape& s) {
 }
 
 // Workspace layout: a 256-byte header (status word, scheduler counters), then
-// the pooled Qa / Ka (fp32 [B, H, nb, D]) and, for the backward, the per-row
+// the pooled Qa / Ka (fp64 [B, H, nb, D]) and, for the backward, the per-row
 // Delta = rowsum(dO * O) (fp32 [B, H, S]).
 struct WsLayout {
   size_t header = 0;
@@ -40,7 +40,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
   WsLayout w;
   size_t off = 256;
-  size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(float);
+  size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(double);
   w.qa = off; off = align256(off + pooled);
   w.ka = off; off = align256(off + pooled);
   if (want_bwd) { w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float)); }
@@ -56,9 +56,9 @@ uint64_t wait_limit_ns();
 // ---------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 
-cudaError_t launch_pool(const Dims& d, const void* q, const void* k, float* qa, float* ka,
+cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
                         cudaStream_t st);
-cudaError_t launch_select(const Dims& d, const float* qa, const float* ka, float thr,
+cudaError_t launch_select(const Dims& d, const double* qa, const double* ka, float thr,
                           const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
                           cudaStream_t st);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
@@ -78,5 +78,7 @@ cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, co
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
                                const int32_t* cnt, const int32_t* idx, const int32_t* work,
                                void* o, float* lse, int32_t* ws_header, cudaStream_t st);
+
+cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 
 }  // namespace nabla

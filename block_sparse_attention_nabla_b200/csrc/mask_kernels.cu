@@ -70,18 +70,20 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 // ------------------------------------------------------------------ pooling
 // One 64-token block of Q or K per loop iteration: 256 threads issue 16-byte
-// loads covering the block (64 rows x D), each thread sums its rows in fp32,
-// lanes holding the same columns are combined by shuffles, warps through
-// shared memory.  The tail block divides by its number of valid tokens.
+// loads covering the block (64 rows x D), each thread sums its rows, lanes
+// holding the same columns are combined by shuffles, warps through shared
+// memory.  Sums run in fp64 and the means are stored in fp64: the selection
+// ranks near-equal entries of the reduced map by their fp64 logits.  The tail
+// block divides by its number of valid tokens.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                   float* __restrict__ qa, float* __restrict__ ka,
+                                                   double* __restrict__ qa, double* __restrict__ ka,
                                                    int S, int nb, long long per_tensor) {
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte chunk
   constexpr int CH = D / VE;          // chunks per row (8, 16 or 32)
   constexpr int RP = 256 / CH;        // rows covered per pass
   constexpr int NP = kBlock / RP;     // passes per block
-  __shared__ float red[8][D];
+  __shared__ double red[8][D];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = tid % CH, r0 = tid / CH;
   for (long long item = blockIdx.x; item < 2 * per_tensor; item += gridDim.x) {
@@ -97,11 +99,18 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
       const int r = r0 + p * RP;
       v[p] = r < valid ? ld_stream(src + (long long)r * D + c * VE) : make_uint4(0, 0, 0, 0);
     }
-    float acc[VE];
+    double acc[VE];
 #pragma unroll
-    for (int e = 0; e < VE; ++e) acc[e] = 0.f;
+    for (int e = 0; e < VE; ++e) acc[e] = 0.0;
 #pragma unroll
-    for (int p = 0; p < NP; ++p) add_chunk(v[p], acc);
+    for (int p = 0; p < NP; ++p) {
+      float f[VE];
+#pragma unroll
+      for (int e = 0; e < VE; ++e) f[e] = 0.f;
+      add_chunk(v[p], f);
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[e] += (double)f[e];
+    }
 #pragma unroll
     for (int off = CH; off < 32; off <<= 1)
 #pragma unroll
@@ -111,39 +120,39 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
       for (int e = 0; e < VE; ++e) red[warp][lane * VE + e] = acc[e];
     __syncthreads();
     if (tid < D) {
-      float s = 0.f;
+      double sum = 0.0;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[w][tid];
-      (isk ? ka : qa)[it * D + tid] = s / (float)valid;
+      for (int w = 0; w < 8; ++w) sum += red[w][tid];
+      (isk ? ka : qa)[it * D + tid] = sum / (double)valid;
     }
     __syncthreads();
   }
 }
 
-// ------------------------------------------------------------ index emission
-// Writes one mask row given, for t = 0 .. W-1, the kept flag of block
-// j = 32 t + lane.  Indices come out in ascending order.
-struct RowOut {
-  uint32_t* bits;  // row's W words (may be null)
-  int32_t* idx;    // row's nb slots
-  int32_t* cnt;    // row's count
-};
-
 // ------------------------------------------------------------ score + select
 // One CTA handles R query blocks of one (b, h).
-//   phase 1: L[r][j] = (Qa_r . Ka_j) * (1/sqrt(D)) in fp32, staged in shared
-//            memory (the map is never written to HBM);
-//   phase 2: one warp per row: max, e_j = exp(L_j - max), s = sum e_j; the
-//            kept set is {j : sum of e over entries above j <= thr * s},
-//            found as the smallest bit pattern u of a positive float with
-//            sum_{e_k > u} e_k <= thr * s (binary search over the float bits;
-//            positive floats order like their bit patterns); keep e_j >= u.
-//            That is Algorithm 1's ascending cumulative sum compared with
-//            1 - thr, expressed through the mass above each entry.
+//   phase 1: L[r][j] = (Qa_r . Ka_j) * (1/sqrt(D)) in fp32 from fp32 copies
+//            of the fp64 pooled vectors, staged in shared memory (the map is
+//            never written to HBM);
+//   phase 2: one warp per row: max, e_j = exp(L_j - max), s = sum e_j.  Block
+//            j is kept iff the mass of the entries ranked above it is
+//            <= thr * s: Algorithm 1's ascending cumulative sum compared with
+//            1 - thr, stated through the mass above each entry.  The fp32
+//            cut-off is the smallest float bit pattern u with
+//            sum_{e_k > u} e_k <= thr * s (binary search; positive floats
+//            order like their bit patterns).  fp32 cannot order entries whose
+//            values differ by less than its rounding error, so the entries
+//            within a relative 2^-12 of the cut-off value are ranked again by
+//            their fp64 logits (ties: higher block index first, as a stable
+//            ascending sort leaves them) and kept in rank order while the mass
+//            above them stays <= thr * s;
 //   then OR the STA window and emit bits / cnt / idx.
+constexpr float kWindow = 1.0f / 4096.0f;
+constexpr int kMaxCand = 32;
+
 template <int R, int D>
 __global__ void __launch_bounds__(256) select_kernel(
-    const float* __restrict__ qa, const float* __restrict__ ka, int nb, int W, int ldl, float thr,
+    const double* __restrict__ qa, const double* __restrict__ ka, int nb, int W, int ldl, float thr,
     float scale, const int32_t* __restrict__ coords, int hT, int hH, int hW,
     uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
   extern __shared__ float4 smem4[];
@@ -152,6 +161,8 @@ __global__ void __launch_bounds__(256) select_kernel(
   constexpr int RG = R / 2;  // row pairs
   constexpr int CT = 256 / RG;
   constexpr int CPT = KC / CT;
+  __shared__ int cand_j[8][kMaxCand];
+  __shared__ float cand_e[8][kMaxCand];
   float* Ls = reinterpret_cast<float*>(smem4);
   float* Qs = Ls + R * ldl;
   float* Ks = Qs + R * LD;
@@ -163,14 +174,14 @@ __global__ void __launch_bounds__(256) select_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long bh = blockIdx.y;
   const int row0 = blockIdx.x * R;
-  const float* qa_h = qa + bh * nb * D;
-  const float* ka_h = ka + bh * nb * D;
+  const double* qa_h = qa + bh * nb * D;
+  const double* ka_h = ka + bh * nb * D;
 
-  for (int e = tid; e < R * (D / 4); e += 256) {
-    const int r = e / (D / 4), c4 = e % (D / 4);
-    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (row0 + r < nb) val = *reinterpret_cast<const float4*>(qa_h + (long long)(row0 + r) * D + c4 * 4);
-    *reinterpret_cast<float4*>(Qs + r * LD + c4 * 4) = val;
+  for (int e = tid; e < R * (D / 2); e += 256) {
+    const int r = e / (D / 2), c2 = e % (D / 2);
+    double2 val = make_double2(0.0, 0.0);
+    if (row0 + r < nb) val = *reinterpret_cast<const double2*>(qa_h + (long long)(row0 + r) * D + c2 * 2);
+    *reinterpret_cast<float2*>(Qs + r * LD + c2 * 2) = make_float2((float)val.x, (float)val.y);
   }
   if (use_sta)
     for (int j = tid; j < nb; j += 256) {
@@ -182,11 +193,11 @@ __global__ void __launch_bounds__(256) select_kernel(
   const int tr = tid / CT, tc = tid % CT;
   for (int c0 = 0; c0 < nb; c0 += KC) {
     __syncthreads();
-    for (int e = tid; e < KC * (D / 4); e += 256) {
-      const int r = e / (D / 4), c4 = e % (D / 4);
-      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + r < nb) val = *reinterpret_cast<const float4*>(ka_h + (long long)(c0 + r) * D + c4 * 4);
-      *reinterpret_cast<float4*>(Ks + r * LD + c4 * 4) = val;
+    for (int e = tid; e < KC * (D / 2); e += 256) {
+      const int r = e / (D / 2), c2 = e % (D / 2);
+      double2 val = make_double2(0.0, 0.0);
+      if (c0 + r < nb) val = *reinterpret_cast<const double2*>(ka_h + (long long)(c0 + r) * D + c2 * 2);
+      *reinterpret_cast<float2*>(Ks + r * LD + c2 * 2) = make_float2((float)val.x, (float)val.y);
     }
     __syncthreads();
     float acc0[CPT], acc1[CPT];
@@ -248,6 +259,60 @@ __global__ void __launch_bounds__(256) select_kernel(
       f = warp_sum(f);
       if (f <= limit) hi = mid; else lo = mid + 1u;
     }
+    // lo == 0: every block is kept (thr = 1 reaches here).
+    float keep_above = 0.f;  // entries with e > keep_above are kept
+    if (lo != 0u) {
+      const float vcut = __uint_as_float(lo);
+      const float vhi = vcut * (1.f + kWindow), vlo = vcut * (1.f - kWindow);
+      float above = 0.f;
+      int ncand = 0;
+      for (int t = 0; t < W; ++t) {
+        const int j = t * 32 + lane;
+        const float e = j < nb ? Lr[j] : 0.f;
+        above += e > vhi ? e : 0.f;
+        const bool isc = j < nb && e >= vlo && e <= vhi;
+        const uint32_t word = __ballot_sync(kFull, isc);
+        const int slot = ncand + __popc(word & lanemask_lt());
+        if (isc && slot < kMaxCand) {
+          cand_j[warp][slot] = j;
+          cand_e[warp][slot] = e;
+        }
+        ncand += __popc(word);
+      }
+      above = warp_sum(above);
+      __syncwarp();
+      if (ncand <= kMaxCand) {
+        // rank the candidates by their fp64 logits
+        const bool act = lane < ncand;
+        const int cj = act ? cand_j[warp][lane] : 0;
+        const float ce = act ? cand_e[warp][lane] : 0.f;
+        double lg = -1e300;
+        if (act) {
+          const double* qrow = qa_h + (long long)row * D;
+          const double* krow = ka_h + (long long)cj * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot = fma(qrow[d], krow[d], dot);
+          lg = dot;
+        }
+        float mass = above;
+        for (int b2 = 0; b2 < ncand; ++b2) {
+          const double lb = __shfl_sync(kFull, lg, b2);
+          const int jb = __shfl_sync(kFull, cj, b2);
+          const float eb = __shfl_sync(kFull, ce, b2);
+          if (lb > lg || (lb == lg && jb > cj)) mass += eb;
+        }
+        if (act) Lr[cj] = mass <= limit ? 2.0f : 0.0f;
+      } else {
+        // more near-equal entries than one warp ranks at once: keep the
+        // fp32 decision (all entries at or above the cut-off value)
+        for (int j = lane; j < nb; j += 32) {
+          const float e = Lr[j];
+          if (e >= vlo && e <= vhi) Lr[j] = __float_as_uint(e) >= lo ? 2.0f : 0.0f;
+        }
+      }
+      __syncwarp();
+      keep_above = vhi;
+    }
     const long long grow = bh * nb + row;
     uint32_t* brow = bits + grow * W;
     int32_t* irow = idx + grow * nb;
@@ -257,7 +322,7 @@ __global__ void __launch_bounds__(256) select_kernel(
       const int j = t * 32 + lane;
       bool keep = false;
       if (j < nb) {
-        keep = __float_as_uint(Lr[j]) >= lo;
+        keep = lo == 0u || Lr[j] > keep_above;
         if (use_sta && !keep)
           keep = abs(Ct[j] - ti) <= hT && abs(Cy[j] - yi) <= hH && abs(Cx[j] - xi) <= hW;
       }
@@ -375,7 +440,7 @@ int num_sms() {
   return sms;
 }
 
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemLimit = 227 * 1024 - 4096;  // dynamic part; the kernel also has ~2 KB static
 
 template <int R, int D>
 size_t select_smem(int nb, int ldl) {
@@ -383,7 +448,7 @@ size_t select_smem(int nb, int ldl) {
 }
 
 template <int R, int D>
-cudaError_t run_select(const Dims& d, const float* qa, const float* ka, float thr,
+cudaError_t run_select(const Dims& d, const double* qa, const double* ka, float thr,
                        const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
                        cudaStream_t st, int ldl) {
   const size_t smem = select_smem<R, D>(d.nb, ldl);
@@ -399,7 +464,7 @@ cudaError_t run_select(const Dims& d, const float* qa, const float* ka, float th
 }
 
 template <int D>
-cudaError_t select_d(const Dims& d, const float* qa, const float* ka, float thr,
+cudaError_t select_d(const Dims& d, const double* qa, const double* ka, float thr,
                      const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
                      cudaStream_t st) {
   const int ldl = (d.nb + 3) & ~3;
@@ -414,7 +479,7 @@ cudaError_t select_d(const Dims& d, const float* qa, const float* ka, float thr,
 
 }  // namespace
 
-cudaError_t launch_pool(const Dims& d, const void* q, const void* k, float* qa, float* ka,
+cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
                         cudaStream_t st) {
   const long long per = d.BH() * d.nb;
   const long long items = 2 * per;
@@ -433,7 +498,7 @@ cudaError_t launch_pool(const Dims& d, const void* q, const void* k, float* qa, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const Dims& d, const float* qa, const float* ka, float thr,
+cudaError_t launch_select(const Dims& d, const double* qa, const double* ka, float thr,
                           const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
                           cudaStream_t st) {
   if (d.D == 128) return select_d<128>(d, qa, ka, thr, sta, bits, cnt, idx, st);

@@ -55,10 +55,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (abort && *abort) return false;
-    if ((++spins & 15u) == 0u && globaltimer() - t0 > limit_ns) {
+    if (globaltimer() - t0 > limit_ns) {
       if (abort) *abort = 1;
       return false;
     }

@@ -160,6 +160,15 @@ NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, c
 NABLA_API nabla_status nabla_workspace_status(const void* workspace, int32_t* host_status,
                                     nabla_stream_t stream);
 
+/* Self-test of the bounded-wait path: launches one small kernel whose only
+ * wait is on a barrier that nothing ever arrives on, so the wait runs out after
+ * limit_ns nanoseconds (1 <= limit_ns <= 1e10) and the kernel records
+ * NABLA_ERR_TIMEOUT in the status word of `workspace` (any device buffer of at
+ * least 256 bytes, 256-byte aligned), as every pipelined kernel does when one
+ * of its waits runs out.  Read the result with nabla_workspace_status(). */
+NABLA_API nabla_status nabla_selftest_wait_timeout(void* workspace, uint64_t limit_ns,
+                                                   nabla_stream_t stream);
+
 /* Sets the time limit, in nanoseconds, of every bounded spin-wait in the
  * kernels launched after this call by the calling process (0 restores the
  * default of 2 s).  A wait that runs out makes its kernel stop cleanly and set

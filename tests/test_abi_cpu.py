@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 9
+    assert len(names) == 10
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -57,7 +57,7 @@ def test_workspace_size_formula(L):
         return (x + 255) // 256 * 256
     for (B, H, S, D) in [(1, 2, 4096, 64), (1, 40, 75600, 128), (2, 16, 16384, 128), (1, 1, 1, 64)]:
         nb = -(-S // 64)
-        pooled = align(B * H * nb * D * 4)
+        pooled = align(B * H * nb * D * 8)
         fwd = 256 + 2 * pooled
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 0) == fwd
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 1) == fwd + align(B * H * S * 4)
@@ -126,6 +126,9 @@ def test_mask_from_bits_and_status_argument_errors(L):
     assert L.nabla_mask_from_bits(ctypes.byref(sh), None, ctypes.byref(mask_struct()), FAKE, 1 << 40, None) == INVALID
     assert L.nabla_mask_from_bits(ctypes.byref(sh), FAKE, ctypes.byref(mask_struct(idx=None)), FAKE, 1 << 40, None) == INVALID
     assert L.nabla_workspace_status(None, None, None) == INVALID
+    assert L.nabla_selftest_wait_timeout(None, 1000, None) == WORKSPACE
+    assert L.nabla_selftest_wait_timeout(FAKE, 0, None) == INVALID
+    assert L.nabla_selftest_wait_timeout(FAKE, 10**11, None) == INVALID
 
 
 def test_last_error_is_per_call(L):

@@ -152,10 +152,27 @@ def test_bwd_pretraining_workload_two_heads():
 
 # ------------------------------------------------------ bounded waits
 
-def test_wait_limit_reports_timeout_and_context_survives():
-    """A wait limit far below the time a tile takes makes the forward kernel's
-    bounded waits run out: the kernel stops, reports NABLA_ERR_TIMEOUT in the
-    workspace status word, and the next call with the default limit works."""
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """A wait on a barrier that nothing arrives on runs out after its limit;
+    the kernel records NABLA_ERR_TIMEOUT and the context stays usable."""
+    x = synth.make_random_qkv(1, 2, 1000, 128, "bf16", seed=5)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    ws = nabla.workspace(q)
+    assert nabla.selftest_wait_timeout(ws, 2_000_000) == 4
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    O, _ = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, "bf16", "O after a timed-out wait")
+
+
+def test_forward_with_tiny_wait_limit_stops_cleanly():
+    """With a 1 ns limit the forward kernel's first wait that is not already
+    satisfied runs out: the kernel stops, drains its own copies and MMAs,
+    frees TMEM and reports NABLA_ERR_TIMEOUT (0 if every wait happened to be
+    satisfied at once).  The next call with the default limit is correct."""
     x = synth.make_random_qkv(1, 4, 4096, 128, "bf16", seed=5)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], 1.0)
     q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
@@ -165,7 +182,7 @@ def test_wait_limit_reports_timeout_and_context_survives():
         nabla.set_wait_limit_ns(1)
         nabla.attn_fwd(q, k, v, mask, ws=ws)
         torch.cuda.synchronize()
-        assert nabla.workspace_status(ws) == 4
+        assert nabla.workspace_status(ws) in (0, 4)
     finally:
         nabla.set_wait_limit_ns(0)
     o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
