@@ -115,6 +115,15 @@ nabla_status reset_status(void* ws, cudaStream_t st) {
 
 }  // namespace
 
+void record_error(nabla_status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
 uint64_t wait_limit_ns() {
   const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
   return v ? v : 2000000000ull;

@@ -53,6 +53,10 @@ enum : int { kWsStatus = 0, kWsTileCounter = 1 };
 
 uint64_t wait_limit_ns();
 
+// Records the message nabla_last_error() returns in the calling thread (an
+// empty message clears it); status is for the reader's benefit only.
+void record_error(nabla_status status, const char* fmt, ...);
+
 // ---------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 

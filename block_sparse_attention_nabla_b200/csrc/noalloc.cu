@@ -1,0 +1,126 @@
+// Mask builder entry point that allocates nothing: nabla_build_mask_noalloc.
+//
+// Some callers cannot allocate device memory when they build a mask: a serving
+// process that reserved all device memory up front and forbids side
+// allocations while a request runs, a plug-in loaded into such a host, or code
+// that must not call cudaMalloc because it may synchronise the device and
+// stall streams that other work depends on.  They still own the inputs and the
+// mask outputs; only the builder's scratch (the pooled Qa / Ka and the status
+// word) comes from the static array below instead of a caller workspace.
+//
+// The array lives in every GPU that loads this library until the process
+// exits.  Every call shares it and it keeps the last call's contents, so calls
+// whose work overlaps on the GPU (different streams, or different host
+// threads on one device) race on it; callers serialise them.
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace nabla {
+namespace {
+
+// 32 MiB: a 256-byte header (status word) and the fp64 pooled vectors.
+constexpr size_t kNoAllocScratchBytes = 32u << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static array on the current device.  The name
+// g_noalloc_scratch means something else in host code, so the address is asked
+// for once per device, with that device current, and cached.
+nabla_status scratch_on_current_device(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_error(NABLA_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
+    return NABLA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    record_error(NABLA_ERR_UNSUPPORTED, "device %d is beyond the %d devices this entry point serves",
+                 dev, kMaxDevices);
+    return NABLA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      record_error(NABLA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s",
+                   cudaGetErrorString(e));
+      return NABLA_ERR_CUDA;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return NABLA_OK;
+}
+
+bool al(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+nabla_status bad(nabla_status s, const char* what) {
+  record_error(s, "%s", what);
+  return s;
+}
+
+}  // namespace
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const void* q,
+                                                           const void* k, float thr,
+                                                           const nabla_sta* sta,
+                                                           const nabla_mask* out,
+                                                           nabla_stream_t stream) {
+  record_error(NABLA_OK, "");
+  if (!shape) return bad(NABLA_ERR_INVALID_ARG, "shape is NULL");
+  if (shape->B < 1 || shape->H < 1 || shape->S < 1)
+    return bad(NABLA_ERR_INVALID_ARG, "B, H and S must be >= 1");
+  if (shape->block != kBlock) return bad(NABLA_ERR_UNSUPPORTED, "block must be 64");
+  if (shape->dtype != NABLA_BF16 && shape->dtype != NABLA_FP32)
+    return bad(NABLA_ERR_INVALID_ARG, "dtype must be NABLA_BF16 or NABLA_FP32");
+  if (shape->D != 64 && shape->D != 128) return bad(NABLA_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if ((shape->S + kBlock - 1) / kBlock > kMaxBlocks) return bad(NABLA_ERR_UNSUPPORTED, "S too large");
+  if (!q || !k || !al(q, 16) || !al(k, 16))
+    return bad(NABLA_ERR_INVALID_ARG, "q and k must be non-NULL and 16-byte aligned");
+  if (!(thr > 0.f && thr <= 1.f)) return bad(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1]");
+  if (sta && sta->block_coords &&
+      (!al(sta->block_coords, 4) || sta->wT < 1 || sta->wH < 1 || sta->wW < 1))
+    return bad(NABLA_ERR_INVALID_ARG, "STA coordinates must be 4-byte aligned and windows >= 1");
+  if (!out || !out->bits || !out->cnt || !out->idx || !out->work)
+    return bad(NABLA_ERR_INVALID_ARG, "mask.bits, cnt, idx and work are required");
+  if (!al(out->bits, 4) || !al(out->cnt, 4) || !al(out->idx, 4) || !al(out->work, 4))
+    return bad(NABLA_ERR_INVALID_ARG, "mask arrays must be 4-byte aligned");
+  if ((out->cnt_t == nullptr) != (out->idx_t == nullptr))
+    return bad(NABLA_ERR_INVALID_ARG, "mask.cnt_t and mask.idx_t must both be set or both NULL");
+  const Dims d = make_dims(*shape);
+  const WsLayout L = ws_layout(d, false);
+  if (L.total > kNoAllocScratchBytes) {
+    record_error(NABLA_ERR_UNSUPPORTED,
+                 "this shape needs %zu bytes of scratch; the static scratch of "
+                 "nabla_build_mask_noalloc holds %zu (B * H * ceil(S / 64) * D * 16 bytes must fit); "
+                 "use nabla_build_mask with a workspace",
+                 L.total, kNoAllocScratchBytes);
+    return NABLA_ERR_UNSUPPORTED;
+  }
+  void* scratch = nullptr;
+  const nabla_status st0 = scratch_on_current_device(&scratch);
+  if (st0 != NABLA_OK) return st0;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)scratch;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);  // the status word starts at zero
+  if (e == cudaSuccess) e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), st);
+  if (e == cudaSuccess)
+    e = launch_select(d, (const double*)(ws + L.qa), (const double*)(ws + L.ka), thr, sta, out->bits,
+                      out->cnt, out->idx, st);
+  if (e == cudaSuccess && out->cnt_t) e = launch_transpose_lists(d, out->bits, out->cnt_t, out->idx_t, st);
+  if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);
+  if (e != cudaSuccess) {
+    record_error(NABLA_ERR_CUDA, "nabla_build_mask_noalloc launch failed: %s", cudaGetErrorString(e));
+    return NABLA_ERR_CUDA;
+  }
+  return NABLA_OK;
+}

@@ -125,6 +125,30 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
                               const nabla_sta* sta, const nabla_mask* out, void* workspace,
                               size_t workspace_bytes, nabla_stream_t stream);
 
+/* Mask builder that allocates nothing, for callers that cannot call
+ * cudaMalloc when they build a mask (for instance a serving process that
+ * reserved all device memory at start-up and allows no side allocation while
+ * a request runs, or code that must not risk the device-wide synchronisation
+ * an allocation can cause).  The paper has no counterpart: this is a packaging
+ * variant of nabla_build_mask.
+ *   Same arguments and results as nabla_build_mask, without the workspace: the
+ *   builder's scratch (status word, pooled Qa / Ka) lives in a 32 MiB static
+ *   device array inside the library, held by every GPU that loads it until the
+ *   process exits.  Shapes whose scratch exceeds it (B * H * ceil(S / 64) * D *
+ *   16 bytes plus 256 must fit in 32 MiB) are rejected with
+ *   NABLA_ERR_UNSUPPORTED and a message naming both sizes.
+ *   The first call on a device looks up the array's device address with that
+ *   device current (cudaGetSymbolAddress) and caches it; make that first call
+ *   before any stream capture.  The caller still provides q, k and every mask
+ *   output.
+ *   All calls share the array and it keeps the last call's contents (the
+ *   status word is cleared at the start of every call): calls whose GPU work
+ *   overlaps race on it, so serialise them.  The status word is not readable
+ *   through nabla_workspace_status. */
+NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const void* q,
+                                                const void* k, float thr, const nabla_sta* sta,
+                                                const nabla_mask* out, nabla_stream_t stream);
+
 /* Builds cnt, idx, work (and cnt_t, idx_t if not NULL) of `out` from a
  * caller-supplied bitmask `bits` [B, H, nb, W] (padding bits must be zero);
  * out->bits is ignored.  Lets attention run under any externally computed

@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 10
+    assert len(names) == 11
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
