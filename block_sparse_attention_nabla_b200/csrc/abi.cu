@@ -201,13 +201,12 @@ nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(check_tensor(v, "v"));
   NABLA_TRY(check_tensor(o, "o"));
   if (lse && !aligned(lse, 4)) return fail(NABLA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
-  NABLA_TRY(check_mask_out(mask, false));
+  NABLA_TRY(check_mask_out(mask, true));
   NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
   cudaStream_t st = (cudaStream_t)stream;
   NABLA_TRY(reset_status(workspace, st));
   if (d.dtype == NABLA_BF16)
-    NABLA_CUDA(launch_attn_fwd_tc(d, q, k, v, mask->cnt, mask->idx, mask->work, o, lse,
-                                  (int32_t*)workspace, st),
+    NABLA_CUDA(launch_attn_fwd_tc(d, q, k, v, mask->bits, mask->work, o, lse, (int32_t*)workspace, st),
                "tensor-core attention forward");
   else
     NABLA_CUDA(launch_attn_fwd_simt(d, q, k, v, mask->cnt, mask->idx, o, lse, st),

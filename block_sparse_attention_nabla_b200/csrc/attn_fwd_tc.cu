@@ -8,18 +8,26 @@
 // tile, so every MMA runs at M = 128.  The unit visits the union of the two
 // blocks' kept key blocks in ascending order; rows whose own block did not keep
 // a visited key block see it as -inf.  Units come from the mask builder's work
-// list (grouped by head so a head's K and V stay in L2, most expensive first);
-// the grid is persistent, one CTA per SM, units assigned round-robin.
+// list (grouped by head so a head's K and V stay in L2, most expensive first),
+// assigned round-robin to a persistent grid of two CTAs per SM: one thread
+// issuing tcgen05 MMAs cannot keep the tensor core busy with these tile
+// shapes, two can.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: Q tile per unit, K and V tiles through an
-//               NS-stage ring, plus the (key block, membership) of each stage;
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM S
-//               buffers, then O += P V with P read from TMEM;
-//   warps 2-5   softmax and epilogue, one thread per row: load S from TMEM,
-//               online softmax in the log2 domain, write P (bf16) over S in
-//               TMEM, rescale O only when the running max grows by more than
-//               2^8 (exact after the final division), finally O / l and LSE.
+// Warp roles (224 threads per CTA):
+//   warp 0      Q and K producer: TMA of the unit's Q tile and of the K tiles
+//               of its key blocks (3-deep ring; a slot is refilled as soon as
+//               its S = Q K^T completes), plus one (key block, membership)
+//               record per tile; it walks the OR of the pair's two bitmask rows;
+//   warp 6      V producer: the same walk, V tiles into a 2-deep ring (a slot
+//               is refilled once its O += P V completes);
+//   warp 1      TMEM owner and MMA issuer.  S of the next tile is issued before
+//               the P V of the current one, into the other of two TMEM S
+//               buffers, so the softmax of one tile overlaps the MMAs of its
+//               neighbours;
+//   warps 2-5   softmax and epilogue, one thread per row: load S, online
+//               softmax in the log2 domain, write P (bf16) over S; rescale O
+//               only when the running max grows by more than 2^8 (exact after
+//               the final division); finally O / l and LSE.
 // TMEM columns: [0, 64) S0 / P0, [64, 128) S1 / P1, [128, 128 + D) O.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -34,8 +42,14 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+// Ring of per-tile (key block, membership) records.  The producer writes the
+// record of tile g only after S of tile g - 3 completed, which needs the
+// softmax of tile g - 5 done, so a record is never overwritten early.
+constexpr int kMeta = 8;
+constexpr int kCtasPerSm = 2;
+constexpr int kThreads = 224;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kOCol = 128;
 constexpr float kRescaleLog2 = 8.0f;
@@ -49,52 +63,74 @@ struct FwdLayout {
   static constexpr uint32_t kQHalf = 128 * 128;             // bytes: 128 rows x 128 B
   static constexpr uint32_t kKVHalf = 64 * 128;             // bytes: 64 rows x 128 B
   static constexpr uint32_t kQBytes = kHalves * kQHalf;
-  static constexpr uint32_t kKVBytes = kHalves * kKVHalf;
+  static constexpr uint32_t kKVBytes = kHalves * kKVHalf;   // one K or V tile
   static constexpr uint32_t q_off = 0;
   static constexpr uint32_t k_off = q_off + kQBytes;
-  static constexpr uint32_t v_off = k_off + kStages * kKVBytes;
-  static constexpr uint32_t bar_off = v_off + kStages * kKVBytes;
-  // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
-  static constexpr int kNumBars = 2 + 3 * kStages + 2 + 2 + 2;
+  static constexpr uint32_t v_off = k_off + kKStages * kKVBytes;
+  static constexpr uint32_t bar_off = v_off + kVStages * kKVBytes;
+  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2],
+  // p_full[2], o_done, o_final, drain, meta_full[kMeta]
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 3 + kMeta;
   static constexpr uint32_t meta_off = bar_off + kNumBars * 8;
-  static constexpr uint32_t misc_off = meta_off + kStages * 4;
+  static constexpr uint32_t misc_off = meta_off + kMeta * 4;
   static constexpr uint32_t bytes = misc_off + 16;
-  static constexpr uint32_t alloc_bytes = bytes + 1024;     // slack for 1024-byte alignment
 };
 
 struct Bars {
-  uint64_t* q_full;
-  uint64_t* q_empty;
-  uint64_t* k_full;
-  uint64_t* v_full;
-  uint64_t* kv_empty;
-  uint64_t* s_full;
-  uint64_t* p_full;
-  uint64_t* o_done;
-  uint64_t* drain;
+  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done,
+      *o_final, *drain, *meta_full;
+};
+
+// Walks the key blocks of one unit in ascending order: the set bits of the OR
+// of the unit's two bitmask rows, with the membership of each.
+struct UnitWalk {
+  const uint32_t* ra;
+  const uint32_t* rb;
+  int W;
+  template <typename F>
+  __device__ __forceinline__ bool run(F&& f) const {
+    for (int w = 0; w < W; ++w) {
+      const uint32_t wa = ra[w], wb = rb ? rb[w] : 0u;
+      uint32_t un = wa | wb;
+      while (un) {
+        const int bit = __ffs(un) - 1;
+        un &= un - 1u;
+        const int flags = (int)((wa >> bit) & 1u) | (int)(((wb >> bit) & 1u) << 1);
+        if (!f(w * 32 + bit, flags)) return false;
+      }
+    }
+    return true;
+  }
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ cnt,
-                  const int32_t* __restrict__ idx, const int32_t* __restrict__ work, int n_units,
-                  int S, int nb, int npairs, float scale_log2, __nv_bfloat16* __restrict__ out,
-                  float* __restrict__ lse, int32_t* __restrict__ status, uint64_t limit_ns) {
+                  const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ bits,
+                  const int32_t* __restrict__ work, int n_units, int S, int nb, int W, int npairs,
+                  float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                  int32_t* __restrict__ status, uint64_t limit_ns) {
   using L = FwdLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The 128-byte swizzle atoms must start on 1024-byte boundaries.
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(status, 0, (int32_t)NABLA_ERR_UNSUPPORTED);
+    return;
+  }
   uint64_t* bars = (uint64_t*)(smem + L::bar_off);
   Bars b;
   b.q_full = bars;
   b.q_empty = bars + 1;
   b.k_full = bars + 2;
-  b.v_full = b.k_full + kStages;
-  b.kv_empty = b.v_full + kStages;
-  b.s_full = b.kv_empty + kStages;
+  b.k_empty = b.k_full + kKStages;
+  b.v_full = b.k_empty + kKStages;
+  b.v_empty = b.v_full + kVStages;
+  b.s_full = b.v_empty + kVStages;
   b.p_full = b.s_full + 2;
   b.o_done = b.p_full + 2;
-  b.drain = b.o_done + 1;
+  b.o_final = b.o_done + 1;
+  b.drain = b.o_final + 1;
+  b.meta_full = b.drain + 1;
   volatile int32_t* meta = (volatile int32_t*)(smem + L::meta_off);
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
@@ -104,17 +140,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(b.q_full, 1);
     mbar_init(b.q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(b.k_full + s, 1);
+      mbar_init(b.k_empty + s, 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(b.v_full + s, 1);
-      mbar_init(b.kv_empty + s, 1);
+      mbar_init(b.v_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(b.s_full + s, 1);
       mbar_init(b.p_full + s, 128);
     }
     mbar_init(b.o_done, 1);
+    mbar_init(b.o_final, 1);
     mbar_init(b.drain, 1);
+    for (int s = 0; s < kMeta; ++s) mbar_init(b.meta_full + s, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -132,11 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t smem_base = smem_u32(smem);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ---------------------------------------------------- Q and K producer
     if (lane == 0) {
-      uint32_t kv_iter = 0, q_iter = 0;
-      int last_use[kStages];
-      for (int s = 0; s < kStages; ++s) last_use[s] = -1;
+      uint32_t q_iter = 0, g = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const int unit = work[2 * u];
@@ -147,66 +186,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < L::kHalves; ++h)
           tma_load_3d(smem + L::q_off + h * L::kQHalf, &tm_q, b.q_full, h * 64, p * 128, bh);
         ++q_iter;
-        const long long ra = (long long)bh * nb + 2 * p;
-        const int na = cnt[ra];
-        const int nbb = (2 * p + 1 < nb) ? cnt[ra + 1] : 0;
-        const int32_t* la = idx + ra * nb;
-        const int32_t* lb = la + nb;
-        int ia = 0, ib = 0;
-        while (ia < na || ib < nbb) {
-          const int ja = ia < na ? la[ia] : 0x7fffffff;
-          const int jb = ib < nbb ? lb[ib] : 0x7fffffff;
-          const int j = min(ja, jb);
-          const int flags = (ja == j ? 1 : 0) | (jb == j ? 2 : 0);
-          ia += ja == j;
-          ib += jb == j;
-          const uint32_t stage = kv_iter % kStages, use = kv_iter / kStages;
-          if (use > 0 && !(ok = mbar_wait(b.kv_empty + stage, (use - 1) & 1, abort_flag, limit_ns))) break;
-          meta[stage] = j | (flags << 30);
-          mbar_expect_tx(b.k_full + stage, L::kKVBytes);
+        const uint32_t* ra = bits + ((long long)bh * nb + 2 * p) * W;
+        UnitWalk walk{ra, 2 * p + 1 < nb ? ra + W : nullptr, W};
+        ok = walk.run([&](int j, int flags) -> bool {
+          const uint32_t ks = g % kKStages, use = g / kKStages;
+          if (use > 0 && !mbar_wait(b.k_empty + ks, (use - 1) & 1, abort_flag, limit_ns)) return false;
+          meta[g % kMeta] = j | (flags << 30);
+          mbar_arrive(b.meta_full + g % kMeta);
+          mbar_expect_tx(b.k_full + ks, L::kKVBytes);
 #pragma unroll
           for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(smem + L::k_off + stage * L::kKVBytes + h * L::kKVHalf, &tm_k, b.k_full + stage,
-                        h * 64, j * 64, bh);
-          mbar_expect_tx(b.v_full + stage, L::kKVBytes);
-#pragma unroll
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(smem + L::v_off + stage * L::kKVBytes + h * L::kKVHalf, &tm_v, b.v_full + stage,
-                        h * 64, j * 64, bh);
-          last_use[stage] = (int)use;
-          ++kv_iter;
-        }
+            tma_load_3d(smem + L::k_off + ks * L::kKVBytes + h * L::kKVHalf, &tm_k, b.k_full + ks, h * 64,
+                        j * 64, bh);
+          ++g;
+          return true;
+        });
       }
-      // Let every copy this thread issued land before the CTA exits.
+      // Let every copy this thread issued land before the CTA exits (the last
+      // use of each slot completes after all earlier ones).
       if (q_iter > 0) mbar_wait(b.q_full, (q_iter - 1) & 1, nullptr, kDrainLimitNs);
-      for (int s = 0; s < kStages; ++s)
-        if (last_use[s] >= 0) {
-          mbar_wait(b.k_full + s, last_use[s] & 1, nullptr, kDrainLimitNs);
-          mbar_wait(b.v_full + s, last_use[s] & 1, nullptr, kDrainLimitNs);
-        }
+      for (uint32_t i = (g > kKStages ? g - kKStages : 0); i < g; ++i)
+        mbar_wait(b.k_full + i % kKStages, (i / kKStages) & 1, nullptr, kDrainLimitNs);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int unit = work[2 * u];
+        const int bh = unit / npairs, p = unit - bh * npairs;
+        const uint32_t* ra = bits + ((long long)bh * nb + 2 * p) * W;
+        UnitWalk walk{ra, 2 * p + 1 < nb ? ra + W : nullptr, W};
+        ok = walk.run([&](int j, int) -> bool {
+          const uint32_t vs = g % kVStages, use = g / kVStages;
+          if (use > 0 && !mbar_wait(b.v_empty + vs, (use - 1) & 1, abort_flag, limit_ns)) return false;
+          mbar_expect_tx(b.v_full + vs, L::kKVBytes);
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_3d(smem + L::v_off + vs * L::kKVBytes + h * L::kKVHalf, &tm_v, b.v_full + vs, h * 64,
+                        j * 64, bh);
+          ++g;
+          return true;
+        });
+      }
+      for (uint32_t i = (g > kVStages ? g - kVStages : 0); i < g; ++i)
+        mbar_wait(b.v_full + i % kVStages, (i / kVStages) & 1, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
-      uint32_t kv_iter = 0, q_iter = 0, g_iter = 0;
+      uint32_t g_iter = 0, q_iter = 0;
       bool ok = true;
-      auto issue_pv = [&](uint32_t t) -> bool {
-        const uint32_t g = g_iter + t;
-        const uint32_t sb = g & 1;
-        if (!mbar_wait(b.p_full + sb, (g >> 1) & 1, abort_flag, limit_ns)) return false;
-        const uint32_t kv = kv_iter + t, stage = kv % kStages;
-        if (!mbar_wait(b.v_full + stage, (kv / kStages) & 1, abort_flag, limit_ns)) return false;
+      uint32_t unit_first = 0;
+      auto issue_pv = [&](uint32_t h) -> bool {
+        const uint32_t sb = h & 1;
+        if (!mbar_wait(b.p_full + sb, (h >> 1) & 1, abort_flag, limit_ns)) return false;
+        const uint32_t vs = h % kVStages;
+        if (!mbar_wait(b.v_full + vs, (h / kVStages) & 1, abort_flag, limit_ns)) return false;
         tc_fence_after();
-        const uint32_t vbase = smem_base + L::v_off + stage * L::kKVBytes;
+        const uint32_t vbase = smem_base + L::v_off + vs * L::kKVBytes;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bdesc = desc_sw128(vbase + ks * 16 * 128, L::kKVHalf, 1024);
-          mma_ts(tmem + kOCol, tmem + sb * 64 + ks * 8, bdesc, idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
+          mma_ts(tmem + kOCol, tmem + sb * 64 + kk * 8, bdesc, idesc_o, (h > unit_first || kk > 0) ? 1u : 0u);
         }
+        mma_commit(b.v_empty + vs);
         mma_commit(b.o_done);
-        mma_commit(b.kv_empty + stage);
         return true;
       };
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -214,26 +262,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(b.q_full, q_iter & 1, abort_flag, limit_ns))) break;
         ++q_iter;
         tc_fence_after();
+        unit_first = g_iter;
+        const uint32_t qbase = smem_base + L::q_off;
         for (uint32_t t = 0; t < n && ok; ++t) {
-          const uint32_t kv = kv_iter + t, stage = kv % kStages;
-          if (!(ok = mbar_wait(b.k_full + stage, (kv / kStages) & 1, abort_flag, limit_ns))) break;
+          const uint32_t g = g_iter + t, ks = g % kKStages, sb = g & 1;
+          if (!(ok = mbar_wait(b.k_full + ks, (g / kKStages) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
-          const uint32_t sb = (g_iter + t) & 1;
-          const uint32_t kbase = smem_base + L::k_off + stage * L::kKVBytes;
-          const uint32_t qbase = smem_base + L::q_off;
+          const uint32_t kbase = smem_base + L::k_off + ks * L::kKVBytes;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (ks & 3) * 32;  // 16 bf16 = 32 B inside the 128-B row
-            const uint64_t adesc = desc_sw128(qbase + (ks >> 2) * L::kQHalf + koff, 16, 1024);
-            const uint64_t bdesc = desc_sw128(kbase + (ks >> 2) * L::kKVHalf + koff, 16, 1024);
-            mma_ss(tmem + sb * 64, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside the 128-B row
+            const uint64_t adesc = desc_sw128(qbase + (kk >> 2) * L::kQHalf + koff, 16, 1024);
+            const uint64_t bdesc = desc_sw128(kbase + (kk >> 2) * L::kKVHalf + koff, 16, 1024);
+            mma_ss(tmem + sb * 64, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
           }
+          mma_commit(b.k_empty + ks);
           mma_commit(b.s_full + sb);
-          if (t >= 1) ok = issue_pv(t - 1);
+          if (t >= 1) ok = issue_pv(g - 1);
         }
-        if (ok && n >= 1) ok = issue_pv(n - 1);
+        if (ok && n >= 1) ok = issue_pv(g_iter + n - 1);
+        if (ok) mma_commit(b.o_final);
         mma_commit(b.q_empty);
-        kv_iter += n;
         g_iter += n;
       }
     }
@@ -242,41 +291,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // row of the 128-row tile == TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint32_t kv_iter = 0, g_iter = 0;
+    const int my_flag = row < 64 ? 1 : 2;
+    uint32_t g_iter = 0, u_local = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
       const int unit = work[2 * u];
       const uint32_t n = (uint32_t)work[2 * u + 1];
       const int bh = unit / npairs, p = unit - bh * npairs;
       const int qrow = p * 128 + row;
-      const int my_flag = row < 64 ? 1 : 2;
       float m = -INFINITY, l = 0.f;
       for (uint32_t t = 0; t < n; ++t) {
         const uint32_t g = g_iter + t, sb = g & 1;
-        const uint32_t kv = kv_iter + t, stage = kv % kStages;
-        bool w1 = mbar_wait(b.s_full + sb, (g >> 1) & 1, abort_flag, limit_ns);
-        bool w2 = w1 && mbar_wait(b.k_full + stage, (kv / kStages) & 1, abort_flag, limit_ns);
+        const bool w1 = mbar_wait(b.s_full + sb, (g >> 1) & 1, abort_flag, limit_ns);
+        const bool w2 = w1 && mbar_wait(b.meta_full + g % kMeta, (g / kMeta) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
         tc_fence_after();
-        const int mt = meta[stage];
+        const int mt = meta[g % kMeta];
         const int j = mt & 0x3fffffff;
+        // All 32 rows of a warp belong to the same query block of the pair,
+        // so `mine` is warp-uniform: a warp whose block did not keep key
+        // block j only writes P = 0.
         const bool mine = ((mt >> 30) & my_flag) != 0;
-        const int kv_lim = (j == nb - 1) ? S - j * 64 : 64;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + sb * 64, r0);
-        tmem_ld32(lane_base + sb * 64 + 32, r1);
-        tmem_ld_wait();
-        float s[64];
-        float rmax = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = (mine && c < kv_lim) ? __uint_as_float(r0[c]) * scale_log2 : -INFINITY;
-          s[c + 32] = (mine && c + 32 < kv_lim) ? __uint_as_float(r1[c]) * scale_log2 : -INFINITY;
-          rmax = fmaxf(rmax, fmaxf(s[c], s[c + 32]));
-        }
+        uint32_t pk[32];
         float corr = 1.f;
         bool rescale = false;
-        if (rmax > -INFINITY) {
+        if (mine) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + sb * 64, r0);
+          tmem_ld32(lane_base + sb * 64 + 32, r1);
+          tmem_ld_wait();
+          float sc[64];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            sc[c] = __uint_as_float(r0[c]);
+            sc[c + 32] = __uint_as_float(r1[c]);
+          }
+          const int kv_lim = (j == nb - 1) ? S - j * 64 : 64;
+          if (kv_lim < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c >= kv_lim) sc[c] = -INFINITY;
+          }
+          float mx0 = sc[0], mx1 = sc[1];
+#pragma unroll
+          for (int c = 2; c < 62; c += 4) {
+            mx0 = fmax3(mx0, sc[c], sc[c + 1]);
+            mx1 = fmax3(mx1, sc[c + 2], sc[c + 3]);
+          }
+          const float rmax = fmax3(mx0, mx1, fmaxf(sc[62], sc[63])) * scale_log2;
           if (m == -INFINITY) {
             m = rmax;
           } else if (rmax > m + kRescaleLog2) {
@@ -284,51 +346,58 @@ __global__ void __launch_bounds__(kThreads, 1)
             m = rmax;
             rescale = true;
           }
-        }
-        uint32_t pk[32];
-        float psum = 0.f;
-        if (m == -INFINITY) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = 0u;
-        } else {
+          const uint64_t sc2 = f2pack(scale_log2, scale_log2);
+          const uint64_t nm2 = f2pack(-m, -m);
+          uint64_t acc2 = f2pack(0.f, 0.f), acc2b = f2pack(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(s[2 * c] - m), p1 = ex2(s[2 * c + 1] - m);
-            psum += p0 + p1;
+            float x0, x1;
+            f2unpack(ffma2(f2pack(sc[2 * c], sc[2 * c + 1]), sc2, nm2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (c & 1) acc2b = fadd2(acc2b, f2pack(p0, p1));
+            else acc2 = fadd2(acc2, f2pack(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
+          float s0, s1, s2, s3;
+          f2unpack(acc2, s0, s1);
+          f2unpack(acc2b, s2, s3);
+          l = l * corr + ((s0 + s1) + (s2 + s3));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
-        l = l * corr + psum;
         tmem_st32(lane_base + sb * 64, pk);
-        tmem_st_wait();
-        if (t >= 1) {
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O must hold the sum over tiles < g before it is scaled.  S of
+          // tile g completed, and it was issued after P V of tile g - 2, so
+          // o_done has completed phase g - 2 and at most phase g - 1: waiting
+          // for the parity of phase g - 1 is unambiguous even though this
+          // thread does not wait on o_done every tile.  (rescale implies
+          // t >= 1.)
           const bool w3 = mbar_wait(b.o_done, (g - 1) & 1, abort_flag, limit_ns);
           if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t ov[32];
-              tmem_ld32(lane_base + kOCol + c0, ov);
-              tmem_ld_wait();
-              if (rescale)
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(lane_base + kOCol + c0, ov);
+            tmem_ld_wait();
+            if (rescale)
 #pragma unroll
-                for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * corr);
-              tmem_st32(lane_base + kOCol + c0, ov);
-            }
-            tmem_st_wait();
+              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * corr);
+            tmem_st32(lane_base + kOCol + c0, ov);
           }
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(b.p_full + sb);
       }
       if (!ok) break;
-      // epilogue
-      if (n >= 1) {
-        const bool w4 = mbar_wait(b.o_done, (g_iter + n - 1) & 1, abort_flag, limit_ns);
-        if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
-        tc_fence_after();
-      }
+      // epilogue: o_final completes once per unit, after its last P V (at
+      // once for a unit without tiles)
+      const bool w4 = mbar_wait(b.o_final, u_local & 1, abort_flag, limit_ns);
+      if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
+      tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool valid = qrow < S;
       __nv_bfloat16* orow = out + ((long long)bh * S + qrow) * D;
@@ -355,7 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (valid && lse) lse[(long long)bh * S + qrow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
-      kv_iter += n;
       g_iter += n;
     }
   }
@@ -377,10 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
-    cudaDriverEntryPointQueryResult q;
+    cudaDriverEntryPointQueryResult qr;
     void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
       fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
   }
   return fn;
@@ -413,34 +481,32 @@ int sm_count() {
 }
 
 template <int D>
-cudaError_t run(const Dims& d, const void* q, const void* k, const void* v, const int32_t* cnt,
-                const int32_t* idx, const int32_t* work, void* o, float* lse, int32_t* ws_header,
-                cudaStream_t st) {
+cudaError_t run(const Dims& d, const void* q, const void* k, const void* v, const uint32_t* bits,
+                const int32_t* work, void* o, float* lse, int32_t* ws_header, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, d, 128) || !make_map(&tk, k, d, 64) || !make_map(&tv, v, d, 64))
     return cudaErrorInvalidValue;
   const int n_units = (int)(d.BH() * d.npairs);
-  const int grid = std::min(n_units, sm_count());
+  const int grid = std::min(n_units, kCtasPerSm * sm_count());
   auto kern = fwd_tc_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)FwdLayout<D>::alloc_bytes);
+                                       (int)FwdLayout<D>::bytes);
   if (e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  kern<<<grid, kThreads, FwdLayout<D>::alloc_bytes, st>>>(tq, tk, tv, cnt, idx, work, n_units, d.S,
-                                                          d.nb, d.npairs, scale_log2,
-                                                          (__nv_bfloat16*)o, lse, ws_header + kWsStatus,
-                                                          wait_limit_ns());
+  kern<<<grid, kThreads, FwdLayout<D>::bytes, st>>>(tq, tk, tv, bits, work, n_units, d.S, d.nb, d.W,
+                                                    d.npairs, scale_log2, (__nv_bfloat16*)o, lse,
+                                                    ws_header + kWsStatus, wait_limit_ns());
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
-                               const int32_t* cnt, const int32_t* idx, const int32_t* work,
-                               void* o, float* lse, int32_t* ws_header, cudaStream_t st) {
+                               const uint32_t* bits, const int32_t* work, void* o, float* lse,
+                               int32_t* ws_header, cudaStream_t st) {
   if (d.dtype != NABLA_BF16) return cudaErrorInvalidValue;
-  if (d.D == 128) return run<128>(d, q, k, v, cnt, idx, work, o, lse, ws_header, st);
-  return run<64>(d, q, k, v, cnt, idx, work, o, lse, ws_header, st);
+  if (d.D == 128) return run<128>(d, q, k, v, bits, work, o, lse, ws_header, st);
+  return run<64>(d, q, k, v, bits, work, o, lse, ws_header, st);
 }
 
 }  // namespace nabla

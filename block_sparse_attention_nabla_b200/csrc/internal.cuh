@@ -80,8 +80,8 @@ cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, co
                                  const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
                                  cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
-                               const int32_t* cnt, const int32_t* idx, const int32_t* work,
-                               void* o, float* lse, int32_t* ws_header, cudaStream_t st);
+                               const uint32_t* bits, const int32_t* work, void* o, float* lse,
+                               int32_t* ws_header, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 

@@ -158,7 +158,9 @@ NABLA_API nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint
                                   nabla_stream_t stream);
 
 /* Block-sparse attention forward, Eq. 4 of §2.2 with M = -inf outside the kept
- * tiles of `mask` (cnt, idx and work are read) and outside the sequence.
+ * tiles of `mask` (bits, cnt, idx and work must all describe the same mask:
+ * the bf16 path walks bits and work, the fp32 path cnt and idx) and outside
+ * the sequence.
  *   o    [B, H, S, D] output, shape->dtype.
  *   lse  float [B, H, S]: natural-log log-sum-exp of the scaled logits
  *        (Q K^T / sqrt(D)) over the attended keys, needed by the backward.
