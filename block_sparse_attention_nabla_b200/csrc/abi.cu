@@ -169,9 +169,12 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const voi
   char* ws = (char*)workspace;
   double* qa = (double*)(ws + L.qa);
   double* ka = (double*)(ws + L.ka);
+  float* qa32 = (float*)(ws + L.qa32);
+  float* ka32 = (float*)(ws + L.ka32);
   NABLA_TRY(reset_status(workspace, st));
-  NABLA_CUDA(launch_pool(d, q, k, qa, ka, st), "pooling kernel");
-  NABLA_CUDA(launch_select(d, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st), "select kernel");
+  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qa32, ka32, st), "pooling kernel");
+  NABLA_CUDA(launch_select(d, qa32, ka32, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st),
+             "select kernel");
   return emit_derived(d, out->bits, out, st);
 }
 

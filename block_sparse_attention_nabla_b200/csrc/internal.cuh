@@ -27,11 +27,11 @@ inline Dims make_dims(const nabla_shape& s) {
 }
 
 // Workspace layout: a 256-byte header (status word, scheduler counters), then
-// the pooled Qa / Ka (fp64 [B, H, nb, D]) and, for the backward, the per-row
-// Delta = rowsum(dO * O) (fp32 [B, H, S]).
+// the pooled Qa / Ka in fp64 and rounded to fp32 ([B, H, nb, D] each) and,
+// for the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]).
 struct WsLayout {
   size_t header = 0;
-  size_t qa = 0, ka = 0, delta = 0;
+  size_t qa = 0, ka = 0, qa32 = 0, ka32 = 0, delta = 0;
   size_t total = 0;
 };
 
@@ -43,6 +43,8 @@ inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
   size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(double);
   w.qa = off; off = align256(off + pooled);
   w.ka = off; off = align256(off + pooled);
+  w.qa32 = off; off = align256(off + pooled / 2);
+  w.ka32 = off; off = align256(off + pooled / 2);
   if (want_bwd) { w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float)); }
   w.total = off;
   return w;
@@ -61,10 +63,10 @@ void record_error(nabla_status status, const char* fmt, ...);
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        cudaStream_t st);
-cudaError_t launch_select(const Dims& d, const double* qa, const double* ka, float thr,
-                          const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          cudaStream_t st);
+                        float* qa32, float* ka32, cudaStream_t st);
+cudaError_t launch_select(const Dims& d, const float* qa32, const float* ka32, const double* qa,
+                          const double* ka, float thr, const nabla_sta* sta, uint32_t* bits,
+                          int32_t* cnt, int32_t* idx, cudaStream_t st);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
                                    int32_t* idx, cudaStream_t st);
 cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,

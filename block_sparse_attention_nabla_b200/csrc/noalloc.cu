@@ -19,7 +19,7 @@
 namespace nabla {
 namespace {
 
-// 32 MiB: a 256-byte header (status word) and the fp64 pooled vectors.
+// 32 MiB: a 256-byte header (status word) and the pooled vectors (fp64 and fp32).
 constexpr size_t kNoAllocScratchBytes = 32u << 20;
 constexpr int kMaxDevices = 64;
 
@@ -101,7 +101,7 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (L.total > kNoAllocScratchBytes) {
     record_error(NABLA_ERR_UNSUPPORTED,
                  "this shape needs %zu bytes of scratch; the static scratch of "
-                 "nabla_build_mask_noalloc holds %zu (B * H * ceil(S / 64) * D * 16 bytes must fit); "
+                 "nabla_build_mask_noalloc holds %zu (B * H * ceil(S / 64) * D * 24 bytes must fit); "
                  "use nabla_build_mask with a workspace",
                  L.total, kNoAllocScratchBytes);
     return NABLA_ERR_UNSUPPORTED;
@@ -112,9 +112,12 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)scratch;
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);  // the status word starts at zero
-  if (e == cudaSuccess) e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), st);
   if (e == cudaSuccess)
-    e = launch_select(d, (const double*)(ws + L.qa), (const double*)(ws + L.ka), thr, sta, out->bits,
+    e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), (float*)(ws + L.qa32),
+                    (float*)(ws + L.ka32), st);
+  if (e == cudaSuccess)
+    e = launch_select(d, (const float*)(ws + L.qa32), (const float*)(ws + L.ka32),
+                      (const double*)(ws + L.qa), (const double*)(ws + L.ka), thr, sta, out->bits,
                       out->cnt, out->idx, st);
   if (e == cudaSuccess && out->cnt_t) e = launch_transpose_lists(d, out->bits, out->cnt_t, out->idx_t, st);
   if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);

@@ -135,7 +135,7 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
  *   builder's scratch (status word, pooled Qa / Ka) lives in a 32 MiB static
  *   device array inside the library, held by every GPU that loads it until the
  *   process exits.  Shapes whose scratch exceeds it (B * H * ceil(S / 64) * D *
- *   16 bytes plus 256 must fit in 32 MiB) are rejected with
+ *   24 bytes plus about 1 KB must fit in 32 MiB) are rejected with
  *   NABLA_ERR_UNSUPPORTED and a message naming both sizes.
  *   The first call on a device looks up the array's device address with that
  *   device current (cudaGetSymbolAddress) and caches it; make that first call
