@@ -38,8 +38,8 @@ THR = 0.8
 # reported only while the source is unchanged.  Filled from the summaries
 # under profiles/.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_tc_720p_h4.md: 414.6 MB at 4 heads, scaled x10 to 40 heads
-    "attn_fwd_tc.cu": ("92ae18f6fe1958b66d79b364e05037f110319ff6d937278f252b0a6e1a1401a3", 4.146e9),
+    # profiles/attn_fwd_tc_720p_h4.md: 384.5 MB at 4 heads, scaled x10 to 40 heads
+    "attn_fwd_tc.cu": ("0734e8f110d062fb5c8406a20afd0b88308bd08823007decee15d46f9fed8278", 3.845e9),
 }
 
 
