@@ -31,6 +31,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "NABLA attn ms/call + achieved TFLOP/s at S=75,600, H=40, D=128 bf16; mask-build GB/s"
 WORKLOAD_ID = 3
+# kernels of this library per step: pool, score GEMM, select, work list
+# (mask builder, no CSC transpose) and the attention forward
+LAUNCHES_PER_STEP = 5
 THR = 0.8
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
@@ -315,7 +318,7 @@ def main() -> None:
                          "traffic": _traffic("attn_fwd_tc.cu"),
                          "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -169,11 +169,16 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const voi
   char* ws = (char*)workspace;
   double* qa = (double*)(ws + L.qa);
   double* ka = (double*)(ws + L.ka);
-  float* qa32 = (float*)(ws + L.qa32);
-  float* ka32 = (float*)(ws + L.ka32);
+  float* qhi = (float*)(ws + L.qhi);
+  float* qlo = (float*)(ws + L.qlo);
+  float* khi = (float*)(ws + L.khi);
+  float* klo = (float*)(ws + L.klo);
+  float* logits = (float*)(ws + L.logits);
   NABLA_TRY(reset_status(workspace, st));
-  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qa32, ka32, st), "pooling kernel");
-  NABLA_CUDA(launch_select(d, qa32, ka32, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st),
+  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, st), "pooling kernel");
+  NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, (int32_t*)workspace + kWsStatus, st),
+             "score GEMM kernel");
+  NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st),
              "select kernel");
   return emit_derived(d, out->bits, out, st);
 }

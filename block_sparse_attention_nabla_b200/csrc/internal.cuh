@@ -26,12 +26,14 @@ inline Dims make_dims(const nabla_shape& s) {
   return d;
 }
 
-// Workspace layout: a 256-byte header (status word, scheduler counters), then
-// the pooled Qa / Ka in fp64 and rounded to fp32 ([B, H, nb, D] each) and,
-// for the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]).
+// Workspace layout: a 256-byte header (status word, scheduler counters), the
+// pooled Qa / Ka in fp64 and as tf32 hi / lo pairs ([B, H, nb, D] each), the
+// reduced logits L (fp32 [B, H, nb, ldl], ldl = nb rounded up to 4) and, for
+// the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]).
 struct WsLayout {
   size_t header = 0;
-  size_t qa = 0, ka = 0, qa32 = 0, ka32 = 0, delta = 0;
+  size_t qa = 0, ka = 0, qhi = 0, qlo = 0, khi = 0, klo = 0, logits = 0, delta = 0;
+  int ldl = 0;
   size_t total = 0;
 };
 
@@ -43,8 +45,12 @@ inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
   size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(double);
   w.qa = off; off = align256(off + pooled);
   w.ka = off; off = align256(off + pooled);
-  w.qa32 = off; off = align256(off + pooled / 2);
-  w.ka32 = off; off = align256(off + pooled / 2);
+  w.qhi = off; off = align256(off + pooled / 2);
+  w.qlo = off; off = align256(off + pooled / 2);
+  w.khi = off; off = align256(off + pooled / 2);
+  w.klo = off; off = align256(off + pooled / 2);
+  w.ldl = (d.nb + 3) & ~3;
+  w.logits = off; off = align256(off + (size_t)d.BH() * d.nb * w.ldl * sizeof(float));
   if (want_bwd) { w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float)); }
   w.total = off;
   return w;
@@ -63,10 +69,12 @@ void record_error(nabla_status status, const char* fmt, ...);
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        float* qa32, float* ka32, cudaStream_t st);
-cudaError_t launch_select(const Dims& d, const float* qa32, const float* ka32, const double* qa,
-                          const double* ka, float thr, const nabla_sta* sta, uint32_t* bits,
-                          int32_t* cnt, int32_t* idx, cudaStream_t st);
+                        float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st);
+cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
+                              const float* klo, float* L, int ldl, int32_t* status, cudaStream_t st);
+cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
+                          float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                          cudaStream_t st);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
                                    int32_t* idx, cudaStream_t st);
 cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,

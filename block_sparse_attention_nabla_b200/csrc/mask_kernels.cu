@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include "internal.cuh"
+#include "sm100.cuh"
 
 namespace nabla {
 namespace {
@@ -73,12 +74,14 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // one 16-byte column chunk and sums its rows in fp64 from 16-byte loads, eight
 // loads in flight per lane; lanes that hold the same chunk for different rows
 // are combined by shuffles.  The means are written in fp64 (the selection
-// ranks near-equal entries by fp64 logits) and rounded to fp32 (operands of
-// the score GEMM).  The tail block divides by its number of valid tokens.
+// ranks near-equal entries by fp64 logits) and as a pair of fp32 values
+// hi + lo with hi the nearest tf32 value (operands of the tensor-core score
+// GEMM).  The tail block divides by its number of valid tokens.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                    double* __restrict__ qa, double* __restrict__ ka,
-                                                   float* __restrict__ qa32, float* __restrict__ ka32,
+                                                   float* __restrict__ qhi, float* __restrict__ qlo,
+                                                   float* __restrict__ khi, float* __restrict__ klo,
                                                    int S, int nb, long long per_tensor) {
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte chunk
   constexpr int CH = D / VE;          // chunks per row (8, 16 or 32)
@@ -123,61 +126,85 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
       for (int e = 0; e < VE; ++e) acc[e] += __shfl_xor_sync(kFull, acc[e], off);
     if (lane < CH) {
       double* dst = (isk ? ka : qa) + it * D + c * VE;
-      float* dst32 = (isk ? ka32 : qa32) + it * D + c * VE;
+      float* dhi = (isk ? khi : qhi) + it * D + c * VE;
+      float* dlo = (isk ? klo : qlo) + it * D + c * VE;
 #pragma unroll
       for (int e = 0; e < VE; ++e) {
         const double mean = acc[e] / (double)valid;
+        const float f = (float)mean;
+        const float h = sm100::to_tf32(f);
         dst[e] = mean;
-        dst32[e] = (float)mean;
+        dhi[e] = h;
+        dlo[e] = f - h;
       }
     }
   }
 }
 
-// ------------------------------------------------------------ score + select
-// One CTA handles R query blocks of one (b, h).
-//   phase 1: L[r][j] = (Qa_r . Ka_j) * (1/sqrt(D)) in fp32 from the fp32
-//            pooled vectors, staged in shared memory (the map is never written
-//            to HBM); Ka chunks are double-buffered with cp.async;
-//   phase 2: one warp per row: max, e_j = exp(L_j - max), s = sum e_j.  Block
-//            j is kept iff the mass of the entries ranked above it is
-//            <= thr * s: Algorithm 1's ascending cumulative sum compared with
-//            1 - thr, stated through the mass above each entry.  The fp32
-//            cut-off is the smallest float bit pattern u with
-//            sum_{e_k > u} e_k <= thr * s (binary search; positive floats
-//            order like their bit patterns).  fp32 cannot order entries whose
-//            values differ by less than its rounding error, so the entries
-//            within a relative 2^-12 of the cut-off value are ranked again by
-//            their fp64 logits (ties: higher block index first, as a stable
-//            ascending sort leaves them) and kept in rank order while the mass
-//            above them stays <= thr * s;
-//   then OR the STA window and emit bits / cnt / idx.
-// The row's values live in registers (NPL per lane, nb <= 32 NPL) during the
-// search, else in shared memory.
-constexpr float kWindow = 1.0f / 4096.0f;
+// ------------------------------------------------------------------ select
+// One warp per row of the reduced map (one query block of one (b, h)); the
+// logits L[i][j] = (Qa_i . Ka_j) / sqrt(D) come from the tensor-core score
+// GEMM (score_tc.cu).  Per row: max, e_j = exp(L_j - max), s = sum e_j.  Block
+// j is kept iff the mass of the entries ranked above it is <= thr * s:
+// Algorithm 1's ascending cumulative sum compared with 1 - thr, stated through
+// the mass above each entry.  The fp32 cut-off is the smallest float bit
+// pattern u with sum_{e_k > u} e_k <= thr * s (binary search; positive floats
+// order like their bit patterns), taken on the top 16 bits: the cut-off
+// bucket is the smallest 16-bit prefix p with sum_{prefix(e_k) > p} e_k <=
+// thr * s.  Entries above the bucket are kept, entries below dropped, and the
+// entries of the bucket (relative width <= 2^-7, typically a handful) are
+// ranked by their fp64 logits (ties: higher block index first, as a stable
+// ascending sort leaves them; fp32 cannot order entries closer than its
+// rounding error) and kept in rank order while the mass above them stays
+// <= thr * s.  Then the STA window is OR-ed in and bits / cnt / idx are
+// written.  The row's values live in registers (NPL per lane, nb <= 32 NPL),
+// else in the logits buffer.
 constexpr int kMaxCand = 32;
-constexpr int KC = 32;  // Ka rows per GEMM chunk
 
 struct SelectCtx {
   const double* qa_h;
   const double* ka_h;
   int nb, W;
   float thr;
-  const int* Ct;
-  const int* Cy;
-  const int* Cx;
-  bool use_sta;
+  const int32_t* coords;  // [nb][3] or null
   int hT, hH, hW;
   int (*cand_j)[kMaxCand];
   float (*cand_e)[kMaxCand];
 };
 
+// fp64 logits Qa_row . Ka_j (unscaled: a positive factor keeps the order) of
+// the n <= 32 candidates cand[0..n): one warp-wide dot product each, lane l
+// taking dimensions l, l + 32, ...; lane b returns candidate b's logit.  The
+// xor butterfly leaves the same sum in every lane.
 template <int D>
-__device__ __forceinline__ double logit64(const double* qrow, const double* krow) {
-  double dot = 0.0;
-#pragma unroll 8
-  for (int d = 0; d < D; ++d) dot = fma(qrow[d], krow[d], dot);
-  return dot;
+__device__ __forceinline__ double candidate_logits(const double* __restrict__ qrow,
+                                                   const double* __restrict__ ka_h, const int* cand, int n,
+                                                   int lane) {
+  constexpr int VD = D / 32;
+  double qv[VD];
+#pragma unroll
+  for (int v = 0; v < VD; ++v) qv[v] = qrow[lane + 32 * v];
+  double mine = -1e300;
+  for (int b0 = 0; b0 < n; b0 += 4) {
+    double part[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      part[u] = 0.0;
+      if (b0 + u < n) {
+        const double* krow = ka_h + (long long)cand[b0 + u] * D;
+#pragma unroll
+        for (int v = 0; v < VD; ++v) part[u] = fma(qv[v], krow[lane + 32 * v], part[u]);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) part[u] += __shfl_xor_sync(kFull, part[u], off);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (lane == b0 + u) mine = part[u];
+  }
+  return mine;
 }
 
 // Warp-wide selection of one row.  NPL > 0: the row's exponentials live in
@@ -214,39 +241,47 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   }
   s = warp_sum(s);
   const float limit = c.thr * s;
-  // e_max = exp(0) = 1, so every entry's bit pattern is <= 0x3F800000 and
-  // the mass strictly above 0x3F800001 is 0 <= limit.
-  uint32_t lo = 0u, hi = 0x3F800001u;
-  while (lo < hi) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    float f = 0.f;
+  // Mass of the entries whose bit pattern, shifted right by `sh`, exceeds u:
+  // for e >= 0 that is e > the float whose pattern is u's bucket top.
+  auto mass_above = [&](uint32_t u, int sh) -> float {
+    const float tv = __uint_as_float((u << sh) | ((1u << sh) - 1u));
+    float f0 = 0.f, f1 = 0.f;
     if constexpr (NPL > 0) {
 #pragma unroll
-      for (int t = 0; t < NPL; ++t) f += __float_as_uint(ev[t]) > mid ? ev[t] : 0.f;
+      for (int t = 0; t < NPL; t += 2) {
+        if (ev[t] > tv) f0 += ev[t];
+        if (t + 1 < NPL && ev[t + 1] > tv) f1 += ev[t + 1];
+      }
     } else {
       for (int j = lane; j < nb; j += 32) {
         const float e = Lr[j];
-        f += __float_as_uint(e) > mid ? e : 0.f;
+        if (e > tv) f0 += e;
       }
     }
-    f = warp_sum(f);
-    if (f <= limit) hi = mid; else lo = mid + 1u;
+    return warp_sum(f0 + f1);
+  };
+  // Binary search over the top 16 bits of the pattern: the smallest prefix p
+  // whose strictly higher prefixes hold mass <= limit.  e_max = 1 has prefix
+  // 0x3F80, so the mass above prefix 0x3F80 is 0.  Entries above the cut-off
+  // bucket (prefix > p) are kept and entries below it dropped; the entries
+  // of bucket p are ranked below.  p == 0 means every block is kept.
+  uint32_t lo = 0u, hi = 0x3F80u;
+  while (lo < hi) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (mass_above(mid, 16) <= limit) hi = mid; else lo = mid + 1u;
   }
-
-  // Decision: keep everything if lo == 0; otherwise keep e > vhi, drop
-  // e < vlo, and settle the candidates in [vlo, vhi] by fp64 rank (or by the
-  // fp32 rule bits(e) >= lo when there are more than kMaxCand of them).
-  const float vcut = __uint_as_float(lo);
-  const float vhi = vcut * (1.f + kWindow), vlo = vcut * (1.f - kWindow);
-  int mode = lo == 0u ? 0 : 1;  // 0 keep all, 1 ranked candidates, 2 fp32 rule
-  uint64_t keepbits = 0;        // register path: ranked-candidate decisions by t
+  const uint32_t pcut = lo;
+  int mode = pcut == 0u ? 0 : 1;  // 0 keep all, 1 ranked bucket, 2 fp32 rule at bits >= cut32
+  uint32_t cut32 = 0u;
+  uint64_t keepbits = 0;          // register path: ranked-candidate decisions by t
   if (mode == 1) {
     float above = 0.f;
     int ncand = 0;
     auto visit = [&](int t, float e) {
       const int j = t * 32 + lane;
-      above += e > vhi ? e : 0.f;
-      const bool isc = j < nb && e >= vlo && e <= vhi;
+      const uint32_t pre = __float_as_uint(e) >> 16;
+      above += pre > pcut ? e : 0.f;
+      const bool isc = j < nb && pre == pcut;
       const uint32_t word = __ballot_sync(kFull, isc);
       const int slot = ncand + __popc(word & lanemask_lt());
       if (isc && slot < kMaxCand) {
@@ -265,12 +300,20 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
     above = warp_sum(above);
     __syncwarp();
     if (ncand > kMaxCand) {
+      // too many entries in one bucket to rank at once: finish the search on
+      // the low 16 bits and keep the fp32 decision bits(e) >= cut32
+      uint32_t l2 = pcut << 16, h2 = (pcut << 16) | 0xFFFFu;
+      while (l2 < h2) {
+        const uint32_t mid = l2 + ((h2 - l2) >> 1);
+        if (mass_above(mid, 0) <= limit) h2 = mid; else l2 = mid + 1u;
+      }
+      cut32 = l2;
       mode = 2;
     } else {
       const bool act = lane < ncand;
       const int cj = act ? c.cand_j[warp][lane] : 0;
       const float ce = act ? c.cand_e[warp][lane] : 0.f;
-      const double lg = act ? logit64<D>(c.qa_h + (long long)row * D, c.ka_h + (long long)cj * D) : -1e300;
+      const double lg = candidate_logits<D>(c.qa_h + (long long)row * D, c.ka_h, c.cand_j[warp], ncand, lane);
       float mass = above;
       for (int b2 = 0; b2 < ncand; ++b2) {
         const double lb = __shfl_sync(kFull, lg, b2);
@@ -283,12 +326,13 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
       const uint32_t kmask = __ballot_sync(kFull, kp);
       for (int b2 = 0; b2 < ncand; ++b2) {
         const int jb = __shfl_sync(kFull, cj, b2);
-        const bool kb = (kmask >> b2) & 1u;
-        if (kb && (jb & 31) == lane) {
-          if constexpr (NPL > 0) keepbits |= 1ull << (jb >> 5);
-          else Lr[jb] = 2.f;  // > vhi: kept by the emission rule below
-        } else if (!kb && (jb & 31) == lane) {
-          if constexpr (NPL == 0) Lr[jb] = 0.f;
+        if ((jb & 31) == lane) {
+          const bool kb = (kmask >> b2) & 1u;
+          if constexpr (NPL > 0) {
+            if (kb) keepbits |= 1ull << (jb >> 5);
+          } else {
+            Lr[jb] = kb ? 2.f : 0.f;  // 2 sits in a bucket above any e <= 1
+          }
         }
       }
       __syncwarp();
@@ -296,16 +340,19 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   }
 
   int running = 0;
-  const int ti = c.use_sta ? c.Ct[row] : 0, yi = c.use_sta ? c.Cy[row] : 0, xi = c.use_sta ? c.Cx[row] : 0;
+  const bool use_sta = c.coords != nullptr;
+  const int ti = use_sta ? c.coords[3 * row] : 0, yi = use_sta ? c.coords[3 * row + 1] : 0,
+            xi = use_sta ? c.coords[3 * row + 2] : 0;
   auto emit = [&](int t, float e, bool ranked_keep) {
     const int j = t * 32 + lane;
     bool keep = false;
     if (j < nb) {
       if (mode == 0) keep = true;
-      else if (mode == 1) keep = e > vhi || ranked_keep;
-      else keep = __float_as_uint(e) >= lo;
-      if (c.use_sta && !keep)
-        keep = abs(c.Ct[j] - ti) <= c.hT && abs(c.Cy[j] - yi) <= c.hH && abs(c.Cx[j] - xi) <= c.hW;
+      else if (mode == 1) keep = (__float_as_uint(e) >> 16) > pcut || ranked_keep;
+      else keep = __float_as_uint(e) >= cut32;
+      if (use_sta && !keep)
+        keep = abs(c.coords[3 * j] - ti) <= c.hT && abs(c.coords[3 * j + 1] - yi) <= c.hH &&
+               abs(c.coords[3 * j + 2] - xi) <= c.hW;
     }
     const uint32_t word = __ballot_sync(kFull, keep);
     if (lane == 0) brow[t] = word;
@@ -322,117 +369,37 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   if (lane == 0) *cntp = running;
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-template <int R, int D>
-__global__ void __launch_bounds__(256, 1) select_kernel(
-    const float* __restrict__ qa32, const float* __restrict__ ka32, const double* __restrict__ qa,
-    const double* __restrict__ ka, int nb, int W, int ldl, float thr, float scale,
-    const int32_t* __restrict__ coords, int hT, int hH, int hW, uint32_t* __restrict__ bits,
-    int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
-  extern __shared__ float4 smem4[];
-  constexpr int LD = D + 4;  // padded Qa/Ka row: LD / 4 is odd -> conflict-free float4 rows
-  constexpr int RG = R / 2;  // row pairs
-  constexpr int CT = 256 / RG;
-  constexpr int CPT = KC / CT > 0 ? KC / CT : 1;
+template <int D, int NPL>
+__global__ void __launch_bounds__(256) select_rows_kernel(
+    const float* __restrict__ L, int ldl, const double* __restrict__ qa, const double* __restrict__ ka,
+    long long rows, int nb, int W, float thr, const int32_t* __restrict__ coords, int hT, int hH, int hW,
+    uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
   __shared__ int cand_j[8][kMaxCand];
   __shared__ float cand_e[8][kMaxCand];
-  float* Ls = reinterpret_cast<float*>(smem4);
-  float* Qs = Ls + R * ldl;
-  float* Ks = Qs + R * LD;  // two buffers of KC rows
-  int* Ct = reinterpret_cast<int*>(Ks + 2 * KC * LD);
-  int* Cy = Ct + nb;
-  int* Cx = Cy + nb;
-  const bool use_sta = coords != nullptr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long grow = (long long)blockIdx.x * 8 + warp;  // (b * H + h) * nb + i
+  if (grow >= rows) return;
+  const long long bh = grow / nb;
+  const int row = (int)(grow - bh * nb);
+  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, coords, hT, hH, hW, cand_j, cand_e};
+  float* Lr = const_cast<float*>(L) + grow * ldl;
+  uint32_t* brow = bits + grow * W;
+  int32_t* irow = idx + grow * nb;
+  select_row<D, NPL>(ctx, Lr, row, brow, irow, cnt + grow, warp, lane);
+}
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long bh = blockIdx.y;
-  const int row0 = blockIdx.x * R;
-  const float* qa_h = qa32 + bh * nb * D;
-  const float* ka_h = ka32 + bh * nb * D;
-
-  auto load_chunk = [&](int c0, int buf) {
-    float* dstb = Ks + buf * KC * LD;
-    for (int e = tid; e < KC * (D / 4); e += 256) {
-      const int r = e / (D / 4), c4 = e % (D / 4);
-      const bool ok = c0 + r < nb;
-      const float* src = ka_h + (long long)(ok ? c0 + r : 0) * D + c4 * 4;
-      cp_async16(dstb + r * LD + c4 * 4, src, ok);
-    }
-    cp_async_commit();
-  };
-
-  for (int e = tid; e < R * (D / 4); e += 256) {
-    const int r = e / (D / 4), c4 = e % (D / 4);
-    const bool ok = row0 + r < nb;
-    cp_async16(Qs + r * LD + c4 * 4, qa_h + (long long)(ok ? row0 + r : 0) * D + c4 * 4, ok);
-  }
-  load_chunk(0, 0);
-  if (use_sta)
-    for (int j = tid; j < nb; j += 256) {
-      Ct[j] = coords[3 * j];
-      Cy[j] = coords[3 * j + 1];
-      Cx[j] = coords[3 * j + 2];
-    }
-
-  const int tr = tid / CT, tc = tid % CT;
-  for (int c0 = 0, buf = 0; c0 < nb; c0 += KC, buf ^= 1) {
-    cp_async_wait_all();
-    __syncthreads();
-    if (c0 + KC < nb) load_chunk(c0 + KC, buf ^ 1);
-    const float* Kb = Ks + buf * KC * LD;
-    float acc0[CPT], acc1[CPT];
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) acc0[j] = acc1[j] = 0.f;
-    if (tc < KC) {
-#pragma unroll 4
-      for (int kk = 0; kk < D; kk += 4) {
-        const float4 a0 = *reinterpret_cast<const float4*>(Qs + (2 * tr) * LD + kk);
-        const float4 a1 = *reinterpret_cast<const float4*>(Qs + (2 * tr + 1) * LD + kk);
-#pragma unroll
-        for (int j = 0; j < CPT; ++j) {
-          const float4 bv = *reinterpret_cast<const float4*>(Kb + (tc + CT * j) * LD + kk);
-          acc0[j] = fmaf(a0.x, bv.x, acc0[j]);
-          acc0[j] = fmaf(a0.y, bv.y, acc0[j]);
-          acc0[j] = fmaf(a0.z, bv.z, acc0[j]);
-          acc0[j] = fmaf(a0.w, bv.w, acc0[j]);
-          acc1[j] = fmaf(a1.x, bv.x, acc1[j]);
-          acc1[j] = fmaf(a1.y, bv.y, acc1[j]);
-          acc1[j] = fmaf(a1.z, bv.z, acc1[j]);
-          acc1[j] = fmaf(a1.w, bv.w, acc1[j]);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        const int col = c0 + tc + CT * j;
-        if (col < nb) {
-          Ls[(2 * tr) * ldl + col] = acc0[j] * scale;
-          Ls[(2 * tr + 1) * ldl + col] = acc1[j] * scale;
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, Ct, Cy, Cx, use_sta, hT, hH, hW, cand_j, cand_e};
-  for (int r = warp; r < R; r += 8) {
-    const int row = row0 + r;
-    if (row >= nb) break;
-    float* Lr = Ls + r * ldl;
-    const long long grow = bh * nb + row;
-    uint32_t* brow = bits + grow * W;
-    int32_t* irow = idx + grow * nb;
-    if (W <= 16) select_row<D, 16>(ctx, Lr, row, brow, irow, cnt + grow, warp, lane);
-    else if (W <= 40) select_row<D, 40>(ctx, Lr, row, brow, irow, cnt + grow, warp, lane);
-    else if (W <= 64) select_row<D, 64>(ctx, Lr, row, brow, irow, cnt + grow, warp, lane);
-    else select_row<D, 0>(ctx, Lr, row, brow, irow, cnt + grow, warp, lane);
-  }
+template <int D>
+void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl, const double* qa,
+                        const double* ka, long long rows, int nb, int W, float thr, const int32_t* coords,
+                        int hT, int hH, int hW, uint32_t* bits, int32_t* cnt, int32_t* idx) {
+  // registers per lane hold ceil(nb / 32) values, rounded up to a few sizes
+  auto k = W <= 8 ? select_rows_kernel<D, 8>
+         : W <= 16 ? select_rows_kernel<D, 16>
+         : W <= 24 ? select_rows_kernel<D, 24>
+         : W <= 40 ? select_rows_kernel<D, 40>
+         : W <= 64 ? select_rows_kernel<D, 64>
+                   : select_rows_kernel<D, 0>;
+  k<<<grid, 256, 0, st>>>(L, ldl, qa, ka, rows, nb, W, thr, coords, hT, hH, hW, bits, cnt, idx);
 }
 
 // ------------------------------------------------------ lists from a bitmask
@@ -542,67 +509,40 @@ int num_sms() {
 
 constexpr size_t kSmemLimit = 227 * 1024 - 4096;  // dynamic part; the kernel also has ~2 KB static
 
-template <int R, int D>
-size_t select_smem(int nb, int ldl) {
-  return sizeof(float) * ((size_t)R * ldl + (size_t)R * (D + 4) + 2 * KC * (D + 4)) + 3 * sizeof(int) * nb;
-}
-
-template <int R, int D>
-cudaError_t run_select(const Dims& d, const float* qa32, const float* ka32, const double* qa,
-                       const double* ka, float thr, const nabla_sta* sta, uint32_t* bits,
-                       int32_t* cnt, int32_t* idx, cudaStream_t st, int ldl) {
-  const size_t smem = select_smem<R, D>(d.nb, ldl);
-  auto kern = select_kernel<R, D>;
-  cudaError_t e = set_smem(kern, smem);
-  if (e != cudaSuccess) return e;
-  const bool use_sta = sta && sta->block_coords;
-  dim3 grid((d.nb + R - 1) / R, (unsigned)d.BH());
-  kern<<<grid, 256, smem, st>>>(qa32, ka32, qa, ka, d.nb, d.W, ldl, thr, 1.0f / sqrtf((float)d.D),
-                                use_sta ? sta->block_coords : nullptr, use_sta ? sta->wT / 2 : 0,
-                                use_sta ? sta->wH / 2 : 0, use_sta ? sta->wW / 2 : 0, bits, cnt, idx);
-  return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t select_d(const Dims& d, const float* qa32, const float* ka32, const double* qa,
-                     const double* ka, float thr, const nabla_sta* sta, uint32_t* bits,
-                     int32_t* cnt, int32_t* idx, cudaStream_t st) {
-  const int ldl = (d.nb + 3) & ~3;
-  if (select_smem<32, D>(d.nb, ldl) <= kSmemLimit)
-    return run_select<32, D>(d, qa32, ka32, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
-  if (select_smem<16, D>(d.nb, ldl) <= kSmemLimit)
-    return run_select<16, D>(d, qa32, ka32, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
-  if (select_smem<8, D>(d.nb, ldl) <= kSmemLimit)
-    return run_select<8, D>(d, qa32, ka32, qa, ka, thr, sta, bits, cnt, idx, st, ldl);
-  return cudaErrorInvalidConfiguration;
-}
-
 }  // namespace
 
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        float* qa32, float* ka32, cudaStream_t st) {
+                        float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st) {
   const long long per = d.BH() * d.nb;
   const long long warps = 2 * per;
   const int grid = (int)std::min<long long>((warps + 7) / 8, (long long)num_sms() * 8);
   if (d.dtype == NABLA_BF16) {
     if (d.D == 128)
-      pool_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qa32, ka32, d.S, d.nb, per);
+      pool_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
     else
-      pool_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qa32, ka32, d.S, d.nb, per);
+      pool_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
   } else {
     if (d.D == 128)
-      pool_kernel<float, 128><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qa32, ka32, d.S, d.nb, per);
+      pool_kernel<float, 128><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
     else
-      pool_kernel<float, 64><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qa32, ka32, d.S, d.nb, per);
+      pool_kernel<float, 64><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const Dims& d, const float* qa32, const float* ka32, const double* qa,
-                          const double* ka, float thr, const nabla_sta* sta, uint32_t* bits,
-                          int32_t* cnt, int32_t* idx, cudaStream_t st) {
-  if (d.D == 128) return select_d<128>(d, qa32, ka32, qa, ka, thr, sta, bits, cnt, idx, st);
-  return select_d<64>(d, qa32, ka32, qa, ka, thr, sta, bits, cnt, idx, st);
+cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
+                          float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
+                          cudaStream_t st) {
+  const long long rows = d.BH() * d.nb;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const bool use_sta = sta && sta->block_coords;
+  const int32_t* coords = use_sta ? sta->block_coords : nullptr;
+  const int hT = use_sta ? sta->wT / 2 : 0, hH = use_sta ? sta->wH / 2 : 0, hW = use_sta ? sta->wW / 2 : 0;
+  if (d.D == 128)
+    launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, coords, hT, hH, hW, bits, cnt, idx);
+  else
+    launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, coords, hT, hH, hW, bits, cnt, idx);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt, int32_t* idx,

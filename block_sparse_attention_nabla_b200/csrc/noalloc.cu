@@ -19,7 +19,8 @@
 namespace nabla {
 namespace {
 
-// 32 MiB: a 256-byte header (status word) and the pooled vectors (fp64 and fp32).
+// 32 MiB: a 256-byte header (status word), the pooled vectors (fp64 and tf32
+// hi / lo pairs) and the reduced logits.
 constexpr size_t kNoAllocScratchBytes = 32u << 20;
 constexpr int kMaxDevices = 64;
 
@@ -101,7 +102,7 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (L.total > kNoAllocScratchBytes) {
     record_error(NABLA_ERR_UNSUPPORTED,
                  "this shape needs %zu bytes of scratch; the static scratch of "
-                 "nabla_build_mask_noalloc holds %zu (B * H * ceil(S / 64) * D * 24 bytes must fit); "
+                 "nabla_build_mask_noalloc holds %zu (B * H * nb * (32 D + 4 nb) bytes, nb = ceil(S / 64), must fit); "
                  "use nabla_build_mask with a workspace",
                  L.total, kNoAllocScratchBytes);
     return NABLA_ERR_UNSUPPORTED;
@@ -113,12 +114,15 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   char* ws = (char*)scratch;
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);  // the status word starts at zero
   if (e == cudaSuccess)
-    e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), (float*)(ws + L.qa32),
-                    (float*)(ws + L.ka32), st);
+    e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), (float*)(ws + L.qhi),
+                    (float*)(ws + L.qlo), (float*)(ws + L.khi), (float*)(ws + L.klo), st);
   if (e == cudaSuccess)
-    e = launch_select(d, (const float*)(ws + L.qa32), (const float*)(ws + L.ka32),
-                      (const double*)(ws + L.qa), (const double*)(ws + L.ka), thr, sta, out->bits,
-                      out->cnt, out->idx, st);
+    e = launch_score_gemm(d, (const float*)(ws + L.qhi), (const float*)(ws + L.qlo),
+                          (const float*)(ws + L.khi), (const float*)(ws + L.klo), (float*)(ws + L.logits),
+                          L.ldl, (int32_t*)ws + kWsStatus, st);
+  if (e == cudaSuccess)
+    e = launch_select(d, (const float*)(ws + L.logits), L.ldl, (const double*)(ws + L.qa),
+                      (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, st);
   if (e == cudaSuccess && out->cnt_t) e = launch_transpose_lists(d, out->bits, out->cnt_t, out->idx_t, st);
   if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);
   if (e != cudaSuccess) {

@@ -132,10 +132,11 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
  * an allocation can cause).  The paper has no counterpart: this is a packaging
  * variant of nabla_build_mask.
  *   Same arguments and results as nabla_build_mask, without the workspace: the
- *   builder's scratch (status word, pooled Qa / Ka) lives in a 32 MiB static
- *   device array inside the library, held by every GPU that loads it until the
- *   process exits.  Shapes whose scratch exceeds it (B * H * ceil(S / 64) * D *
- *   24 bytes plus about 1 KB must fit in 32 MiB) are rejected with
+ *   builder's scratch (status word, pooled Qa / Ka, reduced logits) lives in a
+ *   32 MiB static device array inside the library, held by every GPU that
+ *   loads it until the process exits.  Shapes whose scratch exceeds it
+ *   (B * H * nb * (32 D + 4 nb) bytes plus about 2 KB must fit in 32 MiB,
+ *   nb = ceil(S / 64)) are rejected with
  *   NABLA_ERR_UNSUPPORTED and a message naming both sizes.
  *   The first call on a device looks up the array's device address with that
  *   device current (cudaGetSymbolAddress) and caches it; make that first call

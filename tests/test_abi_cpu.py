@@ -58,7 +58,8 @@ def test_workspace_size_formula(L):
     for (B, H, S, D) in [(1, 2, 4096, 64), (1, 40, 75600, 128), (2, 16, 16384, 128), (1, 1, 1, 64)]:
         nb = -(-S // 64)
         pooled = align(B * H * nb * D * 8)
-        fwd = 256 + 2 * pooled + 2 * align(B * H * nb * D * 4)
+        ldl = (nb + 3) // 4 * 4
+        fwd = 256 + 2 * pooled + 4 * align(B * H * nb * D * 4) + align(B * H * nb * ldl * 4)
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 0) == fwd
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 1) == fwd + align(B * H * S * 4)
 
