@@ -188,6 +188,66 @@ def run_reference(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def measure_training(dev, warmup: int, steps: int) -> dict:
+    """The training leg: mask (with the transposed lists), forward and backward
+    at the pretraining shape (B=2, H=16, S=16,384, D=128, bf16, thr 0.8), each
+    timed with CUDA events on the launching stream.  Backward flops are the
+    algorithmic 10 * 64 * 64 * D per kept tile (five GEMMs)."""
+    import torch
+
+    import block_sparse_attention_nabla_b200 as nabla
+    import synth
+    w = synth.WORKLOADS[4]
+    x = synth.make_inputs(w)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, H, S, D = q.shape
+    ws = nabla.workspace(q, want_bwd=True)
+    mask = nabla.Mask.empty(B, H, S, dev, transpose=True)
+    o, lse = torch.empty_like(q), torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        nabla.build_mask(q, k, w.thresholds[0], out=mask, ws=ws, transpose=True)
+        if ev:
+            ev[1].record(stream)
+        nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+        if ev:
+            ev[2].record(stream)
+        nabla.attn_bwd(q, k, v, o, do, lse, mask, dq=dq, dk=dk, dv=dv, ws=ws)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    if nabla.workspace_status(ws) != 0:
+        raise SystemExit("device status word reports a timeout in the training leg")
+    mask_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    kept = int(mask.cnt.to(torch.int64).sum().item())
+    nb = mask.cnt.shape[-1]
+    peaks = _peaks()
+    bwd_tflops = kept * 10 * 64 * 64 * D / (bwd_ms * 1e-3) / 1e12
+    fwd_tflops = kept * 4 * 64 * 64 * D / (fwd_ms * 1e-3) / 1e12
+    return {"workload": f"{w.name}: B={B} H={H} S={S} D={D} bf16, thr {w.thresholds[0]}, fwd + bwd with dO",
+            "kept_fraction": kept / (B * H * nb * nb), "kept_tiles": kept, "steps": steps,
+            "mask_ms": mask_ms, "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops,
+            "bwd_ms": bwd_ms, "bwd_tflops": bwd_tflops,
+            "bwd_roofline": {"bound": "tensor", "kernels": "bwd_stats + dkdv_tc + dq_tc (attn_bwd_tc.cu)",
+                             "achieved": bwd_tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                             "frac": bwd_tflops / peaks["bf16_sus"],
+                             "algorithmic": "kept tiles x 10*64*64*D flops per call (executed: 14*64*64*D)"},
+            "gpu_launches_per_step": 9}
+
+
 def _config(w, n) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16, {w.T}x{w.Hl}x{w.Wl} tokens, "
                         f"thr {THR}, no STA",
@@ -205,6 +265,9 @@ def main() -> None:
     ap.add_argument("--impl", default="nabla", choices=["nabla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-training", action="store_true", help="skip the forward + backward training leg")
+    ap.add_argument("--only-training", action="store_true",
+                    help="run only the training leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the head count (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
@@ -218,6 +281,12 @@ def main() -> None:
 
     import block_sparse_attention_nabla_b200 as nabla
     import synth
+
+    if args.only_training:
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_training(torch.device("cuda", 0), args.warmup, max(1, args.steps))), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -301,6 +370,10 @@ def main() -> None:
     if not args.no_e2e:
         e2e = run_e2e(nabla, q, k, v, o, lse, mask, ws, stream, args, world, dist, dev, flops)
 
+    training = None
+    if world == 1 and not args.no_training:
+        training = measure_training(dev, args.warmup, max(1, min(args.steps, 5)))
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -318,6 +391,7 @@ def main() -> None:
                          "traffic": _traffic("attn_fwd_tc.cu"),
                          "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
             "e2e": e2e,
+            "training": training,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }

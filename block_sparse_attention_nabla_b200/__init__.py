@@ -250,11 +250,14 @@ def attn_fwd(q, k, v, mask: Mask, o=None, lse=None, ws=None):
     return o, lse
 
 
-def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None):
+def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None, dq=None, dk=None, dv=None):
     """Backward of attn_fwd under the same mask; returns (dq, dk, dv)."""
     sh = _shape_of(q)
     _same(q, k, v, o, do)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq = dq if dq is not None else torch.empty_like(q)
+    dk = dk if dk is not None else torch.empty_like(k)
+    dv = dv if dv is not None else torch.empty_like(v)
+    _same(q, dq, dk, dv)
     ws = ws if ws is not None else workspace(q, want_bwd=True)
     ms = mask.as_struct()
     _check(lib().nabla_attn_bwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),

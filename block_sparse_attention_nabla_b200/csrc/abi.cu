@@ -244,9 +244,16 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   cudaStream_t st = (cudaStream_t)stream;
   const WsLayout L = ws_layout(d, true);
   NABLA_TRY(reset_status(workspace, st));
-  NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
-                                  mask->idx_t, (float*)((char*)workspace + L.delta), dq, dk, dv, st),
-             "attention backward");
+  char* ws = (char*)workspace;
+  if (d.dtype == NABLA_BF16 && d.D == 128)
+    NABLA_CUDA(launch_attn_bwd_tc(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t, mask->idx_t,
+                                  (float*)(ws + L.lse2p), (float*)(ws + L.deltap), dq, dk, dv,
+                                  (int32_t*)ws, st),
+               "tensor-core attention backward");
+  else
+    NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
+                                    mask->idx_t, (float*)(ws + L.delta), dq, dk, dv, st),
+               "attention backward");
   return NABLA_OK;
 }
 

@@ -442,49 +442,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(status, 0, (int32_t)NABLA_ERR_TIMEOUT);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult qr;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-  }
-  return fn;
-}
-
-// 3-D view {D, S, B*H} of a [B, H, S, D] bf16 tensor; box {64, rows, 1};
-// 128-byte swizzle; rows beyond S read as zero.
-bool make_map(CUtensorMap* map, const void* base, const Dims& d, int rows) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d.D, (cuuint64_t)d.S, (cuuint64_t)d.BH()};
-  cuuint64_t strides[2] = {(cuuint64_t)d.D * 2, (cuuint64_t)d.S * d.D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int D>
 cudaError_t run(const Dims& d, const void* q, const void* k, const void* v, const uint32_t* bits,
                 const int32_t* work, void* o, float* lse, int32_t* ws_header, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, d, 128) || !make_map(&tk, k, d, 64) || !make_map(&tv, v, d, 64))
+  if (!make_map_bf16(&tq, q, d, 128) || !make_map_bf16(&tk, k, d, 64) || !make_map_bf16(&tv, v, d, 64))
     return cudaErrorInvalidValue;
   const int n_units = (int)(d.BH() * d.npairs);
   const int grid = std::min(n_units, kCtasPerSm * sm_count());

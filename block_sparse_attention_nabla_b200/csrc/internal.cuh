@@ -1,6 +1,7 @@
 // Internal declarations shared by the translation units of libnabla.so.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,10 +30,12 @@ inline Dims make_dims(const nabla_shape& s) {
 // Workspace layout: a 256-byte header (status word, scheduler counters), the
 // pooled Qa / Ka in fp64 and as tf32 hi / lo pairs ([B, H, nb, D] each), the
 // reduced logits L (fp32 [B, H, nb, ldl], ldl = nb rounded up to 4) and, for
-// the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]).
+// the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]) and the
+// block-padded per-row LSE / ln 2 and Delta of the tensor-core backward (fp32
+// [B, H, nb * 64] each).
 struct WsLayout {
   size_t header = 0;
-  size_t qa = 0, ka = 0, qhi = 0, qlo = 0, khi = 0, klo = 0, logits = 0, delta = 0;
+  size_t qa = 0, ka = 0, qhi = 0, qlo = 0, khi = 0, klo = 0, logits = 0, delta = 0, lse2p = 0, deltap = 0;
   int ldl = 0;
   size_t total = 0;
 };
@@ -51,7 +54,11 @@ inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
   w.klo = off; off = align256(off + pooled / 2);
   w.ldl = (d.nb + 3) & ~3;
   w.logits = off; off = align256(off + (size_t)d.BH() * d.nb * w.ldl * sizeof(float));
-  if (want_bwd) { w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float)); }
+  if (want_bwd) {
+    w.delta = off; off = align256(off + (size_t)d.BH() * d.S * sizeof(float));
+    w.lse2p = off; off = align256(off + (size_t)d.BH() * d.nb * 64 * sizeof(float));
+    w.deltap = off; off = align256(off + (size_t)d.BH() * d.nb * 64 * sizeof(float));
+  }
   w.total = off;
   return w;
 }
@@ -60,6 +67,14 @@ inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
 enum : int { kWsStatus = 0, kWsTileCounter = 1 };
 
 uint64_t wait_limit_ns();
+
+// Tensor maps (tmaps.cu).  make_map_bf16: 3-D view {D, S, B*H} of a
+// [B, H, S, D] bf16 tensor, box {64, box_rows, 1}, 128-byte swizzle, rows
+// beyond S read as zero.  make_map_pooled_f32: view {D, nb, B*H} of a
+// [B, H, nb, D] fp32 array, box {32, 128, 1}, 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* map, const void* base, const Dims& d, int box_rows);
+bool make_map_pooled_f32(CUtensorMap* map, const float* base, const Dims& d);
+int sm_count();
 
 // Records the message nabla_last_error() returns in the calling thread (an
 // empty message clears it); status is for the reader's benefit only.
@@ -92,6 +107,12 @@ cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, co
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
                                const uint32_t* bits, const int32_t* work, void* o, float* lse,
                                int32_t* ws_header, cudaStream_t st);
+
+// bf16, D = 128 only.  lse2p / deltap: workspace [B*H][nb*64] fp32 each.
+cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, const int32_t* cnt, const int32_t* idx,
+                               const int32_t* cnt_t, const int32_t* idx_t, float* lse2p, float* deltap,
+                               void* dq, void* dk, void* dv, int32_t* ws_header, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 

@@ -507,7 +507,6 @@ int num_sms() {
   return sms;
 }
 
-constexpr size_t kSmemLimit = 227 * 1024 - 4096;  // dynamic part; the kernel also has ~2 KB static
 
 }  // namespace
 

@@ -150,39 +150,12 @@ __global__ void __launch_bounds__(128) score_gemm_kernel(
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(status, 0, (int32_t)NABLA_ERR_TIMEOUT);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult qr;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-  }
-  return fn;
-}
-
-// 3-D view {D, nb, B*H} of a [B, H, nb, D] fp32 array; box {32, 128, 1};
-// 128-byte swizzle; rows beyond nb read as zero.
-bool make_map_f32(CUtensorMap* map, const float* base, const Dims& d) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d.D, (cuuint64_t)d.nb, (cuuint64_t)d.BH()};
-  cuuint64_t strides[2] = {(cuuint64_t)d.D * 4, (cuuint64_t)d.nb * d.D * 4};
-  cuuint32_t box[3] = {(cuuint32_t)kSubK, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t run(const Dims& d, const float* qhi, const float* qlo, const float* khi, const float* klo,
                 float* L, int ldl, int32_t* status, cudaStream_t st) {
   CUtensorMap a, b, c, e;
-  if (!make_map_f32(&a, qhi, d) || !make_map_f32(&b, qlo, d) || !make_map_f32(&c, khi, d) ||
-      !make_map_f32(&e, klo, d))
+  if (!make_map_pooled_f32(&a, qhi, d) || !make_map_pooled_f32(&b, qlo, d) ||
+      !make_map_pooled_f32(&c, khi, d) || !make_map_pooled_f32(&e, klo, d))
     return cudaErrorInvalidValue;
   auto kern = score_gemm_kernel<D>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);

@@ -61,7 +61,9 @@ def test_workspace_size_formula(L):
         ldl = (nb + 3) // 4 * 4
         fwd = 256 + 2 * pooled + 4 * align(B * H * nb * D * 4) + align(B * H * nb * ldl * 4)
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 0) == fwd
-        assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 1) == fwd + align(B * H * S * 4)
+        # backward: Delta [B, H, S] and the block-padded LSE2 / Delta [B, H, nb * 64]
+        bwd = align(B * H * S * 4) + 2 * align(B * H * nb * 64 * 4)
+        assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 1) == fwd + bwd
 
 
 def test_workspace_size_rejects_bad_shapes(L):

@@ -150,6 +150,23 @@ def test_bwd_pretraining_workload_two_heads():
     _bwd_parity(x, M, "bf16", heads=[(0, 0), (1, 15)])
 
 
+@pytest.mark.parametrize("B,H,S,seed", [(1, 2, 1000, 21), (2, 3, 2000, 22), (1, 1, 64, 23)])
+def test_bwd_external_mask_empty_rows_columns_and_odd_lists(B, H, S, seed):
+    """A mask given as bits (not built here): some query blocks keep nothing,
+    some key blocks are kept by no query block, list lengths are odd and even,
+    so the stacked pairs of both backward kernels end ragged."""
+    x = synth.make_random_qkv(B, H, S, 128, "bf16", seed=seed, with_grad=True)
+    nb = -(-S // 64)
+    rng = np.random.default_rng(seed)
+    M = rng.random((B, H, nb, nb)) < 0.45
+    if nb > 3:
+        M[:, :, 1, :] = False           # a query block that attends to nothing
+        M[:, :, :, 2] = False           # a key block nobody attends to
+        M[:, :, 3, :] = False
+        M[:, :, 3, nb - 1] = True       # one kept block: a lone (odd) step, ragged tail keys
+    _bwd_parity(x, M, "bf16")
+
+
 # ------------------------------------------------------ bounded waits
 
 def test_bounded_wait_runs_out_and_reports_timeout():
