@@ -31,9 +31,13 @@
 // Every MMA has N = 64, where one issuing thread reaches about a third of the
 // tensor core's rate; each kernel therefore issues its independent MMA
 // streams from separate warps (S, dP, dV, dK: four issuers; S^T, dP^T, dQ^T:
-// three), which together keep the tensor core fed.  One CTA per SM (TMEM: S
-// and dP double-buffered, 256 columns, plus the accumulators), persistent over
-// the units; a 2-deep TMA ring streams the stepped operands.
+// three), which together keep the tensor core fed.  One CTA per SM, persistent
+// over the units.  The step's stages form a chain (load -> S, dP -> P, dS ->
+// accumulate -> slot free), so every hand-off is buffered to let consecutive
+// steps overlap: S and dP double-buffered in TMEM (256 columns, plus the
+// accumulators), P and dS double-buffered in shared memory, and TMA rings for
+// the stepped operands (dkdv: 2 stages of Q + dO; dq: 3 stages of K, and 2 of
+// V, which is free as soon as dP^T completes).
 //
 // Warp roles (dkdv: 13 warps; dq: 12 warps):
 //   warp 0       TMA producer (fixed operands per unit, stepped operands per
@@ -77,52 +81,39 @@ struct DkdvSmem {
   static constexpr uint32_t v_off = kFixed;
   static constexpr uint32_t kStage = 2 * kStacked + 1024;  // Q pair, dO pair, LSE2[128], Delta[128]
   static constexpr uint32_t stage0 = 2 * kFixed;
-  static constexpr uint32_t p_off = stage0 + 2 * kStage;
-  static constexpr uint32_t ds_off = p_off + kTile128;
-  static constexpr uint32_t bar_off = ds_off + kTile128;
-  static constexpr int kBars = 15;
+  static constexpr uint32_t p0 = stage0 + 2 * kStage;      // P[2]
+  static constexpr uint32_t ds0 = p0 + 2 * kTile128;       // dS[2]
+  static constexpr uint32_t bar_off = ds0 + 2 * kTile128;
+  static constexpr int kBars = 17;
   static constexpr uint32_t misc_off = bar_off + kBars * 8;
   static constexpr uint32_t bytes = misc_off + 16;
   static __host__ __device__ constexpr uint32_t stage(uint32_t s) { return stage0 + s * kStage; }
+  static __host__ __device__ constexpr uint32_t p(uint32_t b) { return p0 + b * kTile128; }
+  static __host__ __device__ constexpr uint32_t ds(uint32_t b) { return ds0 + b * kTile128; }
 };
 
 // Shared-memory plan of dq_tc_kernel.
 struct DqSmem {
+  static constexpr int kKStages = 3, kVStages = 2;
   static constexpr uint32_t q_off = 0;
   static constexpr uint32_t do_off = kFixed;
   static constexpr uint32_t st_off = 2 * kFixed;  // LSE2[64], Delta[64] of the unit's query block
-  static constexpr uint32_t kStage = 2 * kStacked; // K pair, V pair
-  static constexpr uint32_t stage0 = st_off + 1024;
-  static constexpr uint32_t ds_off = stage0 + 2 * kStage;
-  static constexpr uint32_t bar_off = ds_off + kTile128;
-  static constexpr int kBars = 15;
+  static constexpr uint32_t k0 = st_off + 1024;   // K pairs [kKStages]
+  static constexpr uint32_t v0 = k0 + kKStages * kStacked;  // V pairs [kVStages]
+  static constexpr uint32_t ds0 = v0 + kVStages * kStacked; // dS^T [2]
+  static constexpr uint32_t bar_off = ds0 + 2 * kTile128;
+  static constexpr int kBars = 23;
   static constexpr uint32_t misc_off = bar_off + kBars * 8;
   static constexpr uint32_t bytes = misc_off + 16;
-  static __host__ __device__ constexpr uint32_t stage(uint32_t s) { return stage0 + s * kStage; }
+  static __host__ __device__ constexpr uint32_t k(uint32_t s) { return k0 + s * kStacked; }
+  static __host__ __device__ constexpr uint32_t v(uint32_t s) { return v0 + s * kStacked; }
+  static __host__ __device__ constexpr uint32_t ds(uint32_t b) { return ds0 + b * kTile128; }
 };
 
-static_assert(DkdvSmem::p_off % 1024 == 0 && DkdvSmem::ds_off % 1024 == 0, "tile alignment");
-static_assert(DkdvSmem::stage(1) % 1024 == 0, "tile alignment");
-static_assert(DqSmem::stage0 % 1024 == 0 && DqSmem::ds_off % 1024 == 0, "tile alignment");
+static_assert(DkdvSmem::stage(1) % 1024 == 0 && DkdvSmem::p0 % 1024 == 0 && DkdvSmem::ds0 % 1024 == 0,
+              "tile alignment");
+static_assert(DqSmem::k0 % 1024 == 0 && DqSmem::v0 % 1024 == 0 && DqSmem::ds0 % 1024 == 0, "tile alignment");
 static_assert(DkdvSmem::bytes <= 227 * 1024 && DqSmem::bytes <= 227 * 1024, "shared memory");
-
-struct Bars {
-  uint64_t *fixed_full, *fixed_empty, *in_full, *in_empty, *s_full, *s_free, *pd_full, *pd_empty,
-      *acc_full, *acc_empty, *drain;
-  __device__ explicit Bars(uint64_t* b) {
-    fixed_full = b;
-    fixed_empty = b + 1;
-    in_full = b + 2;    // [2]
-    in_empty = b + 4;   // [2]
-    s_full = b + 6;     // [2]
-    s_free = b + 8;     // [2]
-    pd_full = b + 10;
-    pd_empty = b + 11;
-    acc_full = b + 12;
-    acc_empty = b + 13;
-    drain = b + 14;
-  }
-};
 
 // K-major operand (rows x D, two 64-column halves of `half` bytes): the
 // descriptor of MMA step kk (16 columns).
@@ -182,25 +173,36 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
     if (threadIdx.x == 0) atomicCAS(status, 0, (int32_t)NABLA_ERR_UNSUPPORTED);
     return;
   }
-  Bars b((uint64_t*)(smem + L::bar_off));
+  uint64_t* bars = (uint64_t*)(smem + L::bar_off);
+  uint64_t* fixed_full = bars;        // K_j, V_j landed
+  uint64_t* fixed_empty = bars + 1;   // S and dP of the unit done with them
+  uint64_t* in_full = bars + 2;       // [2] Q / dO pair + stats landed
+  uint64_t* in_empty = bars + 4;      // [2] dV and dK of the step done with them
+  uint64_t* s_full = bars + 6;        // [2] S and dP in TMEM
+  uint64_t* s_free = bars + 8;        // [2] S and dP read out of TMEM
+  uint64_t* pd_full = bars + 10;      // [2] P and dS written
+  uint64_t* pd_empty = bars + 12;     // [2] dV and dK done with P and dS
+  uint64_t* acc_full = bars + 14;
+  uint64_t* acc_empty = bars + 15;
+  uint64_t* drain = bars + 16;
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(b.fixed_full, 1);
-    mbar_init(b.fixed_empty, 2);  // S and dP issuers
+    mbar_init(fixed_full, 1);
+    mbar_init(fixed_empty, 2);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(b.in_full + s, 1);
-      mbar_init(b.in_empty + s, 2);  // dV and dK issuers
-      mbar_init(b.s_full + s, 2);    // S and dP issuers
-      mbar_init(b.s_free + s, kEwThreads);
+      mbar_init(in_full + s, 1);
+      mbar_init(in_empty + s, 2);
+      mbar_init(s_full + s, 2);
+      mbar_init(s_free + s, kEwThreads);
+      mbar_init(pd_full + s, kEwThreads);
+      mbar_init(pd_empty + s, 2);
     }
-    mbar_init(b.pd_full, kEwThreads);
-    mbar_init(b.pd_empty, 2);
-    mbar_init(b.acc_full, 2);
-    mbar_init(b.acc_empty, kEwThreads);
-    mbar_init(b.drain, 4);
+    mbar_init(acc_full, 2);
+    mbar_init(acc_empty, kEwThreads);
+    mbar_init(drain, 4);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -228,38 +230,43 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
         if (n == 0) continue;
         const int bh = u / nb, j = u - bh * nb;
         const int32_t* list = idx_t + (long long)u * nb;
-        if (fixed_it > 0 && !(ok = mbar_wait(b.fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns))) break;
-        mbar_expect_tx(b.fixed_full, 2 * kFixed);
+        int nx0 = list[0], nx1 = n > 1 ? list[1] : nx0;  // the next step's pair, read one step early
+        if (fixed_it > 0 && !(ok = mbar_wait(fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns))) break;
+        mbar_expect_tx(fixed_full, 2 * kFixed);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_3d(smem + L::k_off + h * kTile64, &tm_k, b.fixed_full, h * 64, j * 64, bh);
-          tma_load_3d(smem + L::v_off + h * kTile64, &tm_v, b.fixed_full, h * 64, j * 64, bh);
+          tma_load_3d(smem + L::k_off + h * kTile64, &tm_k, fixed_full, h * 64, j * 64, bh);
+          tma_load_3d(smem + L::v_off + h * kTile64, &tm_v, fixed_full, h * 64, j * 64, bh);
         }
         ++fixed_it;
         for (int t = 0; 2 * t < n; ++t, ++g) {
+          const int i0 = nx0, i1 = nx1;
+          if (2 * t + 2 < n) {
+            nx0 = list[2 * t + 2];
+            nx1 = 2 * t + 3 < n ? list[2 * t + 3] : nx0;
+          }
           const uint32_t s = g & 1, use = g >> 1;
-          if (use > 0 && !(ok = mbar_wait(b.in_empty + s, (use - 1) & 1, abort_flag, limit_ns))) break;
-          const int i0 = list[2 * t], i1 = 2 * t + 1 < n ? list[2 * t + 1] : i0;
+          if (use > 0 && !(ok = mbar_wait(in_empty + s, (use - 1) & 1, abort_flag, limit_ns))) break;
           uint8_t* st = smem + L::stage(s);
-          mbar_expect_tx(b.in_full + s, 2 * kStacked + 1024);
+          mbar_expect_tx(in_full + s, 2 * kStacked + 1024);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tma_load_3d(st + h * kTile128, &tm_q, b.in_full + s, h * 64, i0 * 64, bh);
-            tma_load_3d(st + h * kTile128 + kTile64, &tm_q, b.in_full + s, h * 64, i1 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128, &tm_do, b.in_full + s, h * 64, i0 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128 + kTile64, &tm_do, b.in_full + s, h * 64, i1 * 64, bh);
+            tma_load_3d(st + h * kTile128, &tm_q, in_full + s, h * 64, i0 * 64, bh);
+            tma_load_3d(st + h * kTile128 + kTile64, &tm_q, in_full + s, h * 64, i1 * 64, bh);
+            tma_load_3d(st + kStacked + h * kTile128, &tm_do, in_full + s, h * 64, i0 * 64, bh);
+            tma_load_3d(st + kStacked + h * kTile128 + kTile64, &tm_do, in_full + s, h * 64, i1 * 64, bh);
           }
           const long long r0 = ((long long)bh * nb + i0) * 64, r1 = ((long long)bh * nb + i1) * 64;
-          bulk_load(st + 2 * kStacked, lse2p + r0, 256, b.in_full + s);
-          bulk_load(st + 2 * kStacked + 256, lse2p + r1, 256, b.in_full + s);
-          bulk_load(st + 2 * kStacked + 512, deltap + r0, 256, b.in_full + s);
-          bulk_load(st + 2 * kStacked + 768, deltap + r1, 256, b.in_full + s);
+          bulk_load(st + 2 * kStacked, lse2p + r0, 256, in_full + s);
+          bulk_load(st + 2 * kStacked + 256, lse2p + r1, 256, in_full + s);
+          bulk_load(st + 2 * kStacked + 512, deltap + r0, 256, in_full + s);
+          bulk_load(st + 2 * kStacked + 768, deltap + r1, 256, in_full + s);
         }
       }
       // Let every copy issued land before the CTA exits.
-      if (fixed_it > 0) mbar_wait(b.fixed_full, (fixed_it - 1) & 1, nullptr, kDrainLimitNs);
+      if (fixed_it > 0) mbar_wait(fixed_full, (fixed_it - 1) & 1, nullptr, kDrainLimitNs);
       for (uint32_t i = (g > 2 ? g - 2 : 0); i < g; ++i)
-        mbar_wait(b.in_full + (i & 1), (i >> 1) & 1, nullptr, kDrainLimitNs);
+        mbar_wait(in_full + (i & 1), (i >> 1) & 1, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1 || warp == 2) {
     // ---------------------------------------- S and dP issuers (one each)
@@ -273,24 +280,24 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const int n = cnt_t[u];
         if (n == 0) continue;
-        if (!(ok = mbar_wait(b.fixed_full, fixed_it & 1, abort_flag, limit_ns))) break;
+        if (!(ok = mbar_wait(fixed_full, fixed_it & 1, abort_flag, limit_ns))) break;
         ++fixed_it;
         const int steps = (n + 1) >> 1;
         for (int t = 0; t < steps; ++t, ++g) {
           const uint32_t s = g & 1;
-          if (!(ok = mbar_wait(b.in_full + s, (g >> 1) & 1, abort_flag, limit_ns))) break;
-          if (g >= 2 && !(ok = mbar_wait(b.s_free + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
+          if (!(ok = mbar_wait(in_full + s, (g >> 1) & 1, abort_flag, limit_ns))) break;
+          if (g >= 2 && !(ok = mbar_wait(s_free + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
           const uint32_t a_base = sbase + L::stage(s) + (is_s ? 0u : kStacked);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tmem + s * 128 + col, kmajor_desc(a_base, kTile128, kk), kmajor_desc(fixed_base, kTile64, kk),
                    idesc, kk > 0 ? 1u : 0u);
-          mma_commit(b.s_full + s);
+          mma_commit(s_full + s);
         }
-        if (ok) mma_commit(b.fixed_empty);
+        if (ok) mma_commit(fixed_empty);
       }
-      mma_commit(b.drain);
+      mma_commit(drain);
     }
   } else if (warp == 3 || warp == 4) {
     // ---------------------------------------- dV and dK issuers (one each)
@@ -298,31 +305,32 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       const bool is_v = warp == 3;
       constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
       const uint32_t acc = tmem + kAccCol0 + (is_v ? 0u : 64u);
-      const uint32_t b_base = sbase + (is_v ? L::p_off : L::ds_off);
       uint32_t g = 0, u_local = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
         const int steps = (cnt_t[u] + 1) >> 1;
         // The epilogue of the previous unit must have read the accumulators
         // (and seen its acc_full phase) before this unit overwrites or signals.
-        if (u_local > 0 && !(ok = mbar_wait(b.acc_empty, (u_local - 1) & 1, abort_flag, limit_ns))) break;
+        if (u_local > 0 && !(ok = mbar_wait(acc_empty, (u_local - 1) & 1, abort_flag, limit_ns))) break;
         for (int t = 0; t < steps; ++t, ++g) {
-          if (!(ok = mbar_wait(b.pd_full, g & 1, abort_flag, limit_ns))) break;
+          const uint32_t pb = g & 1;
+          if (!(ok = mbar_wait(pd_full + pb, (g >> 1) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
           // A = the stacked dO (for dV) or Q (for dK) tile read MN-major: M = D
           // in two 64-column atoms, K = the 128 stacked query rows.
           const uint32_t a_base = sbase + L::stage(g & 1) + (is_v ? kStacked : 0u);
+          const uint32_t b_base = sbase + (is_v ? L::p(pb) : L::ds(pb));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(acc, mnmajor_desc(a_base, kTile128, kk), mnmajor_desc(b_base, kTile128, kk), idesc,
                    (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(b.pd_empty);
-          mma_commit(b.in_empty + (g & 1));
+          mma_commit(pd_empty + pb);
+          mma_commit(in_empty + (g & 1));
         }
         if (!ok) break;
-        mma_commit(b.acc_full);
+        mma_commit(acc_full);
       }
-      mma_commit(b.drain);
+      mma_commit(drain);
     }
   } else {
     // ------------------------------------- elementwise (P, dS) + epilogue
@@ -339,8 +347,8 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       const int steps = (n + 1) >> 1;
       for (int t = 0; t < steps; ++t, ++g) {
         const uint32_t s = g & 1;
-        const bool w1 = mbar_wait(b.s_full + s, (g >> 1) & 1, abort_flag, limit_ns);
-        const bool w2 = w1 && mbar_wait(b.in_full + s, (g >> 1) & 1, abort_flag, limit_ns);
+        const bool w1 = mbar_wait(s_full + s, (g >> 1) & 1, abort_flag, limit_ns);
+        const bool w2 = w1 && mbar_wait(in_full + s, (g >> 1) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[32], dr[32];
@@ -348,23 +356,23 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
         tmem_ld32(lane_base + s * 128 + 64 + half * 32, dr);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(b.s_free + s);  // the S / dP buffer may be overwritten now
+        mbar_arrive(s_free + s);  // the S / dP buffer may be overwritten now
         const float* st = (const float*)(smem + L::stage(s) + 2 * kStacked);
         const float lse2 = st[r], delta = st[128 + r];
         const bool row_ok = r < 64 || 2 * t + 1 < n;
         uint32_t pw[16], dw[16];
         p_ds_pairs(sr, dr, scale_log2, nullptr, nullptr, lse2, delta, half * 32, row_ok ? kv_lim : 0, pw, dw);
-        // P / dS of the previous step must have been consumed.
-        const bool w3 = g == 0 || mbar_wait(b.pd_empty, (g - 1) & 1, abort_flag, limit_ns);
+        // P / dS of two steps back must have been consumed.
+        const bool w3 = g < 2 || mbar_wait(pd_empty + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
-        store_half_row_sw128(smem + L::p_off, r, half, pw);
-        store_half_row_sw128(smem + L::ds_off, r, half, dw);
+        store_half_row_sw128(smem + L::p(s), r, half, pw);
+        store_half_row_sw128(smem + L::ds(s), r, half, dw);
         fence_proxy_async_smem();
-        mbar_arrive(b.pd_full);
+        mbar_arrive(pd_full + s);
       }
       if (!ok) break;
       // epilogue: thread r owns column d = r of dV^T (half 0) or dK^T (half 1)
-      const bool w4 = mbar_wait(b.acc_full, u_local & 1, abort_flag, limit_ns);
+      const bool w4 = mbar_wait(acc_full, u_local & 1, abort_flag, limit_ns);
       if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
       tc_fence_after();
       const long long row0 = (long long)bh * S + (long long)j * 64;
@@ -386,14 +394,14 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
             out[(row0 + h * 32 + c) * D + r] = __float2bfloat16_rn(__uint_as_float(a[c]) * mul);
       }
       tc_fence_before();
-      mbar_arrive(b.acc_empty);
+      mbar_arrive(acc_empty);
     }
   }
 
   // ------------------------------------------------------------- teardown
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0) mbar_wait(b.drain, 0, nullptr, kDrainLimitNs);
+    if (lane == 0) mbar_wait(drain, 0, nullptr, kDrainLimitNs);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -412,30 +420,51 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                  uint64_t limit_ns) {
   static_assert(D == 128, "the tensor-core backward is built for D = 128");
   using L = DqSmem;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) atomicCAS(status, 0, (int32_t)NABLA_ERR_UNSUPPORTED);
     return;
   }
-  Bars b((uint64_t*)(smem + L::bar_off));
+  uint64_t* bars = (uint64_t*)(smem + L::bar_off);
+  uint64_t* fixed_full = bars;              // Q_i, dO_i, stats landed
+  uint64_t* fixed_empty = bars + 1;         // S^T, dP^T and the elementwise threads done with them
+  uint64_t* k_full = bars + 2;              // [KS]
+  uint64_t* k_empty = k_full + KS;          // [KS] dQ^T done with the K pair
+  uint64_t* v_full = k_empty + KS;          // [VS]
+  uint64_t* v_empty = v_full + VS;          // [VS] dP^T done with the V pair
+  uint64_t* s_full = v_empty + VS;          // [2]
+  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* pd_full = s_free + 2;           // [2] dS^T written
+  uint64_t* pd_empty = pd_full + 2;         // [2] dQ^T done with dS^T
+  uint64_t* acc_full = pd_empty + 2;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  static_assert(2 + 2 * KS + 2 * VS + 8 + 3 == L::kBars, "barrier count");
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(b.fixed_full, 1);
-    mbar_init(b.fixed_empty, 2 + kEwThreads);  // S^T and dP^T issuers, and the elementwise threads (stats)
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(b.in_full + s, 1);
-      mbar_init(b.in_empty + s, 1);  // dQ issuer
-      mbar_init(b.s_full + s, 2);
-      mbar_init(b.s_free + s, kEwThreads);
+    mbar_init(fixed_full, 1);
+    mbar_init(fixed_empty, 2 + kEwThreads);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
     }
-    mbar_init(b.pd_full, kEwThreads);
-    mbar_init(b.pd_empty, 1);
-    mbar_init(b.acc_full, 1);
-    mbar_init(b.acc_empty, kEwThreads);
-    mbar_init(b.drain, 3);
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 2);
+      mbar_init(s_free + s, kEwThreads);
+      mbar_init(pd_full + s, kEwThreads);
+      mbar_init(pd_empty + s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEwThreads);
+    mbar_init(drain, 3);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -456,41 +485,58 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   if (warp == 0) {
     // -------------------------------------------------------- TMA producer
     if (lane == 0) {
-      uint32_t g = 0, fixed_it = 0;
+      uint32_t g = 0, fixed_it = 0, gk = 0, gv = 0;  // steps begun, K and V pair loads issued
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const int n = cnt[u];
         if (n == 0) continue;
         const int bh = u / nb, i = u - bh * nb;
         const int32_t* list = idx + (long long)u * nb;
-        if (fixed_it > 0 && !(ok = mbar_wait(b.fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns))) break;
-        mbar_expect_tx(b.fixed_full, 2 * kFixed + 512);
+        int nx0 = list[0], nx1 = n > 1 ? list[1] : nx0;
+        if (fixed_it > 0 && !(ok = mbar_wait(fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns))) break;
+        mbar_expect_tx(fixed_full, 2 * kFixed + 512);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_3d(smem + L::q_off + h * kTile64, &tm_q, b.fixed_full, h * 64, i * 64, bh);
-          tma_load_3d(smem + L::do_off + h * kTile64, &tm_do, b.fixed_full, h * 64, i * 64, bh);
+          tma_load_3d(smem + L::q_off + h * kTile64, &tm_q, fixed_full, h * 64, i * 64, bh);
+          tma_load_3d(smem + L::do_off + h * kTile64, &tm_do, fixed_full, h * 64, i * 64, bh);
         }
-        bulk_load(smem + L::st_off, lse2p + (long long)u * 64, 256, b.fixed_full);
-        bulk_load(smem + L::st_off + 256, deltap + (long long)u * 64, 256, b.fixed_full);
+        bulk_load(smem + L::st_off, lse2p + (long long)u * 64, 256, fixed_full);
+        bulk_load(smem + L::st_off + 256, deltap + (long long)u * 64, 256, fixed_full);
         ++fixed_it;
         for (int t = 0; 2 * t < n; ++t, ++g) {
-          const uint32_t s = g & 1, use = g >> 1;
-          if (use > 0 && !(ok = mbar_wait(b.in_empty + s, (use - 1) & 1, abort_flag, limit_ns))) break;
-          const int j0 = list[2 * t], j1 = 2 * t + 1 < n ? list[2 * t + 1] : j0;
-          uint8_t* st = smem + L::stage(s);
-          mbar_expect_tx(b.in_full + s, 2 * kStacked);
+          const int j0 = nx0, j1 = nx1;
+          if (2 * t + 2 < n) {
+            nx0 = list[2 * t + 2];
+            nx1 = 2 * t + 3 < n ? list[2 * t + 3] : nx0;
+          }
+          const uint32_t ks = g % KS, kuse = g / KS;
+          if (kuse > 0 && !(ok = mbar_wait(k_empty + ks, (kuse - 1) & 1, abort_flag, limit_ns))) break;
+          uint8_t* kt = smem + L::k(ks);
+          mbar_expect_tx(k_full + ks, kStacked);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tma_load_3d(st + h * kTile128, &tm_k, b.in_full + s, h * 64, j0 * 64, bh);
-            tma_load_3d(st + h * kTile128 + kTile64, &tm_k, b.in_full + s, h * 64, j1 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128, &tm_v, b.in_full + s, h * 64, j0 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128 + kTile64, &tm_v, b.in_full + s, h * 64, j1 * 64, bh);
+            tma_load_3d(kt + h * kTile128, &tm_k, k_full + ks, h * 64, j0 * 64, bh);
+            tma_load_3d(kt + h * kTile128 + kTile64, &tm_k, k_full + ks, h * 64, j1 * 64, bh);
           }
+          ++gk;
+          const uint32_t vs = g % VS, vuse = g / VS;
+          if (vuse > 0 && !(ok = mbar_wait(v_empty + vs, (vuse - 1) & 1, abort_flag, limit_ns))) break;
+          uint8_t* vt = smem + L::v(vs);
+          mbar_expect_tx(v_full + vs, kStacked);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tma_load_3d(vt + h * kTile128, &tm_v, v_full + vs, h * 64, j0 * 64, bh);
+            tma_load_3d(vt + h * kTile128 + kTile64, &tm_v, v_full + vs, h * 64, j1 * 64, bh);
+          }
+          ++gv;
         }
       }
-      if (fixed_it > 0) mbar_wait(b.fixed_full, (fixed_it - 1) & 1, nullptr, kDrainLimitNs);
-      for (uint32_t i = (g > 2 ? g - 2 : 0); i < g; ++i)
-        mbar_wait(b.in_full + (i & 1), (i >> 1) & 1, nullptr, kDrainLimitNs);
+      // Let every copy issued land before the CTA exits.
+      if (fixed_it > 0) mbar_wait(fixed_full, (fixed_it - 1) & 1, nullptr, kDrainLimitNs);
+      for (uint32_t i = (gk > KS ? gk - KS : 0); i < gk; ++i)
+        mbar_wait(k_full + i % KS, (i / KS) & 1, nullptr, kDrainLimitNs);
+      for (uint32_t i = (gv > VS ? gv - VS : 0); i < gv; ++i)
+        mbar_wait(v_full + i % VS, (i / VS) & 1, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1 || warp == 2) {
     // -------------------------------------- S^T and dP^T issuers (one each)
@@ -504,24 +550,31 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const int n = cnt[u];
         if (n == 0) continue;
-        if (!(ok = mbar_wait(b.fixed_full, fixed_it & 1, abort_flag, limit_ns))) break;
+        if (!(ok = mbar_wait(fixed_full, fixed_it & 1, abort_flag, limit_ns))) break;
         ++fixed_it;
         const int steps = (n + 1) >> 1;
         for (int t = 0; t < steps; ++t, ++g) {
           const uint32_t s = g & 1;
-          if (!(ok = mbar_wait(b.in_full + s, (g >> 1) & 1, abort_flag, limit_ns))) break;
-          if (g >= 2 && !(ok = mbar_wait(b.s_free + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
+          uint32_t a_base;
+          if (is_s) {
+            if (!(ok = mbar_wait(k_full + g % KS, (g / KS) & 1, abort_flag, limit_ns))) break;
+            a_base = sbase + L::k(g % KS);
+          } else {
+            if (!(ok = mbar_wait(v_full + g % VS, (g / VS) & 1, abort_flag, limit_ns))) break;
+            a_base = sbase + L::v(g % VS);
+          }
+          if (g >= 2 && !(ok = mbar_wait(s_free + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
-          const uint32_t a_base = sbase + L::stage(s) + (is_s ? 0u : kStacked);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tmem + s * 128 + col, kmajor_desc(a_base, kTile128, kk), kmajor_desc(fixed_base, kTile64, kk),
                    idesc, kk > 0 ? 1u : 0u);
-          mma_commit(b.s_full + s);
+          mma_commit(s_full + s);
+          if (!is_s) mma_commit(v_empty + g % VS);
         }
-        if (ok) mma_commit(b.fixed_empty);
+        if (ok) mma_commit(fixed_empty);
       }
-      mma_commit(b.drain);
+      mma_commit(drain);
     }
   } else if (warp == 3) {
     // --------------------------------------------------------- dQ issuer
@@ -531,23 +584,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
         const int steps = (cnt[u] + 1) >> 1;
-        if (u_local > 0 && !(ok = mbar_wait(b.acc_empty, (u_local - 1) & 1, abort_flag, limit_ns))) break;
+        if (u_local > 0 && !(ok = mbar_wait(acc_empty, (u_local - 1) & 1, abort_flag, limit_ns))) break;
         for (int t = 0; t < steps; ++t, ++g) {
-          if (!(ok = mbar_wait(b.pd_full, g & 1, abort_flag, limit_ns))) break;
+          const uint32_t pb = g & 1;
+          if (!(ok = mbar_wait(pd_full + pb, (g >> 1) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
           // A = the stacked K tile read MN-major (M = D), B = dS^T (N = 64 queries).
-          const uint32_t a_base = sbase + L::stage(g & 1);
+          const uint32_t a_base = sbase + L::k(g % KS);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + kAccCol0, mnmajor_desc(a_base, kTile128, kk), mnmajor_desc(sbase + L::ds_off, kTile128, kk),
+            mma_ss(tmem + kAccCol0, mnmajor_desc(a_base, kTile128, kk), mnmajor_desc(sbase + L::ds(pb), kTile128, kk),
                    idesc, (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(b.pd_empty);
-          mma_commit(b.in_empty + (g & 1));
+          mma_commit(pd_empty + pb);
+          mma_commit(k_empty + g % KS);
         }
         if (!ok) break;
-        mma_commit(b.acc_full);
+        mma_commit(acc_full);
       }
-      mma_commit(b.drain);
+      mma_commit(drain);
     }
   } else {
     // ------------------------------------------- elementwise (dS^T) + epilogue
@@ -557,21 +611,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float* lse2c = (const float*)(smem + L::st_off) + half * 32;
     const float* deltac = lse2c + 64;
+    const int tail_keys = S - (nb - 1) * 64;  // valid keys of the last key block
     uint32_t g = 0, u_local = 0, fixed_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
       const int n = cnt[u];
       const int bh = u / nb, i = u - bh * nb;
-      const int32_t* list = idx + (long long)u * nb;
       const int steps = (n + 1) >> 1;
+      // Lists are ascending, so the last key block (the only one with padded
+      // keys) can only be the list's last entry.
+      const bool ends_in_tail = n > 0 && idx[(long long)u * nb + n - 1] == nb - 1;
       if (steps > 0) {
-        const bool w0 = mbar_wait(b.fixed_full, fixed_it & 1, abort_flag, limit_ns);
+        const bool w0 = mbar_wait(fixed_full, fixed_it & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w0)) { ok = false; break; }
         ++fixed_it;
       }
       for (int t = 0; t < steps; ++t, ++g) {
         const uint32_t s = g & 1;
-        const bool w1 = mbar_wait(b.s_full + s, (g >> 1) & 1, abort_flag, limit_ns);
+        const bool w1 = mbar_wait(s_full + s, (g >> 1) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[32], dr[32];
@@ -579,23 +636,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tmem_ld32(lane_base + s * 128 + 64 + half * 32, dr);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(b.s_free + s);
-        const bool second = r >= 64;
-        const int jb = second ? (2 * t + 1 < n ? list[2 * t + 1] : -1) : list[2 * t];
-        const int key = jb * 64 + (r & 63);
-        const bool row_ok = jb >= 0 && key < S;
+        mbar_arrive(s_free + s);
+        const int pos = 2 * t + (r >= 64 ? 1 : 0);  // list position of this row's key block
+        const bool row_ok = pos < n && !(ends_in_tail && pos == n - 1 && (r & 63) >= tail_keys);
         uint32_t dw[16];
         p_ds_pairs(sr, dr, scale_log2, lse2c, deltac, 0.f, 0.f, 0, row_ok ? 32 : 0, nullptr, dw);
-        const bool w3 = g == 0 || mbar_wait(b.pd_empty, (g - 1) & 1, abort_flag, limit_ns);
+        const bool w3 = g < 2 || mbar_wait(pd_empty + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
-        store_half_row_sw128(smem + L::ds_off, r, half, dw);
+        store_half_row_sw128(smem + L::ds(s), r, half, dw);
         fence_proxy_async_smem();
-        mbar_arrive(b.pd_full);
+        mbar_arrive(pd_full + s);
       }
       if (!ok) break;
-      if (steps > 0) mbar_arrive(b.fixed_empty);  // done with this unit's LSE2 / Delta
+      if (steps > 0) mbar_arrive(fixed_empty);  // done with this unit's LSE2 / Delta
       // epilogue: thread r owns column d = r of dQ^T, query columns [32 half, 32 half + 32)
-      const bool w4 = mbar_wait(b.acc_full, u_local & 1, abort_flag, limit_ns);
+      const bool w4 = mbar_wait(acc_full, u_local & 1, abort_flag, limit_ns);
       if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
       tc_fence_after();
       const long long row0 = (long long)bh * S + (long long)i * 64 + half * 32;
@@ -612,13 +667,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       for (int c = 0; c < 32; ++c)
         if (c < q_lim) dq[(row0 + c) * D + r] = __float2bfloat16_rn(__uint_as_float(a[c]) * scale);
       tc_fence_before();
-      mbar_arrive(b.acc_empty);
+      mbar_arrive(acc_empty);
     }
   }
 
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0) mbar_wait(b.drain, 0, nullptr, kDrainLimitNs);
+    if (lane == 0) mbar_wait(drain, 0, nullptr, kDrainLimitNs);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
