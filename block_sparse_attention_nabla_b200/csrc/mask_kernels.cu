@@ -245,27 +245,30 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   // for e >= 0 that is e > the float whose pattern is u's bucket top.
   auto mass_above = [&](uint32_t u, int sh) -> float {
     const float tv = __uint_as_float((u << sh) | ((1u << sh) - 1u));
-    float f0 = 0.f, f1 = 0.f;
+    float f[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums: short add chains
     if constexpr (NPL > 0) {
 #pragma unroll
-      for (int t = 0; t < NPL; t += 2) {
-        if (ev[t] > tv) f0 += ev[t];
-        if (t + 1 < NPL && ev[t + 1] > tv) f1 += ev[t + 1];
-      }
+      for (int t = 0; t < NPL; ++t)
+        if (ev[t] > tv) f[t & 3] += ev[t];
     } else {
       for (int j = lane; j < nb; j += 32) {
         const float e = Lr[j];
-        if (e > tv) f0 += e;
+        if (e > tv) f[0] += e;
       }
     }
-    return warp_sum(f0 + f1);
+    return warp_sum((f[0] + f[1]) + (f[2] + f[3]));
   };
   // Binary search over the top 16 bits of the pattern: the smallest prefix p
   // whose strictly higher prefixes hold mass <= limit.  e_max = 1 has prefix
   // 0x3F80, so the mass above prefix 0x3F80 is 0.  Entries above the cut-off
   // bucket (prefix > p) are kept and entries below it dropped; the entries
   // of bucket p are ranked below.  p == 0 means every block is kept.
+  // Lower end: entries at or below u = (1 - thr) s / (2 nb) hold at most
+  // nb u = (1 - thr) s / 2 of the mass, so every prefix below prefix(u) still
+  // has more than thr s above it (by half the dropped mass, far beyond fp32
+  // rounding of the sums) and cannot be the cut-off.
   uint32_t lo = 0u, hi = 0x3F80u;
+  if (c.thr < 1.f) lo = min(__float_as_uint((1.f - c.thr) * s / (float)(2 * nb)) >> 16, hi);
   while (lo < hi) {
     const uint32_t mid = lo + ((hi - lo) >> 1);
     if (mass_above(mid, 16) <= limit) hi = mid; else lo = mid + 1u;
