@@ -41,8 +41,9 @@ THR = 0.8
 # reported only while the source is unchanged.  Filled from the summaries
 # under profiles/.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_tc_720p_h4.md: 384.5 MB at 4 heads, scaled x10 to 40 heads
-    "attn_fwd_tc.cu": ("0734e8f110d062fb5c8406a20afd0b88308bd08823007decee15d46f9fed8278", 3.845e9),
+    # profiles/attn_fwd_tc_720p_h4.md: 384.5 MB at 4 heads, scaled x10 to 40 heads (the
+    # kernel is unchanged since; its tensor-map helpers moved to tmaps.cu)
+    "attn_fwd_tc.cu": ("941b67b4c9e4ec51746dd049faf6a8c52ebc25cdf347bc8616f8bee37bc84c6c", 3.845e9),
 }
 
 
@@ -248,6 +249,56 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
             "gpu_launches_per_step": 9}
 
 
+def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
+    """The sparsity sweep at the 720p shape (thresholds 0.5 ... 1.0, the last
+    the dense path) and the threshold-0.8 mask OR-ed with the STA window of
+    3 x 3 x 3 tiles: per case the kept fraction, mask-build and attention
+    ms/call and the attention TFLOP/s on kept tiles (CUDA events on the
+    launching stream)."""
+    import torch
+    B, H, S, D = q.shape
+    ws = nabla.workspace(q)
+    mask = nabla.Mask.empty(B, H, S, q.device, transpose=False)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream()
+    rows = []
+    cases = [(t, False) for t in (0.5, 0.7, 0.8, 0.9, 0.95, 1.0)] + [(0.8, True)]
+    for thr, sta in cases:
+        kw = dict(sta_coords=coords, sta_window=(3, 3, 3)) if sta else {}
+
+        def one(ev=None):
+            if ev:
+                ev[0].record(stream)
+            nabla.build_mask(q, k, thr, out=mask, ws=ws, transpose=False, **kw)
+            if ev:
+                ev[1].record(stream)
+            nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+            if ev:
+                ev[2].record(stream)
+
+        for _ in range(max(warmup, 1)):
+            one()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in evs:
+            one(e)
+        torch.cuda.synchronize()
+        if nabla.workspace_status(ws) != 0:
+            raise SystemExit("device status word reports a timeout in the sweep")
+        kept = int(mask.cnt.to(torch.int64).sum().item())
+        nb = mask.cnt.shape[-1]
+        attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        rows.append({"thr": thr, "sta": "3x3x3 tiles" if sta else None,
+                     "kept_fraction": kept / (B * H * nb * nb),
+                     "mask_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs), "attn_ms": attn,
+                     "attn_tflops": kept * 4 * 64 * 64 * D / (attn * 1e-3) / 1e12})
+    dense = next(r for r in rows if r["thr"] == 1.0)
+    for r in rows:
+        r["speedup_vs_dense"] = dense["attn_ms"] / r["attn_ms"]
+    return {"workload": f"720p shape B={B} H={H} S={S} D={D} bf16, same inputs as the main line",
+            "steps": steps, "cases": rows}
+
+
 def _config(w, n) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16, {w.T}x{w.Hl}x{w.Wl} tokens, "
                         f"thr {THR}, no STA",
@@ -266,6 +317,7 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-training", action="store_true", help="skip the forward + backward training leg")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the threshold sweep and the STA case")
     ap.add_argument("--only-training", action="store_true",
                     help="run only the training leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
@@ -355,6 +407,9 @@ def main() -> None:
     kept_tiles = int(mask.cnt.to(torch.int64).sum().item())
     nb = mask.cnt.shape[-1]
     kept_frac = kept_tiles / (B * H * nb * nb)
+    # tiles the kernel executes: a unit of two query blocks computes the union
+    # of their kept lists at M = 128, i.e. two 64 x 64 tiles per union entry
+    union_tiles = 2 * int(mask.work[:, 1].to(torch.int64).sum().item())
     flops = kept_tiles * 4 * 64 * 64 * D                     # per problem, tile basis
     ms_step = total_ms / args.steps
     value = world * flops / (ms_step * 1e-3) / 1e12
@@ -374,6 +429,10 @@ def main() -> None:
     if world == 1 and not args.no_training:
         training = measure_training(dev, args.warmup, max(1, min(args.steps, 5)))
 
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -383,6 +442,8 @@ def main() -> None:
             "attn_frac_of_bf16_peak": attn_tflops / peaks["bf16_sus"],
             "mask_build_ms": mask_avg, "mask_build_gbs": mask_gbs, "mask_build_frac_hbm": mask_gbs / peaks["hbm"],
             "kept_fraction": kept_frac, "kept_tiles": kept_tiles,
+            "executed_tiles": union_tiles, "union_efficiency": kept_tiles / union_tiles,
+            "attn_tflops_executed": union_tiles * 4 * 64 * 64 * D / (attn_avg * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel<128> (attn_fwd_tc.cu)",
                          "achieved": attn_tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
                          "frac": attn_tflops / peaks["bf16_sus"],
@@ -392,6 +453,7 @@ def main() -> None:
                          "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
             "e2e": e2e,
             "training": training,
+            "sweep": sweep,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }
