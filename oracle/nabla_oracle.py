@@ -17,6 +17,8 @@ arXiv 2507.13546v1):
 * §2.2, Eq. 4: masked attention softmax(QK^T / sqrt(D) + M) V with
   M in {-inf, 0}; §2.1, Eq. 2-3: dense attention.
 * §2.2: the STA window is a fixed 3D window of tiles centred on the query tile.
+* §3.1.1, Figure 3: fractal flattening of the token sequence (P x P patches
+  made contiguous, temporal order kept) and its inverse.
 
 Readings where the paper is silent (listed with reasons in the design notes):
 
@@ -28,7 +30,9 @@ Readings where the paper is silent (listed with reasons in the design notes):
   tokens, and its missing key positions are excluded from attention;
 * STA window: |dt| <= wT // 2, |dy| <= wH // 2, |dx| <= wW // 2 in tile units,
   truncated at the grid edge (no shifting of the window);
-* the mask is a constant of the backward pass (no gradient through pooling).
+* the mask is a constant of the backward pass (no gradient through pooling);
+* edge patches of a frame whose sides are not multiples of P keep their valid
+  tokens, row-major.
 
 Every function here is pinned by the CPU tests in tests/test_oracle_*.py
 against values the paper fixes (Table 1 STA sparsities), closed forms,
@@ -242,6 +246,39 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK):
                 dQ[b, h, rows] = dS @ K[b, h, keys] * scale
                 dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
     return dQ, dK, dV
+
+
+# ------------------------------------------------- §3.1.1 token reordering
+
+def fractal_order(T: int, Hl: int, Wl: int, P: int = 8) -> np.ndarray:
+    """Fractal flattening of §3.1.1 (Figure 3) as a gather index: entry f is
+    the raster index t * Hl * Wl + y * Wl + x of the token that lands at
+    position f of the reordered sequence.  Frames keep their temporal order;
+    inside a frame the P x P patches follow in row-major patch order, each
+    patch's tokens contiguous and row-major inside the patch.  Edge patches of
+    a frame whose height or width is not a multiple of P hold only their
+    valid tokens, still row-major (the reading used throughout)."""
+    order = []
+    for t in range(T):
+        for py in range(0, Hl, P):
+            for px in range(0, Wl, P):
+                for y in range(py, min(py + P, Hl)):
+                    for x in range(px, min(px + P, Wl)):
+                        order.append((t * Hl + y) * Wl + x)
+    return np.asarray(order, dtype=np.int64)
+
+
+def fractal_reorder(X, T: int, Hl: int, Wl: int, P: int = 8, inverse: bool = False) -> np.ndarray:
+    """Applies the reordering to X [B, S, ...] (S = T * Hl * Wl): the network
+    input goes from raster to fractal order; inverse=True is the output-stage
+    inverse, fractal back to raster order (§3.1.1)."""
+    X = np.asarray(X)
+    perm = fractal_order(T, Hl, Wl, P)
+    if not inverse:
+        return X[:, perm]
+    out = np.empty_like(X)
+    out[:, perm] = X
+    return out
 
 
 # ------------------------------------------------------------ error metrics

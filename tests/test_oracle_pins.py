@@ -284,3 +284,43 @@ def test_error_metrics():
     x = ref + np.array([0.1, 0.0, -0.2])
     assert abs(orc.max_abs(x, ref) - 0.2) < 1e-15
     assert abs(orc.mean_rel(x, ref) - (0.3 / 3) / (7 / 3)) < 1e-15
+
+
+# ---------------------------------------------------- §3.1.1 token reordering
+
+@pytest.mark.parametrize("case", _read_golden("fractal_order_cases.txt"))
+def test_fractal_order_hand_cases(case):
+    T, H, W, P = (int(v) for v in case[0])
+    expect = [int(v) for v in case[1]]
+    assert orc.fractal_order(T, H, W, P).tolist() == expect
+
+
+def test_fractal_order_figure3_closed_form():
+    """Figure 3's 16 x 16 latent with P = 8: position f = patch * 64 + dy * 8 + dx
+    holds raster token (8 py + dy) * 16 + 8 px + dx, patches row-major."""
+    f = np.arange(256)
+    patch, dy, dx = f // 64, (f % 64) // 8, f % 8
+    raster = (8 * (patch // 2) + dy) * 16 + 8 * (patch % 2) + dx
+    assert (orc.fractal_order(1, 16, 16, 8) == raster).all()
+
+
+@pytest.mark.parametrize("T,H,W,P", [(3, 30, 52, 8), (2, 45, 80, 8), (1, 7, 9, 4), (4, 8, 8, 8)])
+def test_fractal_order_is_a_framewise_bijection_with_contiguous_patches(T, H, W, P):
+    perm = orc.fractal_order(T, H, W, P)
+    HW = H * W
+    assert sorted(perm.tolist()) == list(range(T * HW))
+    # temporal order kept: position f stays in its frame
+    assert (perm // HW == np.arange(T * HW) // HW).all()
+    # each patch is one contiguous run of positions
+    y, x = (perm % HW) // W, perm % W
+    pid = (perm // HW) * 10**6 + (y // P) * 1000 + x // P
+    runs = np.flatnonzero(np.diff(pid)) + 1
+    assert len(runs) + 1 == T * (-(-H // P)) * (-(-W // P))
+
+
+def test_fractal_reorder_inverse_restores_raster_order():
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((2, 3 * 9 * 11, 4))
+    Y = orc.fractal_reorder(X, 3, 9, 11, 4)
+    assert not np.array_equal(Y, X)
+    assert np.array_equal(orc.fractal_reorder(Y, 3, 9, 11, 4, inverse=True), X)
