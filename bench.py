@@ -299,6 +299,34 @@ def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
             "steps": steps, "cases": rows}
 
 
+def measure_reorder(nabla, dev, warmup: int, steps: int) -> dict:
+    """Fractal token reordering (§3.1.1) of [B, T*H*W, C] activations at the
+    720p latent (T=21, H=45, W=80, P=8) with C = 5120 bf16 channels, forward and
+    inverse; HBM-bound: every row read once and written once (2 x 774 MB per
+    call; inputs larger than L2)."""
+    import torch
+    T, H, W, P, C = 21, 45, 80, 8, 5120
+    x = torch.randn(1, T * H * W, C, device=dev, dtype=torch.bfloat16)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    res = {}
+    peaks = _peaks()
+    for inv in (False, True):
+        for _ in range(max(warmup, 1)):
+            nabla.fractal_reorder(x, T, H, W, P, inverse=inv, out=y)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            nabla.fractal_reorder(x, T, H, W, P, inverse=inv, out=y)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        gbs = 2 * x.numel() * x.element_size() / (ms * 1e-3) / 1e9
+        res["inverse" if inv else "forward"] = {"ms": ms, "gbs": gbs, "frac_hbm": gbs / peaks["hbm"]}
+    return {"workload": f"[1, {T}x{H}x{W}, {C}] bf16, P={P}", "bytes_per_call": 2 * x.numel() * x.element_size(),
+            "kernel": "reorder_kernel (reorder.cu)", **res}
+
+
 def _config(w, n) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16, {w.T}x{w.Hl}x{w.Wl} tokens, "
                         f"thr {THR}, no STA",
@@ -429,6 +457,10 @@ def main() -> None:
     if world == 1 and not args.no_training:
         training = measure_training(dev, args.warmup, max(1, min(args.steps, 5)))
 
+    reorder = None
+    if world == 1 and not args.no_sweep:
+        reorder = measure_reorder(nabla, dev, 3, 10)
+
     sweep = None
     if world == 1 and not args.no_sweep:
         sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
@@ -454,6 +486,7 @@ def main() -> None:
             "e2e": e2e,
             "training": training,
             "sweep": sweep,
+            "fractal_reorder": reorder,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }

@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
-           "selftest_wait_timeout", "build_mask_noalloc",
+           "selftest_wait_timeout", "build_mask_noalloc", "fractal_reorder",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -31,7 +31,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_noalloc",
            "nabla_mask_from_bits", "nabla_attn_fwd",
-           "nabla_attn_bwd", "nabla_selftest_wait_timeout", "nabla_workspace_status",
+           "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
            "nabla_last_error", "nabla_abi_version"]
 
@@ -78,13 +78,14 @@ def lib() -> ctypes.CDLL:
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
+    L.nabla_fractal_reorder.argtypes = [P, P, I32, I32, I32, I32, I32, SZ, I32, P]
     L.nabla_workspace_status.argtypes = [P, ctypes.POINTER(I32), P]
     L.nabla_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.nabla_set_wait_limit_ns.argtypes, L.nabla_set_wait_limit_ns.restype = [ctypes.c_uint64], None
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
-                 "nabla_attn_fwd", "nabla_attn_bwd",
+                 "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
         getattr(L, name).restype = I32
     _lib = L
@@ -233,6 +234,22 @@ def mask_from_bits(bits: torch.Tensor, q_shape, dtype=torch.bfloat16, out: Mask 
     ms = out.as_struct()
     _check(lib().nabla_mask_from_bits(ctypes.byref(sh), bits.data_ptr(), ctypes.byref(ms),
                                       ws.data_ptr(), ws.numel(), _stream()), "nabla_mask_from_bits")
+    return out
+
+
+def fractal_reorder(x: torch.Tensor, T: int, H: int, W: int, P: int = 8, inverse: bool = False,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """Fractal token reordering of §3.1.1 on x [B, T*H*W, ...] (raster -> fractal
+    order; inverse=True: fractal -> raster).  Rows are moved as bytes."""
+    if not x.is_cuda or not x.is_contiguous():
+        raise NablaError("x must be a contiguous CUDA tensor")
+    B, S = x.shape[0], x.shape[1]
+    if S != T * H * W:
+        raise NablaError(f"x has {S} tokens, T * H * W = {T * H * W}")
+    out = torch.empty_like(x) if out is None else out
+    row_bytes = x[0, 0].numel() * x.element_size()
+    _check(lib().nabla_fractal_reorder(x.data_ptr(), out.data_ptr(), B, T, H, W, P, row_bytes,
+                                       1 if inverse else 0, _stream()), "nabla_fractal_reorder")
     return out
 
 

@@ -183,6 +183,26 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const voi
   return emit_derived(d, out->bits, out, st);
 }
 
+nabla_status nabla_fractal_reorder(const void* x, void* y, int32_t B, int32_t T, int32_t H, int32_t W,
+                                   int32_t P, size_t row_bytes, int32_t inverse, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_tensor(x, "x"));
+  NABLA_TRY(check_tensor(y, "y"));
+  if (B < 1 || T < 1 || H < 1 || W < 1 || P < 1)
+    return fail(NABLA_ERR_INVALID_ARG, "B, T, H, W, P must be >= 1 (got %d, %d, %d, %d, %d)", B, T, H, W, P);
+  if (row_bytes == 0 || row_bytes % 16 != 0)
+    return fail(NABLA_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %zu)", row_bytes);
+  if (inverse != 0 && inverse != 1) return fail(NABLA_ERR_INVALID_ARG, "inverse must be 0 or 1 (got %d)", inverse);
+  if ((long long)H * W > (1ll << 30) || row_bytes / 16 > (1ull << 30))
+    return fail(NABLA_ERR_UNSUPPORTED, "frame of %d x %d tokens or rows of %zu bytes too large", H, W, row_bytes);
+  const unsigned long long bytes = (unsigned long long)B * T * H * W * row_bytes;
+  const uintptr_t xs = (uintptr_t)x, ys = (uintptr_t)y;
+  if (xs < ys + bytes && ys < xs + bytes) return fail(NABLA_ERR_INVALID_ARG, "x and y overlap");
+  NABLA_CUDA(launch_fractal_reorder(x, y, B, T, H, W, P, row_bytes, inverse, (cudaStream_t)stream),
+             "fractal reorder kernel");
+  return NABLA_OK;
+}
+
 nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits,
                                   const nabla_mask* out, void* workspace, size_t workspace_bytes,
                                   nabla_stream_t stream) {

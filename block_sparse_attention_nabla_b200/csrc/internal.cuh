@@ -104,6 +104,8 @@ cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, co
                                  const int32_t* cnt, const int32_t* idx, const int32_t* cnt_t,
                                  const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
                                  cudaStream_t st);
+cudaError_t launch_fractal_reorder(const void* x, void* y, int B, int T, int H, int W, int P,
+                                   size_t row_bytes, int inverse, cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
                                const uint32_t* bits, const int32_t* work, void* o, float* lse,
                                int32_t* ws_header, cudaStream_t st);

@@ -181,6 +181,27 @@ NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, c
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 
+/* Fractal token reordering of §3.1.1 (Figure 3) and its inverse: the
+ * permutation a DiT applies to its token sequence at the input stage (and
+ * inverts at the output stage) so that the tokens of every P x P spatial
+ * patch of a latent frame form one contiguous run; frames keep their temporal
+ * order.
+ *   x, y      device arrays of B * T * H * W rows of row_bytes bytes each (the
+ *             rows are moved, not interpreted: any element type, e.g. [B, S, C]
+ *             activations with row_bytes = C * element size); 16-byte aligned;
+ *             row_bytes a positive multiple of 16; y must not overlap x.
+ *   T, H, W   latent frames and frame height and width in tokens (>= 1);
+ *   P         patch side in tokens (>= 1; 8 in the paper, so a patch is one
+ *             64-token block);
+ *   inverse   0: x in raster order (t, y, x) -> y in fractal order;
+ *             1: x in fractal order -> y in raster order.
+ * Reading for frames whose H or W is not a multiple of P (the pages show full
+ * patches only): an edge patch holds its valid tokens, row-major, as one run.
+ * Memory-bound: every row is read once and written once. */
+NABLA_API nabla_status nabla_fractal_reorder(const void* x, void* y, int32_t B, int32_t T, int32_t H,
+                                             int32_t W, int32_t P, size_t row_bytes, int32_t inverse,
+                                             nabla_stream_t stream);
+
 /* Reads the device status word of `workspace` into *host_status (a host
  * pointer): NABLA_OK, or NABLA_ERR_TIMEOUT if a bounded wait inside a kernel of
  * the most recent call on this workspace ran out.  Synchronises `stream`. */

@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 11
+    assert len(names) == 12
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -140,3 +140,20 @@ def test_last_error_is_per_call(L):
     assert L.nabla_workspace_size(ctypes.byref(shape()), 0) > 0   # does not touch the message
     assert _build(L, q=None) == INVALID
     assert b"thr" not in L.nabla_last_error()
+
+
+def test_fractal_reorder_argument_errors(L):
+    ok = dict(x=FAKE, y=FAKE + (1 << 30), B=1, T=2, H=3, W=5, P=2, row_bytes=32, inverse=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.nabla_fractal_reorder(a["x"], a["y"], a["B"], a["T"], a["H"], a["W"], a["P"], a["row_bytes"],
+                                       a["inverse"], None)
+    assert call(x=None) == INVALID
+    assert call(y=FAKE + 8) == INVALID                 # misaligned
+    assert call(y=FAKE + 64) == INVALID                # overlaps x
+    assert call(P=0) == INVALID
+    assert call(H=0) == INVALID
+    assert call(row_bytes=24) == INVALID
+    assert call(inverse=2) == INVALID
+    assert b"inverse" in L.nabla_last_error()
