@@ -2,8 +2,9 @@
 in test_oracle_pins.py catch every one of them: a wrong sort direction, a
 strict comparison, an exclusive cumulative sum, thr for 1 - thr, a missing
 order restoration, a tail block divided by 64, transposed or unscaled scores,
-softmax over the wrong axis, a wrong STA half-width, a transposed block mask
-and a dropped term in the backward pass."""
+softmax over the wrong axis, a wrong STA half-width, a transposed block mask,
+a dropped term in the backward pass, and a fractal order with tokens or
+patches taken column-major or edge patches moved to the end of the frame."""
 import numpy as np
 import pytest
 
@@ -19,10 +20,15 @@ def _all_pins():
         checks.append(lambda c=case: pins.test_cdf_hand_cases(c))
     for case in pins._read_golden("sta_table1.txt"):
         checks.append(lambda c=case: pins.test_sta_reproduces_table1_sparsity(c))
+    for case in pins._read_golden("fractal_order_cases.txt"):
+        checks.append(lambda c=case: pins.test_fractal_order_hand_cases(c))
+    for args in [(3, 30, 52, 8), (2, 45, 80, 8), (1, 7, 9, 4), (4, 8, 8, 8)]:
+        checks.append(lambda a=args: pins.test_fractal_order_is_a_framewise_bijection_with_contiguous_patches(*a))
     for name in dir(pins):
         fn = getattr(pins, name)
         if name.startswith("test_") and callable(fn) and name not in (
-                "test_cdf_hand_cases", "test_sta_reproduces_table1_sparsity"):
+                "test_cdf_hand_cases", "test_sta_reproduces_table1_sparsity", "test_fractal_order_hand_cases",
+                "test_fractal_order_is_a_framewise_bijection_with_contiguous_patches"):
             checks.append(fn)
     return checks
 
@@ -97,6 +103,25 @@ def _bwd_no_rowsum(Q, K, V, dO, M, N=64):
     return dQ, dK, dV
 
 
+def _fractal_variant(col_major_tokens=False, col_major_patches=False, edges_last=False):
+    def f(T, Hl, Wl, P=8):
+        order = []
+        for t in range(T):
+            frame, tail = [], []
+            patches = [(py, px) for py in range(0, Hl, P) for px in range(0, Wl, P)]
+            if col_major_patches:
+                patches = [(py, px) for px in range(0, Wl, P) for py in range(0, Hl, P)]
+            for py, px in patches:
+                toks = [(y, x) for y in range(py, min(py + P, Hl)) for x in range(px, min(px + P, Wl))]
+                if col_major_tokens:
+                    toks = [(y, x) for x in range(px, min(px + P, Wl)) for y in range(py, min(py + P, Hl))]
+                full = py + P <= Hl and px + P <= Wl
+                (frame if full or not edges_last else tail).extend(toks)
+            order += [(t * Hl + y) * Wl + x for y, x in frame + tail]
+        return np.asarray(order, dtype=np.int64)
+    return f
+
+
 MUTANTS = {
     "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
     "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
@@ -114,6 +139,9 @@ MUTANTS = {
     "attention_unscaled": ("masked_attention", _attn_unscaled),
     "attention_mask_transposed": ("masked_attention", _attn_transposed_mask),
     "backward_no_rowsum": ("masked_attention_bwd", _bwd_no_rowsum),
+    "fractal_tokens_column_major": ("fractal_order", _fractal_variant(col_major_tokens=True)),
+    "fractal_patches_column_major": ("fractal_order", _fractal_variant(col_major_patches=True)),
+    "fractal_edge_patches_last": ("fractal_order", _fractal_variant(edges_last=True)),
 }
 
 
