@@ -19,6 +19,8 @@ arXiv 2507.13546v1):
 * §2.2: the STA window is a fixed 3D window of tiles centred on the query tile.
 * §3.1.1, Figure 3: fractal flattening of the token sequence (P x P patches
   made contiguous, temporal order kept) and its inverse.
+* page 1 (review of v2, Appendix C): the fixed-budget Top-k selection the CDF
+  rule is compared with.
 
 Readings where the paper is silent (listed with reasons in the design notes):
 
@@ -104,6 +106,34 @@ def cdf_binarize(A: np.ndarray, thr: float):
     np.put_along_axis(M, order, keep_sorted, axis=-1)
     np.put_along_axis(C, order, cvals, axis=-1)
     return M, C
+
+
+def topk_binarize(A: np.ndarray, k: int) -> np.ndarray:
+    """Fixed-budget comparator of the CDF rule (the Top-k selection the paper's
+    Appendix C compares against, per the page-1 review): every row keeps its k
+    largest entries.  Reading: k is clipped to [1, nb]; among equal values the
+    order is that of the stable ascending sort used by cdf_binarize (the
+    higher column index ranks higher), so exactly k entries are kept."""
+    nb = A.shape[-1]
+    k = min(max(int(k), 1), nb)
+    order = np.argsort(A, axis=-1, kind="stable")
+    keep_sorted = np.zeros(A.shape, dtype=bool)
+    keep_sorted[..., nb - k:] = True
+    M = np.zeros(A.shape, dtype=bool)
+    np.put_along_axis(M, order, keep_sorted, axis=-1)
+    return M
+
+
+def topk_mask(Q, K, k: int, coords=None, window=None, N: int = BLOCK):
+    """Top-k counterpart of nabla_mask: the same pooled scores and softmax
+    (the order is that of the logits), k blocks per row, optional STA union."""
+    Qa = block_pool(as_f64(Q), N)
+    Ka = block_pool(as_f64(K), N)
+    P = row_softmax(reduced_scores(Qa, Ka))
+    M = topk_binarize(P, k)
+    if window is not None:
+        M = M | sta_mask(coords, window)[None, None]
+    return M, P
 
 
 def sta_mask(coords: np.ndarray, window) -> np.ndarray:

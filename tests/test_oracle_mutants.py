@@ -20,6 +20,8 @@ def _all_pins():
         checks.append(lambda c=case: pins.test_cdf_hand_cases(c))
     for case in pins._read_golden("sta_table1.txt"):
         checks.append(lambda c=case: pins.test_sta_reproduces_table1_sparsity(c))
+    for case in pins._read_golden("topk_select_cases.txt"):
+        checks.append(lambda c=case: pins.test_topk_hand_cases(c))
     for case in pins._read_golden("fractal_order_cases.txt"):
         checks.append(lambda c=case: pins.test_fractal_order_hand_cases(c))
     for args in [(3, 30, 52, 8), (2, 45, 80, 8), (1, 7, 9, 4), (4, 8, 8, 8)]:
@@ -28,6 +30,7 @@ def _all_pins():
         fn = getattr(pins, name)
         if name.startswith("test_") and callable(fn) and name not in (
                 "test_cdf_hand_cases", "test_sta_reproduces_table1_sparsity", "test_fractal_order_hand_cases",
+                "test_topk_hand_cases",
                 "test_fractal_order_is_a_framewise_bijection_with_contiguous_patches"):
             checks.append(fn)
     return checks
@@ -122,6 +125,20 @@ def _fractal_variant(col_major_tokens=False, col_major_patches=False, edges_last
     return f
 
 
+def _topk_variant(ties_low_first=False, smallest=False, one_more=False):
+    def f(A, k):
+        nb = A.shape[-1]
+        k = min(max(int(k), 1), nb) + (1 if one_more else 0)
+        k = min(k, nb)
+        order = np.argsort(-A, axis=-1, kind="stable") if ties_low_first else np.argsort(A, axis=-1, kind="stable")[..., ::-1]
+        if smallest:
+            order = np.argsort(A, axis=-1, kind="stable")
+        M = np.zeros(A.shape, dtype=bool)
+        np.put_along_axis(M, order[..., :k], True, axis=-1)
+        return M
+    return f
+
+
 MUTANTS = {
     "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
     "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
@@ -139,6 +156,9 @@ MUTANTS = {
     "attention_unscaled": ("masked_attention", _attn_unscaled),
     "attention_mask_transposed": ("masked_attention", _attn_transposed_mask),
     "backward_no_rowsum": ("masked_attention_bwd", _bwd_no_rowsum),
+    "topk_ties_lower_index_first": ("topk_binarize", _topk_variant(ties_low_first=True)),
+    "topk_keeps_smallest": ("topk_binarize", _topk_variant(smallest=True)),
+    "topk_keeps_one_more": ("topk_binarize", _topk_variant(one_more=True)),
     "fractal_tokens_column_major": ("fractal_order", _fractal_variant(col_major_tokens=True)),
     "fractal_patches_column_major": ("fractal_order", _fractal_variant(col_major_patches=True)),
     "fractal_edge_patches_last": ("fractal_order", _fractal_variant(edges_last=True)),

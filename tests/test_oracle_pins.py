@@ -324,3 +324,30 @@ def test_fractal_reorder_inverse_restores_raster_order():
     Y = orc.fractal_reorder(X, 3, 9, 11, 4)
     assert not np.array_equal(Y, X)
     assert np.array_equal(orc.fractal_reorder(Y, 3, 9, 11, 4, inverse=True), X)
+
+
+# ------------------------------------------------ fixed-budget comparator
+
+@pytest.mark.parametrize("case", _read_golden("topk_select_cases.txt"))
+def test_topk_hand_cases(case):
+    k = int(case[0][0])
+    row = np.array([float(v) for v in case[1]])
+    expect = np.array([v == "1" for v in case[2]])
+    assert (orc.topk_binarize(row[None], k)[0] == expect).all()
+
+
+def test_topk_brute_force_and_invariants():
+    rng = np.random.default_rng(11)
+    for nb in (1, 2, 5, 9):
+        for _ in range(20):
+            A = orc.row_softmax(rng.standard_normal((3, nb)) * 2)
+            for k in range(1, nb + 1):
+                M = orc.topk_binarize(A, k)
+                assert (M.sum(-1) == k).all()
+                for r in range(3):
+                    kept, dropped = A[r][M[r]], A[r][~M[r]]
+                    assert dropped.size == 0 or kept.min() >= dropped.max()
+                    best = max(itertools.combinations(range(nb), k), key=lambda c: A[r][list(c)].sum())
+                    assert set(np.flatnonzero(M[r])) == set(best)
+                if k < nb:
+                    assert (orc.topk_binarize(A, k + 1) >= M).all()   # monotone in k
