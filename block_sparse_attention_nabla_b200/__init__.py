@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
-           "selftest_wait_timeout", "build_mask_noalloc", "fractal_reorder",
+           "selftest_wait_timeout", "build_mask_noalloc", "fractal_reorder", "build_mask_topk",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -29,7 +29,7 @@ _DTYPES = {torch.bfloat16: BF16, torch.float32: FP32}
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so")
 
 # Exported symbols, in the order include/nabla.h declares them.
-SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_noalloc",
+SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc",
            "nabla_mask_from_bits", "nabla_attn_fwd",
            "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
     SH, ST, MK = ctypes.POINTER(_Shape), ctypes.POINTER(_Sta), ctypes.POINTER(_Mask)
     L.nabla_workspace_size.argtypes, L.nabla_workspace_size.restype = [SH, I32], SZ
     L.nabla_build_mask.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P, SZ, P]
+    L.nabla_build_mask_topk.argtypes = [SH, P, P, I32, ST, MK, P, SZ, P]
     L.nabla_mask_from_bits.argtypes = [SH, P, MK, P, SZ, P]
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
@@ -84,7 +85,7 @@ def lib() -> ctypes.CDLL:
     L.nabla_set_wait_limit_ns.argtypes, L.nabla_set_wait_limit_ns.restype = [ctypes.c_uint64], None
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
-    for name in ("nabla_build_mask", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
+    for name in ("nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
                  "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
         getattr(L, name).restype = I32
@@ -195,6 +196,27 @@ def build_mask(q: torch.Tensor, k: torch.Tensor, thr: float, sta_coords: torch.T
     _check(lib().nabla_build_mask(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), ctypes.c_float(thr),
                                   ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
                                   ws.data_ptr(), ws.numel(), _stream()), "nabla_build_mask")
+    return out
+
+
+def build_mask_topk(q: torch.Tensor, k: torch.Tensor, topk: int, sta_coords: torch.Tensor | None = None,
+                    sta_window: tuple | None = None, out: Mask | None = None, ws: torch.Tensor | None = None,
+                    transpose: bool = True) -> Mask:
+    """Fixed-budget comparator of build_mask: every row keeps its topk largest
+    reduced-map entries (plus the STA union when given)."""
+    sh = _shape_of(q)
+    _same(q, k)
+    out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
+    ws = workspace(q) if ws is None else ws
+    sta = None
+    if sta_coords is not None:
+        if sta_window is None:
+            raise NablaError("sta_window is required with sta_coords")
+        sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    ms = out.as_struct()
+    _check(lib().nabla_build_mask_topk(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), int(topk),
+                                       ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
+                                       ws.data_ptr(), ws.numel(), _stream()), "nabla_build_mask_topk")
     return out
 
 

@@ -146,16 +146,16 @@ size_t nabla_workspace_size(const nabla_shape* shape, int32_t want_bwd) {
   return ws_layout(make_dims(*shape), want_bwd != 0).total;
 }
 
-nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const void* k, float thr,
-                              const nabla_sta* sta, const nabla_mask* out, void* workspace,
-                              size_t workspace_bytes, nabla_stream_t stream) {
-  g_last_error.clear();
+static nabla_status build_mask_impl(const nabla_shape* shape, const void* q, const void* k, float thr,
+                                    int32_t topk, const nabla_sta* sta, const nabla_mask* out,
+                                    void* workspace, size_t workspace_bytes, nabla_stream_t stream) {
   NABLA_TRY(check_shape(shape));
   const Dims d = make_dims(*shape);
   NABLA_TRY(check_tensor(q, "q"));
   NABLA_TRY(check_tensor(k, "k"));
-  if (!(thr > 0.f && thr <= 1.f))
+  if (topk == 0 && !(thr > 0.f && thr <= 1.f))
     return fail(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1] (got %g)", (double)thr);
+  if (topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
   if (sta && sta->block_coords) {
     NABLA_TRY(check_i32(sta->block_coords, "sta.block_coords"));
     if (sta->wT < 1 || sta->wH < 1 || sta->wW < 1)
@@ -178,9 +178,25 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const voi
   NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, st), "pooling kernel");
   NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, (int32_t*)workspace + kWsStatus, st),
              "score GEMM kernel");
-  NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, thr, sta, out->bits, out->cnt, out->idx, st),
+  NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, topk ? 1.f : thr, sta, out->bits, out->cnt, out->idx,
+                           st, topk),
              "select kernel");
   return emit_derived(d, out->bits, out, st);
+}
+
+nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const void* k, float thr,
+                              const nabla_sta* sta, const nabla_mask* out, void* workspace,
+                              size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  return build_mask_impl(shape, q, k, thr, 0, sta, out, workspace, workspace_bytes, stream);
+}
+
+nabla_status nabla_build_mask_topk(const nabla_shape* shape, const void* q, const void* k, int32_t topk,
+                                   const nabla_sta* sta, const nabla_mask* out, void* workspace,
+                                   size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  if (topk < 1) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
+  return build_mask_impl(shape, q, k, 1.f, topk, sta, out, workspace, workspace_bytes, stream);
 }
 
 nabla_status nabla_fractal_reorder(const void* x, void* y, int32_t B, int32_t T, int32_t H, int32_t W,

@@ -87,9 +87,11 @@ cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa,
                         float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st);
 cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
                               const float* klo, float* L, int ldl, int32_t* status, cudaStream_t st);
+// topk > 0 selects the fixed-budget rule (the topk largest entries per row)
+// instead of the CDF rule with thr.
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          cudaStream_t st);
+                          cudaStream_t st, int topk = 0);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
                                    int32_t* idx, cudaStream_t st);
 cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,

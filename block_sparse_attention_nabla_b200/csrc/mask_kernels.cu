@@ -166,6 +166,7 @@ struct SelectCtx {
   const double* ka_h;
   int nb, W;
   float thr;
+  int topk;  // > 0: fixed-budget rule, keep the topk largest entries (thr unused)
   const int32_t* coords;  // [nb][3] or null
   int hT, hH, hW;
   int (*cand_j)[kMaxCand];
@@ -240,8 +241,12 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
     }
   }
   s = warp_sum(s);
-  const float limit = c.thr * s;
-  // Mass of the entries whose bit pattern, shifted right by `sh`, exceeds u:
+  // Both rules keep an entry iff the weight of the entries ranked above it is
+  // <= limit: weight e and limit thr * s for the CDF rule, weight 1 and limit
+  // topk - 1 for the fixed budget (exactly topk entries kept).
+  const bool tk = c.topk > 0;
+  const float limit = tk ? (float)(min(c.topk, nb) - 1) : c.thr * s;
+  // Weight of the entries whose bit pattern, shifted right by `sh`, exceeds u:
   // for e >= 0 that is e > the float whose pattern is u's bucket top.
   auto mass_above = [&](uint32_t u, int sh) -> float {
     const float tv = __uint_as_float((u << sh) | ((1u << sh) - 1u));
@@ -249,11 +254,11 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
     if constexpr (NPL > 0) {
 #pragma unroll
       for (int t = 0; t < NPL; ++t)
-        if (ev[t] > tv) f[t & 3] += ev[t];
+        if (ev[t] > tv) f[t & 3] += tk ? 1.f : ev[t];
     } else {
       for (int j = lane; j < nb; j += 32) {
         const float e = Lr[j];
-        if (e > tv) f[0] += e;
+        if (e > tv) f[0] += tk ? 1.f : e;
       }
     }
     return warp_sum((f[0] + f[1]) + (f[2] + f[3]));
@@ -268,13 +273,16 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   // has more than thr s above it (by half the dropped mass, far beyond fp32
   // rounding of the sums) and cannot be the cut-off.
   uint32_t lo = 0u, hi = 0x3F80u;
-  if (c.thr < 1.f) lo = min(__float_as_uint((1.f - c.thr) * s / (float)(2 * nb)) >> 16, hi);
+  if (!tk && c.thr < 1.f) lo = min(__float_as_uint((1.f - c.thr) * s / (float)(2 * nb)) >> 16, hi);
   while (lo < hi) {
     const uint32_t mid = lo + ((hi - lo) >> 1);
     if (mass_above(mid, 16) <= limit) hi = mid; else lo = mid + 1u;
   }
   const uint32_t pcut = lo;
-  int mode = pcut == 0u ? 0 : 1;  // 0 keep all, 1 ranked bucket, 2 fp32 rule at bits >= cut32
+  // 0 keep all, 1 ranked bucket, 2 fp32 rule at bits >= cut32.  The fixed
+  // budget ranks bucket 0 too (entries whose e underflowed stay ordered by
+  // their logits).
+  int mode = (pcut == 0u && !tk) ? 0 : 1;
   uint32_t cut32 = 0u;
   uint64_t keepbits = 0;          // register path: ranked-candidate decisions by t
   if (mode == 1) {
@@ -283,7 +291,7 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
     auto visit = [&](int t, float e) {
       const int j = t * 32 + lane;
       const uint32_t pre = __float_as_uint(e) >> 16;
-      above += pre > pcut ? e : 0.f;
+      above += pre > pcut ? (tk ? 1.f : e) : 0.f;
       const bool isc = j < nb && pre == pcut;
       const uint32_t word = __ballot_sync(kFull, isc);
       const int slot = ncand + __popc(word & lanemask_lt());
@@ -322,7 +330,7 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
         const double lb = __shfl_sync(kFull, lg, b2);
         const int jb = __shfl_sync(kFull, cj, b2);
         const float eb = __shfl_sync(kFull, ce, b2);
-        if (lb > lg || (lb == lg && jb > cj)) mass += eb;
+        if (lb > lg || (lb == lg && jb > cj)) mass += tk ? 1.f : eb;
       }
       const bool kp = act && mass <= limit;
       // hand each candidate's decision to the lane that owns its block
@@ -375,8 +383,8 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
 template <int D, int NPL>
 __global__ void __launch_bounds__(256) select_rows_kernel(
     const float* __restrict__ L, int ldl, const double* __restrict__ qa, const double* __restrict__ ka,
-    long long rows, int nb, int W, float thr, const int32_t* __restrict__ coords, int hT, int hH, int hW,
-    uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
+    long long rows, int nb, int W, float thr, int topk, const int32_t* __restrict__ coords, int hT, int hH,
+    int hW, uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
   __shared__ int cand_j[8][kMaxCand];
   __shared__ float cand_e[8][kMaxCand];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -384,7 +392,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   if (grow >= rows) return;
   const long long bh = grow / nb;
   const int row = (int)(grow - bh * nb);
-  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, coords, hT, hH, hW, cand_j, cand_e};
+  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, topk, coords, hT, hH, hW, cand_j, cand_e};
   float* Lr = const_cast<float*>(L) + grow * ldl;
   uint32_t* brow = bits + grow * W;
   int32_t* irow = idx + grow * nb;
@@ -393,7 +401,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
 
 template <int D>
 void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl, const double* qa,
-                        const double* ka, long long rows, int nb, int W, float thr, const int32_t* coords,
+                        const double* ka, long long rows, int nb, int W, float thr, int topk, const int32_t* coords,
                         int hT, int hH, int hW, uint32_t* bits, int32_t* cnt, int32_t* idx) {
   // registers per lane hold ceil(nb / 32) values, rounded up to a few sizes
   auto k = W <= 8 ? select_rows_kernel<D, 8>
@@ -402,7 +410,7 @@ void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl,
          : W <= 40 ? select_rows_kernel<D, 40>
          : W <= 64 ? select_rows_kernel<D, 64>
                    : select_rows_kernel<D, 0>;
-  k<<<grid, 256, 0, st>>>(L, ldl, qa, ka, rows, nb, W, thr, coords, hT, hH, hW, bits, cnt, idx);
+  k<<<grid, 256, 0, st>>>(L, ldl, qa, ka, rows, nb, W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
 }
 
 // ------------------------------------------------------ lists from a bitmask
@@ -534,16 +542,16 @@ cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa,
 
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          cudaStream_t st) {
+                          cudaStream_t st, int topk) {
   const long long rows = d.BH() * d.nb;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   const bool use_sta = sta && sta->block_coords;
   const int32_t* coords = use_sta ? sta->block_coords : nullptr;
   const int hT = use_sta ? sta->wT / 2 : 0, hH = use_sta ? sta->wH / 2 : 0, hW = use_sta ? sta->wW / 2 : 0;
   if (d.D == 128)
-    launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, coords, hT, hH, hW, bits, cnt, idx);
+    launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
   else
-    launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, coords, hT, hH, hW, bits, cnt, idx);
+    launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
   return cudaGetLastError();
 }
 

@@ -125,6 +125,20 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
                               const nabla_sta* sta, const nabla_mask* out, void* workspace,
                               size_t workspace_bytes, nabla_stream_t stream);
 
+/* Fixed-budget variant of the mask builder: the comparator the paper sets the
+ * CDF rule against (Appendix C of the v2 paper, per its page-1 review: CDF
+ * thresholding against a fixed Top-k at the same average block budget).
+ * Identical pooling and reduced scores; every row then keeps its topk
+ * largest entries of softmax(Qa Ka^T / sqrt(D)) instead of the CDF set (topk
+ * >= 1, clipped to nb; entries with equal values ranked as the stable
+ * ascending sort leaves them, the higher block index first; a row whose cut
+ * falls inside more than 32 entries of one 2^-7-wide value bucket keeps every
+ * entry tied in fp32 with the cut-off).  STA union, outputs, workspace and
+ * errors as nabla_build_mask. */
+NABLA_API nabla_status nabla_build_mask_topk(const nabla_shape* shape, const void* q, const void* k,
+                                             int32_t topk, const nabla_sta* sta, const nabla_mask* out,
+                                             void* workspace, size_t workspace_bytes, nabla_stream_t stream);
+
 /* Mask builder that allocates nothing, for callers that cannot call
  * cudaMalloc when they build a mask (for instance a serving process that
  * reserved all device memory at start-up and allows no side allocation while

@@ -111,3 +111,27 @@ def assert_close(x: torch.Tensor, ref: np.ndarray, kind: str, what: str = "",
     else:
         assert ma <= tol["max_abs"] and mr <= tol["mean_rel"], f"{what}: max_abs {ma:.3g} mean_rel {mr:.3g}"
     return dict(max_abs=ma, mean_rel=mr)
+
+
+def oracle_topk(q, k, topk, coords=None, window=None):
+    """Oracle Top-k mask per (b, h) and the exemption for near-ties at the cut:
+    entries whose fp64 reduced-map value lies within 1e-12 (relative) of the
+    row's k-th largest, where pooling in another summation order may reorder."""
+    B, H, S, D = q.shape
+    nb = orc.num_blocks(S)
+    M = np.zeros((B, H, nb, nb), dtype=bool)
+    X = np.zeros((B, H, nb, nb), dtype=bool)
+    kk = min(max(int(topk), 1), nb)
+    for b in range(B):
+        for h in range(H):
+            m, P = orc.topk_mask(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], topk)
+            M[b, h] = m[0, 0]
+            row = P[0, 0]
+            kth = np.sort(row, axis=-1)[:, nb - kk][:, None]
+            X[b, h] = np.abs(row - kth) <= 1e-12 * np.abs(kth)
+    sta = None
+    if window is not None:
+        sta = orc.sta_mask(np.asarray(coords), window)
+        M |= sta[None, None]
+        X &= ~sta[None, None]
+    return M, X

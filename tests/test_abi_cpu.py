@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 12
+    assert len(names) == 13
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -157,3 +157,12 @@ def test_fractal_reorder_argument_errors(L):
     assert call(row_bytes=24) == INVALID
     assert call(inverse=2) == INVALID
     assert b"inverse" in L.nabla_last_error()
+
+
+def test_build_mask_topk_argument_errors(L):
+    sh = shape()
+    ms = mask_struct()
+    assert L.nabla_build_mask_topk(ctypes.byref(sh), FAKE, FAKE, 0, None, ctypes.byref(ms), FAKE, 1 << 40, None) == INVALID
+    assert b"topk" in L.nabla_last_error()
+    assert L.nabla_build_mask_topk(ctypes.byref(sh), None, FAKE, 4, None, ctypes.byref(ms), FAKE, 1 << 40, None) == INVALID
+    assert L.nabla_build_mask_topk(ctypes.byref(sh), FAKE, FAKE, 4, None, ctypes.byref(ms), None, 0, None) == WORKSPACE

@@ -96,3 +96,45 @@ def test_mask_from_bits_edge_rows():
     torch.cuda.synchronize()
     assert (orc.bits_to_mask(gu.gpu_bits(mask), nb) == M).all()
     gu.check_lists(mask, nb)
+
+
+# ------------------------------------------------ fixed-budget comparator
+
+def _topk_check(mask, M, X, nb, topk, sta=False):
+    G = orc.bits_to_mask(gu.gpu_bits(mask), nb)
+    bad = int(((G != M) & ~X).sum())
+    assert bad == 0, (bad, int(X.sum()))
+    if not sta:
+        # exactly min(topk, nb) per row wherever no near-tie sits at the cut
+        rows = ~X.any(-1)
+        assert (G.sum(-1)[rows] == min(topk, nb)).all()
+    gu.check_lists(mask, nb)
+
+
+@pytest.mark.parametrize("S", [1000, 414, 64, 1, 130])
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("topk", [1, 3, 8, 40])
+def test_topk_small_ragged_bf16(S, D, topk):
+    x = synth.make_random_qkv(2, 3, S, D, "bf16", seed=S + D + 7)
+    q, k = x["q"].cuda(), x["k"].cuda()
+    mask = nabla.build_mask_topk(q, k, topk)
+    torch.cuda.synchronize()
+    M, X = gu.oracle_topk(x["q"], x["k"], topk)
+    _topk_check(mask, M, X, x["nb"], topk)
+
+
+@pytest.mark.parametrize("sta", [False, True])
+def test_topk_720p_two_heads_at_the_cdf_budget(sta):
+    """720p frames, two heads, k = the mean kept count of the CDF rule at thr 0.8
+    on the same heads (the equal-budget comparison of the pages)."""
+    w = synth.WORKLOADS[3].scaled(H=2)
+    x = synth.make_inputs(w)
+    q, k = x["q"].cuda(), x["k"].cuda()
+    cdf = nabla.build_mask(q, k, 0.8)
+    topk = int(round(cdf.cnt.float().mean().item()))
+    coords = x["coords"].cuda().int().contiguous() if sta else None
+    mask = nabla.build_mask_topk(q, k, topk, sta_coords=coords, sta_window=w.sta_window if sta else None)
+    torch.cuda.synchronize()
+    M, X = gu.oracle_topk(x["q"], x["k"], topk, x["coords"].numpy() if sta else None,
+                          w.sta_window if sta else None)
+    _topk_check(mask, M, X, w.nb, topk, sta)
