@@ -20,7 +20,8 @@ arXiv 2507.13546v1):
 * §3.1.1, Figure 3: fractal flattening of the token sequence (P x P patches
   made contiguous, temporal order kept) and its inverse.
 * page 1 (review of v2, Appendix C): the fixed-budget Top-k selection the CDF
-  rule is compared with.
+  rule is compared with, and the per-block fidelity check of the pooling
+  proxy (token-level attention mass inside the retained blocks).
 
 Readings where the paper is silent (listed with reasons in the design notes):
 
@@ -276,6 +277,39 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK):
                 dQ[b, h, rows] = dS @ K[b, h, keys] * scale
                 dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
     return dQ, dK, dV
+
+
+# ------------------------------------------------- block fidelity of a mask
+
+def block_mass(Q, K, N: int = BLOCK) -> np.ndarray:
+    """True token-level attention mass per block: with the dense attention
+    distribution p_s = softmax(q_s K^T / sqrt(D)) of every query token s over
+    all S keys (§2.1, Eq. 2-3), A[i, j] is the mean over the valid query
+    tokens s of block i of the mass p_s puts on the keys of block j.  Every row
+    of A sums to 1.  This is the per-block fidelity quantity the page-1 review
+    asks for ("what fraction of token-level attention mass falls inside the
+    retained blocks").  Q, K [B, H, S, D] -> A [B, H, nb, nb]."""
+    Q, K = as_f64(Q), as_f64(K)
+    B, H, S, D = Q.shape
+    nb = num_blocks(S, N)
+    A = np.zeros((B, H, nb, nb))
+    for b in range(B):
+        for h in range(H):
+            L = Q[b, h] @ K[b, h].T / np.sqrt(D)
+            P = np.exp(L - L.max(-1, keepdims=True))
+            P /= P.sum(-1, keepdims=True)
+            for i in range(nb):
+                rows = P[i * N:min(i * N + N, S)]
+                for j in range(nb):
+                    A[b, h, i, j] = rows[:, j * N:min(j * N + N, S)].sum(-1).mean()
+    return A
+
+
+def mask_recall(A: np.ndarray, M: np.ndarray) -> np.ndarray:
+    """Kept token-level mass of each query block under block mask M:
+    R[..., i] = sum_j M[..., i, j] A[..., i, j] (1 when the mask keeps all the
+    attention mass of the block's queries)."""
+    return (A * M).sum(-1)
 
 
 # ------------------------------------------------- §3.1.1 token reordering

@@ -139,6 +139,25 @@ def _topk_variant(ties_low_first=False, smallest=False, one_more=False):
     return f
 
 
+_ORIG_MASS = orc.block_mass
+
+
+def _mass_rows_summed(Q, K, N=64):
+    A = _ORIG_MASS(Q, K, N)
+    S = np.asarray(orc.as_f64(Q)).shape[-2]
+    n = np.array([min(N, S - i * N) for i in range(A.shape[-1])], dtype=float)
+    return A * n[:, None]
+
+
+def _mass_transposed(Q, K, N=64):
+    return np.swapaxes(_ORIG_MASS(Q, K, N), -1, -2)
+
+
+def _mass_unscaled(Q, K, N=64):
+    D = np.asarray(orc.as_f64(Q)).shape[-1]
+    return _ORIG_MASS(orc.as_f64(Q) * np.sqrt(D), K, N)
+
+
 MUTANTS = {
     "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
     "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
@@ -159,6 +178,9 @@ MUTANTS = {
     "topk_ties_lower_index_first": ("topk_binarize", _topk_variant(ties_low_first=True)),
     "topk_keeps_smallest": ("topk_binarize", _topk_variant(smallest=True)),
     "topk_keeps_one_more": ("topk_binarize", _topk_variant(one_more=True)),
+    "block_mass_rows_summed": ("block_mass", _mass_rows_summed),
+    "block_mass_transposed": ("block_mass", _mass_transposed),
+    "block_mass_unscaled": ("block_mass", _mass_unscaled),
     "fractal_tokens_column_major": ("fractal_order", _fractal_variant(col_major_tokens=True)),
     "fractal_patches_column_major": ("fractal_order", _fractal_variant(col_major_patches=True)),
     "fractal_edge_patches_last": ("fractal_order", _fractal_variant(edges_last=True)),

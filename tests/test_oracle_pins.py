@@ -351,3 +351,47 @@ def test_topk_brute_force_and_invariants():
                     assert set(np.flatnonzero(M[r])) == set(best)
                 if k < nb:
                     assert (orc.topk_binarize(A, k + 1) >= M).all()   # monotone in k
+
+
+# ------------------------------------------------------- block fidelity
+
+def test_block_mass_rows_sum_to_one_and_uniform_case():
+    rng = np.random.default_rng(3)
+    Q = rng.standard_normal((1, 2, 200, 16))
+    K = rng.standard_normal((1, 2, 200, 16))
+    A = orc.block_mass(Q, K)
+    assert A.shape == (1, 2, 4, 4)
+    assert np.allclose(A.sum(-1), 1.0, atol=1e-12)
+    # zero queries: every key equally likely, block mass = block size / S
+    A0 = orc.block_mass(np.zeros_like(Q), K)
+    assert np.allclose(A0, np.array([64, 64, 64, 8]) / 200.0, atol=1e-12)
+
+
+def test_block_mass_brute_force_per_token():
+    """Independent restatement: per query token, softmax with math.exp over
+    the keys one by one, then the block sums averaged over the block's rows."""
+    rng = np.random.default_rng(4)
+    S, D = 70, 4
+    Q = rng.standard_normal((1, 1, S, D))
+    K = rng.standard_normal((1, 1, S, D))
+    ref = np.zeros((2, 2))
+    for s in range(S):
+        logits = [sum(Q[0, 0, s, d] * K[0, 0, t, d] for d in range(D)) / math.sqrt(D) for t in range(S)]
+        mx = max(logits)
+        w = [math.exp(x - mx) for x in logits]
+        tot = sum(w)
+        for j in range(2):
+            ref[s // 64, j] += sum(w[t] for t in range(j * 64, min(j * 64 + 64, S))) / tot
+    ref[0] /= 64
+    ref[1] /= 6
+    assert np.allclose(orc.block_mass(Q, K)[0, 0], ref, atol=1e-12)
+
+
+def test_mask_recall_bounds():
+    rng = np.random.default_rng(6)
+    A = orc.block_mass(rng.standard_normal((1, 1, 256, 8)), rng.standard_normal((1, 1, 256, 8)))
+    full = np.ones(A.shape, dtype=bool)
+    assert np.allclose(orc.mask_recall(A, full), 1.0)
+    assert (orc.mask_recall(A, ~full) == 0).all()
+    diag = np.eye(4, dtype=bool)[None, None]
+    assert np.allclose(orc.mask_recall(A, diag), np.diagonal(A, axis1=-2, axis2=-1))
