@@ -21,6 +21,7 @@ import torch
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
            "selftest_wait_timeout", "build_mask_noalloc", "fractal_reorder", "build_mask_topk",
+           "block_mass", "mask_recall",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -31,7 +32,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc",
            "nabla_mask_from_bits", "nabla_attn_fwd",
-           "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
+           "nabla_attn_bwd", "nabla_block_mass", "nabla_mask_recall", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
            "nabla_last_error", "nabla_abi_version"]
 
@@ -80,13 +81,16 @@ def lib() -> ctypes.CDLL:
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_fractal_reorder.argtypes = [P, P, I32, I32, I32, I32, I32, SZ, I32, P]
+    L.nabla_block_mass.argtypes = [SH, P, P, P, P, SZ, P]
+    L.nabla_mask_recall.argtypes = [SH, P, P, P, P]
     L.nabla_workspace_status.argtypes = [P, ctypes.POINTER(I32), P]
     L.nabla_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.nabla_set_wait_limit_ns.argtypes, L.nabla_set_wait_limit_ns.restype = [ctypes.c_uint64], None
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
-                 "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder",
+                 "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_block_mass",
+                 "nabla_mask_recall",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
         getattr(L, name).restype = I32
     _lib = L
@@ -257,6 +261,30 @@ def mask_from_bits(bits: torch.Tensor, q_shape, dtype=torch.bfloat16, out: Mask 
     _check(lib().nabla_mask_from_bits(ctypes.byref(sh), bits.data_ptr(), ctypes.byref(ms),
                                       ws.data_ptr(), ws.numel(), _stream()), "nabla_mask_from_bits")
     return out
+
+
+def block_mass(q: torch.Tensor, k: torch.Tensor, out: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None) -> torch.Tensor:
+    """True token-level attention mass of every 64 x 64 block of dense attention,
+    float [B, H, nb, nb] (rows sum to 1)."""
+    sh = _shape_of(q)
+    _same(q, k)
+    nb = num_blocks(sh.S)
+    out = torch.empty(sh.B, sh.H, nb, nb, dtype=torch.float32, device=q.device) if out is None else out
+    ws = torch.zeros(256, dtype=torch.uint8, device=q.device) if ws is None else ws
+    _check(lib().nabla_block_mass(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), out.data_ptr(), ws.data_ptr(),
+                                  ws.numel(), _stream()), "nabla_block_mass")
+    return out
+
+
+def mask_recall(mass: torch.Tensor, mask: Mask, q_shape, dtype=torch.bfloat16) -> torch.Tensor:
+    """Kept token-level mass of every query block under `mask`, float [B, H, nb]."""
+    B, H, S, D = q_shape
+    sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    rec = torch.empty(mass.shape[:-1], dtype=torch.float32, device=mass.device)
+    _check(lib().nabla_mask_recall(ctypes.byref(sh), mass.data_ptr(), mask.bits.data_ptr(), rec.data_ptr(),
+                                   _stream()), "nabla_mask_recall")
+    return rec
 
 
 def fractal_reorder(x: torch.Tensor, T: int, H: int, W: int, P: int = 8, inverse: bool = False,

@@ -219,6 +219,36 @@ nabla_status nabla_fractal_reorder(const void* x, void* y, int32_t B, int32_t T,
   return NABLA_OK;
 }
 
+nabla_status nabla_block_mass(const nabla_shape* shape, const void* q, const void* k, float* mass,
+                              void* workspace, size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  if (d.dtype != NABLA_BF16)
+    return fail(NABLA_ERR_UNSUPPORTED, "nabla_block_mass runs on the tensor cores: bf16 inputs only");
+  NABLA_TRY(check_tensor(q, "q"));
+  NABLA_TRY(check_tensor(k, "k"));
+  NABLA_TRY(check_i32(mass, "mass"));
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < 256)
+    return fail(NABLA_ERR_WORKSPACE, "workspace must be >= 256 bytes and 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_block_mass(d, q, k, mass, (int32_t*)workspace, st), "block mass kernel");
+  return NABLA_OK;
+}
+
+nabla_status nabla_mask_recall(const nabla_shape* shape, const float* mass, const uint32_t* bits,
+                               float* recall, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_i32(mass, "mass"));
+  NABLA_TRY(check_i32(bits, "bits"));
+  NABLA_TRY(check_i32(recall, "recall"));
+  NABLA_CUDA(launch_mask_recall(d, mass, bits, recall, (cudaStream_t)stream), "recall kernel");
+  return NABLA_OK;
+}
+
 nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits,
                                   const nabla_mask* out, void* workspace, size_t workspace_bytes,
                                   nabla_stream_t stream) {

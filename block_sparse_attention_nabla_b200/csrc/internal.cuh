@@ -106,6 +106,10 @@ cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, co
                                  const int32_t* cnt, const int32_t* idx, const int32_t* cnt_t,
                                  const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
                                  cudaStream_t st);
+cudaError_t launch_block_mass(const Dims& d, const void* q, const void* k, float* mass, int32_t* ws_header,
+                              cudaStream_t st);
+cudaError_t launch_mask_recall(const Dims& d, const float* mass, const uint32_t* bits, float* recall,
+                               cudaStream_t st);
 cudaError_t launch_fractal_reorder(const void* x, void* y, int B, int T, int H, int W, int P,
                                    size_t row_bytes, int inverse, cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,

@@ -195,6 +195,28 @@ NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, c
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 
+/* Per-block fidelity of a block mask (the check the page-1 review of the v2
+ * paper asks of Algorithm 1's pooling proxy: how much of dense attention's
+ * token-level mass falls inside the retained blocks).
+ * nabla_block_mass writes the true block mass of dense attention (§2.1,
+ * Eq. 2-3, softmax over all S keys):
+ *   mass[b, h, i, j] = mean over the valid query tokens s of block i of
+ *                      sum over the keys t of block j of softmax_t(q_s . k_t / sqrt(D))
+ *   mass   float [B, H, nb, nb], caller-allocated; every row sums to 1.
+ *   q, k   [B, H, S, D] bf16 (tensor cores; fp32 inputs: NABLA_ERR_UNSUPPORTED).
+ *   workspace  any device buffer of >= 256 bytes, 256-byte aligned (its status
+ *          word reports a bounded wait that ran out, NABLA_ERR_TIMEOUT).
+ * Two dense passes of S = Q K^T (4 S^2 D flops per (b, h)); no V. */
+NABLA_API nabla_status nabla_block_mass(const nabla_shape* shape, const void* q, const void* k, float* mass,
+                                        void* workspace, size_t workspace_bytes, nabla_stream_t stream);
+
+/* Kept mass of every query block under a block mask:
+ *   recall[b, h, i] = sum over the kept key blocks j of row i of mass[b, h, i, j]
+ * mass from nabla_block_mass; bits [B, H, nb, W] as in nabla_mask (padding bits
+ * zero); recall float [B, H, nb]. */
+NABLA_API nabla_status nabla_mask_recall(const nabla_shape* shape, const float* mass, const uint32_t* bits,
+                                         float* recall, nabla_stream_t stream);
+
 /* Fractal token reordering of §3.1.1 (Figure 3) and its inverse: the
  * permutation a DiT applies to its token sequence at the input stage (and
  * inverts at the output stage) so that the tokens of every P x P spatial

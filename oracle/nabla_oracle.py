@@ -305,6 +305,23 @@ def block_mass(Q, K, N: int = BLOCK) -> np.ndarray:
     return A
 
 
+def block_mass_rows(Q, K, b: int, h: int, blocks, N: int = BLOCK) -> np.ndarray:
+    """Rows `blocks` of block_mass for one (b, h): the same definition on the
+    query tokens of the listed blocks only (for full-size spot checks).
+    Returns [len(blocks), nb]."""
+    q, k = as_f64(Q[b, h]), as_f64(K[b, h])
+    S, D = k.shape
+    nb = num_blocks(S, N)
+    out = np.zeros((len(blocks), nb))
+    for r, i in enumerate(blocks):
+        L = q[i * N:min(i * N + N, S)] @ k.T / np.sqrt(D)
+        P = np.exp(L - L.max(-1, keepdims=True))
+        P /= P.sum(-1, keepdims=True)
+        for j in range(nb):
+            out[r, j] = P[:, j * N:min(j * N + N, S)].sum(-1).mean()
+    return out
+
+
 def mask_recall(A: np.ndarray, M: np.ndarray) -> np.ndarray:
     """Kept token-level mass of each query block under block mask M:
     R[..., i] = sum_j M[..., i, j] A[..., i, j] (1 when the mask keeps all the

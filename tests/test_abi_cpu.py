@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 13
+    assert len(names) == 15
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -166,3 +166,13 @@ def test_build_mask_topk_argument_errors(L):
     assert b"topk" in L.nabla_last_error()
     assert L.nabla_build_mask_topk(ctypes.byref(sh), None, FAKE, 4, None, ctypes.byref(ms), FAKE, 1 << 40, None) == INVALID
     assert L.nabla_build_mask_topk(ctypes.byref(sh), FAKE, FAKE, 4, None, ctypes.byref(ms), None, 0, None) == WORKSPACE
+
+
+def test_block_mass_and_recall_argument_errors(L):
+    sh = shape()
+    assert L.nabla_block_mass(ctypes.byref(sh), FAKE, FAKE, FAKE, None, 0, None) == WORKSPACE
+    assert L.nabla_block_mass(ctypes.byref(sh), FAKE, None, FAKE, FAKE, 256, None) == INVALID
+    sh32 = shape(dtype=1)
+    assert L.nabla_block_mass(ctypes.byref(sh32), FAKE, FAKE, FAKE, FAKE, 256, None) == UNSUPPORTED
+    assert L.nabla_mask_recall(ctypes.byref(sh), FAKE, None, FAKE, None) == INVALID
+    assert L.nabla_mask_recall(ctypes.byref(sh), FAKE + 2, FAKE, FAKE, None) == INVALID

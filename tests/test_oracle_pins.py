@@ -395,3 +395,11 @@ def test_mask_recall_bounds():
     assert (orc.mask_recall(A, ~full) == 0).all()
     diag = np.eye(4, dtype=bool)[None, None]
     assert np.allclose(orc.mask_recall(A, diag), np.diagonal(A, axis1=-2, axis2=-1))
+
+
+def test_block_mass_rows_equal_the_full_map():
+    rng = np.random.default_rng(8)
+    Q = rng.standard_normal((2, 2, 300, 8))
+    K = rng.standard_normal((2, 2, 300, 8))
+    A = orc.block_mass(Q, K)
+    assert np.allclose(orc.block_mass_rows(Q, K, 1, 0, [0, 4, 2]), A[1, 0, [0, 4, 2]], atol=1e-14)
