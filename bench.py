@@ -299,6 +299,45 @@ def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
             "steps": steps, "cases": rows}
 
 
+def measure_fidelity(nabla, q, k) -> dict:
+    """The per-block fidelity check at the 720p shape: the true token-level
+    block mass of dense attention (block_mass_kernel, two dense passes of
+    S = Q K^T: 4 S^2 D flops per head) and the kept mass (recall) of the CDF
+    masks at thr 0.5 and 0.8 against fixed-budget Top-k masks with the same
+    mean number of blocks per row."""
+    import torch
+    B, H, S, D = q.shape
+    ws = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    A = nabla.block_mass(q, k, ws=ws)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    nabla.block_mass(q, k, out=A, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if nabla.workspace_status(ws) != 0:
+        raise SystemExit("device status word reports a timeout in the block-mass kernel")
+    ms = e0.elapsed_time(e1)
+    rows = []
+    for thr in (0.5, 0.8):
+        cdf = nabla.build_mask(q, k, thr, transpose=False)
+        budget = int(round(cdf.cnt.float().mean().item()))
+        tk = nabla.build_mask_topk(q, k, budget, transpose=False)
+        rc = nabla.mask_recall(A, cdf, tuple(q.shape))
+        rt = nabla.mask_recall(A, tk, tuple(q.shape))
+        nb = cdf.cnt.shape[-1]
+        rows.append({"thr": thr, "topk_budget": budget,
+                     "kept_fraction_cdf": cdf.cnt.float().mean().item() / nb,
+                     "kept_fraction_topk": tk.cnt.float().mean().item() / nb,
+                     "recall_cdf_mean": rc.mean().item(), "recall_cdf_min": rc.min().item(),
+                     "recall_topk_mean": rt.mean().item(), "recall_topk_min": rt.min().item(),
+                     "rows_cdf_better": (rc > rt).float().mean().item()})
+    flops = 4.0 * B * H * S * S * D
+    return {"workload": f"720p shape B={B} H={H} S={S} D={D} bf16, same inputs as the main line",
+            "block_mass_ms": ms, "block_mass_tflops": flops / (ms * 1e-3) / 1e12,
+            "kernel": "block_mass_kernel<128> (fidelity.cu)", "cases": rows}
+
+
 def measure_reorder(nabla, dev, warmup: int, steps: int) -> dict:
     """Fractal token reordering (§3.1.1) of [B, T*H*W, C] activations at the
     720p latent (T=21, H=45, W=80, P=8) with C = 5120 bf16 channels, forward and
@@ -461,6 +500,10 @@ def main() -> None:
     if world == 1 and not args.no_sweep:
         reorder = measure_reorder(nabla, dev, 3, 10)
 
+    fidelity = None
+    if world == 1 and not args.no_sweep:
+        fidelity = measure_fidelity(nabla, q, k)
+
     sweep = None
     if world == 1 and not args.no_sweep:
         sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
@@ -487,6 +530,7 @@ def main() -> None:
             "training": training,
             "sweep": sweep,
             "fractal_reorder": reorder,
+            "fidelity": fidelity,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }
