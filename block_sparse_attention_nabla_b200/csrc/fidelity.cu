@@ -1,6 +1,6 @@
 // Per-block fidelity of a block mask: the true token-level attention mass of
 // every 64 x 64 block, and the share of it a mask keeps.  This is the check
-// the page-1 review of "∇NABLA: Neighborhood Adaptive Block-Level Attention"
+// the pith.science review of "∇NABLA: Neighborhood Adaptive Block-Level Attention"
 // (arXiv 2507.13546v2) asks of Algorithm 1's pooling proxy: what fraction of
 // the attention mass of dense attention (§2.1, Eq. 2-3) falls inside the
 // retained blocks.

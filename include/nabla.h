@@ -126,7 +126,7 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
                               size_t workspace_bytes, nabla_stream_t stream);
 
 /* Fixed-budget variant of the mask builder: the comparator the paper sets the
- * CDF rule against (Appendix C of the v2 paper, per its page-1 review: CDF
+ * CDF rule against (Appendix C of the v2 paper, per its pith.science review: CDF
  * thresholding against a fixed Top-k at the same average block budget).
  * Identical pooling and reduced scores; every row then keeps its topk
  * largest entries of softmax(Qa Ka^T / sqrt(D)) instead of the CDF set (topk
@@ -195,8 +195,8 @@ NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, c
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 
-/* Per-block fidelity of a block mask (the check the page-1 review of the v2
- * paper asks of Algorithm 1's pooling proxy: how much of dense attention's
+/* Per-block fidelity of a block mask (the check the pith.science review of the
+ * v2 paper asks of Algorithm 1's pooling proxy: how much of dense attention's
  * token-level mass falls inside the retained blocks).
  * nabla_block_mass writes the true block mass of dense attention (§2.1,
  * Eq. 2-3, softmax over all S keys):

@@ -19,7 +19,7 @@ arXiv 2507.13546v1):
 * §2.2: the STA window is a fixed 3D window of tiles centred on the query tile.
 * §3.1.1, Figure 3: fractal flattening of the token sequence (P x P patches
   made contiguous, temporal order kept) and its inverse.
-* page 1 (review of v2, Appendix C): the fixed-budget Top-k selection the CDF
+* the pith.science review of v2 (Appendix C): the fixed-budget Top-k selection the CDF
   rule is compared with, and the per-block fidelity check of the pooling
   proxy (token-level attention mass inside the retained blocks).
 
@@ -111,7 +111,7 @@ def cdf_binarize(A: np.ndarray, thr: float):
 
 def topk_binarize(A: np.ndarray, k: int) -> np.ndarray:
     """Fixed-budget comparator of the CDF rule (the Top-k selection the paper's
-    Appendix C compares against, per the page-1 review): every row keeps its k
+    Appendix C compares against, per the pith.science review): every row keeps its k
     largest entries.  Reading: k is clipped to [1, nb]; among equal values the
     order is that of the stable ascending sort used by cdf_binarize (the
     higher column index ranks higher), so exactly k entries are kept."""
@@ -286,7 +286,7 @@ def block_mass(Q, K, N: int = BLOCK) -> np.ndarray:
     distribution p_s = softmax(q_s K^T / sqrt(D)) of every query token s over
     all S keys (§2.1, Eq. 2-3), A[i, j] is the mean over the valid query
     tokens s of block i of the mass p_s puts on the keys of block j.  Every row
-    of A sums to 1.  This is the per-block fidelity quantity the page-1 review
+    of A sums to 1.  This is the per-block fidelity quantity the pith.science review
     asks for ("what fraction of token-level attention mass falls inside the
     retained blocks").  Q, K [B, H, S, D] -> A [B, H, nb, nb]."""
     Q, K = as_f64(Q), as_f64(K)

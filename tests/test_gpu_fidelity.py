@@ -1,4 +1,4 @@
-"""GPU parity of the per-block fidelity kernels (the check the page-1 review of
+"""GPU parity of the per-block fidelity kernels (the check the pith.science review of
 "∇NABLA: Neighborhood Adaptive Block-Level Attention" asks of Algorithm 1's
 pooling proxy) against the fp64 oracle: the true token-level block mass of
 dense attention and the kept mass (recall) of a block mask.
