@@ -387,6 +387,10 @@ def main() -> None:
     ap.add_argument("--no-sweep", action="store_true", help="skip the threshold sweep and the STA case")
     ap.add_argument("--only-training", action="store_true",
                     help="run only the training leg and print its object (profiling; not a bench line)")
+    ap.add_argument("--only-reorder", action="store_true",
+                    help="run only the fractal-reorder leg and print its object (profiling; not a bench line)")
+    ap.add_argument("--only-fidelity", action="store_true",
+                    help="run only the block-fidelity leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the head count (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
@@ -405,6 +409,18 @@ def main() -> None:
         import torch
         torch.cuda.set_device(0)
         print(json.dumps(measure_training(torch.device("cuda", 0), args.warmup, max(1, args.steps))), flush=True)
+        return
+    if args.only_reorder:
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_reorder(nabla, torch.device("cuda", 0), args.warmup, max(1, args.steps))), flush=True)
+        return
+    if args.only_fidelity:
+        torch.cuda.set_device(0)
+        wf = synth.WORKLOADS[WORKLOAD_ID]
+        if args.heads:
+            wf = wf.scaled(H=args.heads)
+        xf = synth.make_inputs(wf)
+        print(json.dumps(measure_fidelity(nabla, xf["q"].cuda(), xf["k"].cuda())), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
