@@ -122,6 +122,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def rank_workload(w, rank: int):
+    """Every rank times its own independent problem of the same shape (weak
+    scaling): rank r > 0 draws its inputs from seed + 1000 r."""
+    return w.scaled(seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(values, dist=None, device=None) -> list:
+    """Element-wise maximum of per-rank timings over all ranks (the slowest
+    rank sets the job's time); unchanged without a process group."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: the kept-tile flops of all ranks' problems over
+    the max-over-ranks step time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def cpu_baseline(x: dict, thr: float, budget_s: float = 12.0) -> dict:
     """The fp64 oracle, as it stands, on a bounded sample of the workload: the
     full mask of one head, then masked attention for as many query blocks of
@@ -435,7 +458,7 @@ def main() -> None:
     w = synth.WORKLOADS[WORKLOAD_ID]
     if args.heads:
         w = w.scaled(H=args.heads, name=f"{w.name}_h{args.heads}")
-    wr = w.scaled(seed=w.seed + 1000 * rank) if rank else w
+    wr = rank_workload(w, rank)
     x = synth.make_inputs(wr)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     B, H, S, D = q.shape
@@ -480,12 +503,8 @@ def main() -> None:
     if nabla.workspace_status(ws) != 0:
         raise SystemExit("device status word reports a timeout")
 
-    if world > 1:
-        t = torch.tensor([total_ms, statistics.mean(attn_ms), statistics.mean(mask_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, attn_avg, mask_avg = t.tolist()
-    else:
-        attn_avg, mask_avg = statistics.mean(attn_ms), statistics.mean(mask_ms)
+    total_ms, attn_avg, mask_avg = max_over_ranks(
+        [total_ms, statistics.mean(attn_ms), statistics.mean(mask_ms)], dist if world > 1 else None, dev)
 
     kept_tiles = int(mask.cnt.to(torch.int64).sum().item())
     nb = mask.cnt.shape[-1]
@@ -495,7 +514,7 @@ def main() -> None:
     union_tiles = 2 * int(mask.work[:, 1].to(torch.int64).sum().item())
     flops = kept_tiles * 4 * 64 * 64 * D                     # per problem, tile basis
     ms_step = total_ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
     attn_tflops = flops / (attn_avg * 1e-3) / 1e12
     W = -(-nb // 32)
     mask_bytes = 2 * q.numel() * q.element_size() + B * H * nb * (W * 4 + 4) + kept_tiles * 4 \
@@ -581,13 +600,10 @@ def run_e2e(nabla, q, k, v, o, lse, mask, ws, stream, args, world, dist, dev, fl
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([e2e_ms], dist if world > 1 else None, dev)[0]
     h2d = 3 * q.numel() * q.element_size()
     d2h = o.numel() * o.element_size()
-    return {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
