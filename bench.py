@@ -41,9 +41,8 @@ THR = 0.8
 # reported only while the source is unchanged.  Filled from the summaries
 # under profiles/.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_tc_720p_h4.md: 384.5 MB at 4 heads, scaled x10 to 40 heads (the
-    # kernel is unchanged since; its tensor-map helpers moved to tmaps.cu)
-    "attn_fwd_tc.cu": ("941b67b4c9e4ec51746dd049faf6a8c52ebc25cdf347bc8616f8bee37bc84c6c", 3.845e9),
+    # profiles/attn_fwd_tc_720p_h4.md: 374.2 MB at 4 heads, scaled x10 to 40 heads
+    "attn_fwd_tc.cu": ("c7b4383b2fad3e53a1051a0755b29b9f12b9bc679065ff3f17f00f3b87e443a2", 3.742e9),
 }
 
 

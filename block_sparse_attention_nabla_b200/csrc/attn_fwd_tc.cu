@@ -16,8 +16,9 @@
 // Warp roles (224 threads per CTA):
 //   warp 0      Q and K producer: TMA of the unit's Q tile and of the K tiles
 //               of its key blocks (3-deep ring; a slot is refilled as soon as
-//               its S = Q K^T completes), plus one (key block, membership)
-//               record per tile; it walks the OR of the pair's two bitmask rows;
+//               its S = Q K^T completes); it walks the OR of the pair's two
+//               bitmask rows (the softmax threads walk the same rows to learn
+//               each tile's key block and membership);
 //   warp 6      V producer: the same walk, V tiles into a 2-deep ring (a slot
 //               is refilled once its O += P V completes);
 //   warp 1      TMEM owner and MMA issuer.  S of the next tile is issued before
@@ -44,10 +45,6 @@ using namespace sm100;
 
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-// Ring of per-tile (key block, membership) records.  The producer writes the
-// record of tile g only after S of tile g - 3 completed, which needs the
-// softmax of tile g - 5 done, so a record is never overwritten early.
-constexpr int kMeta = 8;
 constexpr int kCtasPerSm = 2;
 constexpr int kThreads = 224;
 constexpr uint32_t kTmemCols = 256;
@@ -69,16 +66,15 @@ struct FwdLayout {
   static constexpr uint32_t v_off = k_off + kKStages * kKVBytes;
   static constexpr uint32_t bar_off = v_off + kVStages * kKVBytes;
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2],
-  // p_full[2], o_done, o_final, drain, meta_full[kMeta]
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 3 + kMeta;
-  static constexpr uint32_t meta_off = bar_off + kNumBars * 8;
-  static constexpr uint32_t misc_off = meta_off + kMeta * 4;
+  // p_full[2], o_done, o_final, drain
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 3;
+  static constexpr uint32_t misc_off = bar_off + kNumBars * 8;
   static constexpr uint32_t bytes = misc_off + 16;
 };
 
 struct Bars {
   uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done,
-      *o_final, *drain, *meta_full;
+      *o_final, *drain;
 };
 
 // Walks the key blocks of one unit in ascending order: the set bits of the OR
@@ -100,6 +96,37 @@ struct UnitWalk {
       }
     }
     return true;
+  }
+};
+
+// The same walk as an iterator, for the softmax threads (which follow the
+// producer's order without waiting on it); the next bitmask words are
+// fetched one word ahead.
+struct WalkIter {
+  const uint32_t* ra;
+  const uint32_t* rb;
+  int W, w;
+  uint32_t wa, wb, un, na, nbw;
+  __device__ __forceinline__ WalkIter(const uint32_t* a, const uint32_t* b, int W_) : ra(a), rb(b), W(W_), w(0) {
+    wa = W > 0 ? ra[0] : 0u;
+    wb = (W > 0 && rb) ? rb[0] : 0u;
+    un = wa | wb;
+    na = W > 1 ? ra[1] : 0u;
+    nbw = (W > 1 && rb) ? rb[1] : 0u;
+  }
+  __device__ __forceinline__ void next(int& j, int& flags) {
+    while (un == 0u && w + 1 < W) {
+      ++w;
+      wa = na;
+      wb = nbw;
+      un = wa | wb;
+      na = w + 1 < W ? ra[w + 1] : 0u;
+      nbw = (w + 1 < W && rb) ? rb[w + 1] : 0u;
+    }
+    const int bit = __ffs(un) - 1;
+    un &= un - 1u;
+    j = w * 32 + bit;
+    flags = (int)((wa >> bit) & 1u) | (int)(((wb >> bit) & 1u) << 1);
   }
 };
 
@@ -130,8 +157,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   b.o_done = b.p_full + 2;
   b.o_final = b.o_done + 1;
   b.drain = b.o_final + 1;
-  b.meta_full = b.drain + 1;
-  volatile int32_t* meta = (volatile int32_t*)(smem + L::meta_off);
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
 
@@ -155,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     mbar_init(b.o_done, 1);
     mbar_init(b.o_final, 1);
     mbar_init(b.drain, 1);
-    for (int s = 0; s < kMeta; ++s) mbar_init(b.meta_full + s, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -188,11 +212,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         ++q_iter;
         const uint32_t* ra = bits + ((long long)bh * nb + 2 * p) * W;
         UnitWalk walk{ra, 2 * p + 1 < nb ? ra + W : nullptr, W};
-        ok = walk.run([&](int j, int flags) -> bool {
+        ok = walk.run([&](int j, int) -> bool {
           const uint32_t ks = g % kKStages, use = g / kKStages;
           if (use > 0 && !mbar_wait(b.k_empty + ks, (use - 1) & 1, abort_flag, limit_ns)) return false;
-          meta[g % kMeta] = j | (flags << 30);
-          mbar_arrive(b.meta_full + g % kMeta);
           mbar_expect_tx(b.k_full + ks, L::kKVBytes);
 #pragma unroll
           for (int h = 0; h < L::kHalves; ++h)
@@ -300,18 +322,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const int bh = unit / npairs, p = unit - bh * npairs;
       const int qrow = p * 128 + row;
       float m = -INFINITY, l = 0.f;
+      const uint32_t* ra = bits + ((long long)bh * nb + 2 * p) * W;
+      WalkIter walk(ra, 2 * p + 1 < nb ? ra + W : nullptr, W);
       for (uint32_t t = 0; t < n; ++t) {
         const uint32_t g = g_iter + t, sb = g & 1;
+        int j, flags;
+        walk.next(j, flags);
         const bool w1 = mbar_wait(b.s_full + sb, (g >> 1) & 1, abort_flag, limit_ns);
-        const bool w2 = w1 && mbar_wait(b.meta_full + g % kMeta, (g / kMeta) & 1, abort_flag, limit_ns);
-        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
         tc_fence_after();
-        const int mt = meta[g % kMeta];
-        const int j = mt & 0x3fffffff;
         // All 32 rows of a warp belong to the same query block of the pair,
         // so `mine` is warp-uniform: a warp whose block did not keep key
         // block j only writes P = 0.
-        const bool mine = ((mt >> 30) & my_flag) != 0;
+        const bool mine = (flags & my_flag) != 0;
         uint32_t pk[32];
         float corr = 1.f;
         bool rescale = false;
