@@ -321,6 +321,82 @@ def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
             "steps": steps, "cases": rows}
 
 
+# Table 1 of the pages (§4.1): sparsity and whole-model inference time of
+# Wan 2.1 14B at 720p on 4 x H100, printed beside this library's numbers for
+# context only (another machine, another metric).
+PAGES_TABLE1 = {"Baseline": (0.0, 8.35), "STA(18,40,40)": (79.45, 4.00), "NABLA(0.7)": (80.13, 4.02),
+                "NABLA(0.5)+STA(11,40,40)": (81.0, 3.58), "STA(18,24,24)": (91.28, 3.08),
+                "NABLA(0.4)": (92.5, 3.07), "NABLA(0.2)+STA(11,24,24)": (92.27, 3.13)}
+
+
+def measure_table1(nabla, dev, warmup: int, steps: int, heads: int | None = None) -> dict:
+    """The seven configurations of Table 1 on the padded 720p layout (21 x 48 x
+    80 = 80,640 tokens, 21 x 6 x 10 tiles): the dense baseline (thr 1.0), STA
+    alone (nabla_build_sta_mask), NABLA alone and NABLA + STA.  Per case the
+    sparsity, mask-build and attention ms/call (CUDA events on the launching
+    stream), attention TFLOP/s on kept tiles and the attention speed-up over
+    the baseline."""
+    import torch
+    import synth
+    w = synth.WORKLOADS[6]
+    if heads:
+        w = w.scaled(H=heads)
+    x = synth.make_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    coords = x["coords"].to(dev).int().contiguous()
+    B, H, S, D = q.shape
+    ws = nabla.workspace(q)
+    mask = nabla.Mask.empty(B, H, S, dev, transpose=False)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    rows = []
+    for name, thr, window in synth.TABLE1:
+        tiles = synth.sta_tiles(window) if window else None
+
+        def build():
+            if thr is None:
+                nabla.build_sta_mask(tuple(q.shape), coords, tiles, out=mask, transpose=False)
+            else:
+                nabla.build_mask(q, k, thr, sta_coords=coords if tiles else None, sta_window=tiles, out=mask,
+                                 ws=ws, transpose=False)
+
+        def one(ev=None):
+            if ev:
+                ev[0].record(stream)
+            build()
+            if ev:
+                ev[1].record(stream)
+            nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+            if ev:
+                ev[2].record(stream)
+
+        for _ in range(max(warmup, 1)):
+            one()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in evs:
+            one(e)
+        torch.cuda.synchronize()
+        if nabla.workspace_status(ws) != 0:
+            raise SystemExit("device status word reports a timeout in the Table 1 leg")
+        nb = mask.cnt.shape[-1]
+        kept = int(mask.cnt.to(torch.int64).sum().item())
+        attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        pages = PAGES_TABLE1[name]
+        rows.append({"method": name, "thr": thr, "sta_window_tokens": window, "sta_window_tiles": tiles,
+                     "kept_fraction": kept / (B * H * nb * nb), "sparsity_pct": 100.0 * (1 - kept / (B * H * nb * nb)),
+                     "mask_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs), "attn_ms": attn,
+                     "attn_tflops": kept * 4 * 64 * 64 * D / (attn * 1e-3) / 1e12,
+                     "pages_sparsity_pct": pages[0], "pages_inference_min_4xH100": pages[1]})
+    base = rows[0]["attn_ms"]
+    for r in rows:
+        r["attn_speedup_vs_baseline"] = base / r["attn_ms"]
+    return {"workload": f"table1_720p_padded: B={B} H={H} S={S} D={D} bf16, 21x48x80 tokens (frames padded "
+                        f"45 -> 48 rows), tiles 21x6x10",
+            "steps": steps, "note": "pages_* = Table 1 of the pages (Wan 2.1 14B, 4 x H100, whole-model "
+                                    "inference minutes): context only", "cases": rows}
+
+
 def measure_fidelity(nabla, q, k) -> dict:
     """The per-block fidelity check at the 720p shape: the true token-level
     block mass of dense attention (block_mass_kernel, two dense passes of
@@ -411,6 +487,8 @@ def main() -> None:
                     help="run only the training leg and print its object (profiling; not a bench line)")
     ap.add_argument("--only-reorder", action="store_true",
                     help="run only the fractal-reorder leg and print its object (profiling; not a bench line)")
+    ap.add_argument("--only-table1", action="store_true",
+                    help="run only the Table 1 configurations (padded 720p layout) and print their JSON")
     ap.add_argument("--only-fidelity", action="store_true",
                     help="run only the block-fidelity leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
@@ -435,6 +513,11 @@ def main() -> None:
     if args.only_reorder:
         torch.cuda.set_device(0)
         print(json.dumps(measure_reorder(nabla, torch.device("cuda", 0), args.warmup, max(1, args.steps))), flush=True)
+        return
+    if args.only_table1:
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_table1(nabla, torch.device("cuda", 0), max(1, args.warmup), max(1, args.steps),
+                                        args.heads)), flush=True)
         return
     if args.only_fidelity:
         torch.cuda.set_device(0)
@@ -542,6 +625,10 @@ def main() -> None:
     if world == 1 and not args.no_sweep:
         sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
 
+    table1 = None
+    if world == 1 and not args.no_sweep:
+        table1 = measure_table1(nabla, dev, 1, 2)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -563,6 +650,7 @@ def main() -> None:
             "e2e": e2e,
             "training": training,
             "sweep": sweep,
+            "table1": table1,
             "fractal_reorder": reorder,
             "fidelity": fidelity,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -31,7 +31,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc",
-           "nabla_mask_from_bits", "nabla_attn_fwd",
+           "nabla_build_sta_mask", "nabla_mask_from_bits", "nabla_attn_fwd",
            "nabla_attn_bwd", "nabla_block_mass", "nabla_mask_recall", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
            "nabla_last_error", "nabla_abi_version"]
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
     L.nabla_build_mask.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P, SZ, P]
     L.nabla_build_mask_topk.argtypes = [SH, P, P, I32, ST, MK, P, SZ, P]
     L.nabla_mask_from_bits.argtypes = [SH, P, MK, P, SZ, P]
+    L.nabla_build_sta_mask.argtypes = [SH, ST, MK, P]
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
+                 "nabla_build_sta_mask",
                  "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_block_mass",
                  "nabla_mask_recall",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
@@ -244,6 +246,22 @@ def build_mask_noalloc(q: torch.Tensor, k: torch.Tensor, thr: float,
                                           ctypes.c_float(thr),
                                           ctypes.byref(sta) if sta is not None else None,
                                           ctypes.byref(ms), _stream()), "nabla_build_mask_noalloc")
+    return out
+
+
+def build_sta_mask(q_shape, sta_coords: torch.Tensor, sta_window: tuple, dtype=torch.bfloat16,
+                   out: Mask | None = None, transpose: bool = True) -> Mask:
+    """Sliding-tile (STA) mask alone, the same for every (b, h): query block i
+    keeps key block j iff j lies in the window (in tiles) centred on i."""
+    B, H, S, D = q_shape
+    sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    if sta_coords.dtype != torch.int32 or not sta_coords.is_cuda or not sta_coords.is_contiguous():
+        raise NablaError("sta_coords must be a contiguous int32 CUDA tensor [nb, 3]")
+    sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    out = out or Mask.empty(B, H, S, sta_coords.device, transpose)
+    ms = out.as_struct()
+    _check(lib().nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(sta), ctypes.byref(ms), _stream()),
+           "nabla_build_sta_mask")
     return out
 
 

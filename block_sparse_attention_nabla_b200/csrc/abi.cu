@@ -249,6 +249,23 @@ nabla_status nabla_mask_recall(const nabla_shape* shape, const float* mass, cons
   return NABLA_OK;
 }
 
+nabla_status nabla_build_sta_mask(const nabla_shape* shape, const nabla_sta* sta, const nabla_mask* out,
+                                  nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  if (!sta || !sta->block_coords) return fail(NABLA_ERR_INVALID_ARG, "sta and sta->block_coords are required");
+  NABLA_TRY(check_i32(sta->block_coords, "sta.block_coords"));
+  if (sta->wT < 1 || sta->wH < 1 || sta->wW < 1)
+    return fail(NABLA_ERR_INVALID_ARG, "STA window sizes must be >= 1 (got %d, %d, %d)", sta->wT, sta->wH,
+                sta->wW);
+  NABLA_TRY(check_mask_out(out, true));
+  cudaStream_t st = (cudaStream_t)stream;
+  NABLA_CUDA(launch_sta_bits(d, *sta, out->bits, st), "STA mask kernel");
+  NABLA_CUDA(launch_lists_from_bits(d, out->bits, out->cnt, out->idx, st), "lists kernel");
+  return emit_derived(d, out->bits, out, st);
+}
+
 nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits,
                                   const nabla_mask* out, void* workspace, size_t workspace_bytes,
                                   nabla_stream_t stream) {

@@ -92,6 +92,8 @@ cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo,
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
                           cudaStream_t st, int topk = 0);
+// STA-only bitmask (every sample and head): the sliding-tile window alone.
+cudaError_t launch_sta_bits(const Dims& d, const nabla_sta& sta, uint32_t* bits, cudaStream_t st);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,
                                    int32_t* idx, cudaStream_t st);
 cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t* cnt_t,

@@ -413,6 +413,29 @@ void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl,
   k<<<grid, 256, 0, st>>>(L, ldl, qa, ka, rows, nb, W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
 }
 
+// ----------------------------------------------------------- STA-only masks
+// The sliding-tile mask alone (§2.2, Eq. 5; the STA rows of Table 1): one warp
+// per row (b, h, i); bit j is set iff block j lies in the window around block
+// i, the same test as the STA union of the selection.  Every row keeps at
+// least its own block.
+__global__ void __launch_bounds__(256) sta_bits_kernel(const int32_t* __restrict__ coords, long long rows,
+                                                       int nb, int W, int hT, int hH, int hW,
+                                                       uint32_t* __restrict__ bits) {
+  const long long grow = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (grow >= rows) return;  // uniform across the warp
+  const int i = (int)(grow % nb);
+  const int ti = coords[3 * i], yi = coords[3 * i + 1], xi = coords[3 * i + 2];
+  uint32_t* brow = bits + grow * W;
+  for (int t = 0; t < W; ++t) {
+    const int j = t * 32 + lane;
+    const bool keep = j < nb && abs(coords[3 * j] - ti) <= hT && abs(coords[3 * j + 1] - yi) <= hH &&
+                      abs(coords[3 * j + 2] - xi) <= hW;
+    const uint32_t word = __ballot_sync(kFull, keep);
+    if (lane == 0) brow[t] = word;
+  }
+}
+
 // ------------------------------------------------------ lists from a bitmask
 __global__ void __launch_bounds__(256) lists_kernel(const uint32_t* __restrict__ bits, long long rows,
                                                     int nb, int W, int32_t* __restrict__ cnt,
@@ -552,6 +575,14 @@ cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* 
     launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
   else
     launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sta_bits(const Dims& d, const nabla_sta& sta, uint32_t* bits, cudaStream_t st) {
+  const long long rows = d.BH() * d.nb;
+  const long long blocks = (rows * 32 + 255) / 256;
+  sta_bits_kernel<<<(unsigned)blocks, 256, 0, st>>>(sta.block_coords, rows, d.nb, d.W, sta.wT / 2, sta.wH / 2,
+                                                    sta.wW / 2, bits);
   return cudaGetLastError();
 }
 

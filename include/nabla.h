@@ -164,6 +164,23 @@ NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const 
                                                 const void* k, float thr, const nabla_sta* sta,
                                                 const nabla_mask* out, nabla_stream_t stream);
 
+/* Sliding-tile (STA) mask alone, without the NABLA selection: the STA
+ * configurations of Table 1 (§4.1) and the neighbourhood mask of §2.2 (Eq. 5).
+ *   sta    required: block_coords (device int32 [nb][3]) and the window, as in
+ *          nabla_sta; query block i keeps key block j iff j lies in the window
+ *          centred on i (every row keeps at least block i).  The same mask for
+ *          every sample and head.
+ *   out    bits, cnt, idx, work are required; cnt_t/idx_t are filled if not NULL.
+ * Needs no workspace and allocates nothing.  Errors: NABLA_ERR_INVALID_ARG for
+ * an invalid shape, a NULL sta or coordinate pointer, a window size < 1 or a
+ * missing or misaligned output; NABLA_ERR_UNSUPPORTED for a block size, D or
+ * sequence length this build does not handle (as nabla_build_mask);
+ * NABLA_ERR_CUDA if a launch fails.  The
+ * coordinates must name tiles of the grid the tokens were laid out on (for
+ * instance the result of nabla_sta_block_coords); they are not range-checked. */
+NABLA_API nabla_status nabla_build_sta_mask(const nabla_shape* shape, const nabla_sta* sta, const nabla_mask* out,
+                                            nabla_stream_t stream);
+
 /* Builds cnt, idx, work (and cnt_t, idx_t if not NULL) of `out` from a
  * caller-supplied bitmask `bits` [B, H, nb, W] (padding bits must be zero);
  * out->bits is ignored.  Lets attention run under any externally computed

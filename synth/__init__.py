@@ -113,8 +113,12 @@ class Workload:
         return Workload(**d)
 
 
-# The five workloads: a tiny fp32 case, 480p- and 720p-shaped forwards, a
-# pretraining-shaped forward+backward and a threshold sweep at the 720p shape.
+# The workloads: a tiny fp32 case, 480p- and 720p-shaped forwards, a
+# pretraining-shaped forward+backward, a threshold sweep at the 720p shape, and
+# the configurations of Table 1 (§4.1): the 720p latent with every frame padded
+# from 45 to 48 token rows, so that the 21 x 6 x 10 tiles of 8 x 8 tokens are
+# exactly the 64-token blocks (80,640 tokens; the padding rows carry synthetic
+# values like the rest).
 WORKLOADS = {
     1: Workload("tiny_fp32", 1, 2, 4, 32, 32, 64, "fp32", [0.9], 0, False),
     2: Workload("fwd_480p", 1, 40, 21, 30, 52, 128, "bf16", [0.7, 0.8, 0.9], 2, True),
@@ -122,7 +126,27 @@ WORKLOADS = {
     4: Workload("train_512", 2, 16, 16, 32, 32, 128, "bf16", [0.8], 4, False, with_grad=True),
     5: Workload("sweep_720p", 1, 40, 21, 45, 80, 128, "bf16",
                 [0.5, 0.7, 0.8, 0.9, 0.95, 1.0], 3, True),
+    6: Workload("table1_720p_padded", 1, 40, 21, 48, 80, 128, "bf16", [0.7, 0.4, 0.5, 0.2], 6, True),
 }
+
+# Table 1 (§4.1): method name, NABLA threshold (None: no NABLA selection) and
+# STA window in tokens (frames, rows, columns; None: no STA).  A window of w
+# tokens spans w / 8 tiles of 8 x 8 tokens; the frame count is already in tiles.
+TABLE1 = [
+    ("Baseline", 1.0, None),
+    ("STA(18,40,40)", None, (18, 40, 40)),
+    ("NABLA(0.7)", 0.7, None),
+    ("NABLA(0.5)+STA(11,40,40)", 0.5, (11, 40, 40)),
+    ("STA(18,24,24)", None, (18, 24, 24)),
+    ("NABLA(0.4)", 0.4, None),
+    ("NABLA(0.2)+STA(11,24,24)", 0.2, (11, 24, 24)),
+]
+
+
+def sta_tiles(window_tokens: tuple, P: int = 8) -> tuple:
+    """(frames, rows, columns) in tokens -> the window in tiles."""
+    wt, wh, ww = window_tokens
+    return (wt, wh // P, ww // P)
 
 
 def make_inputs(w: Workload, heads: list | None = None) -> dict:

@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 15
+    assert len(names) == 16
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -176,3 +176,21 @@ def test_block_mass_and_recall_argument_errors(L):
     assert L.nabla_block_mass(ctypes.byref(sh32), FAKE, FAKE, FAKE, FAKE, 256, None) == UNSUPPORTED
     assert L.nabla_mask_recall(ctypes.byref(sh), FAKE, None, FAKE, None) == INVALID
     assert L.nabla_mask_recall(ctypes.byref(sh), FAKE + 2, FAKE, FAKE, None) == INVALID
+
+
+def test_build_sta_mask_argument_errors(L):
+    sh = shape()
+    ms = mask_struct()
+    sta = nabla._Sta(FAKE, 3, 3, 3)
+    assert L.nabla_build_sta_mask(ctypes.byref(sh), None, ctypes.byref(ms), None) == INVALID
+    assert b"sta" in L.nabla_last_error()
+    assert L.nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(nabla._Sta(None, 3, 3, 3)), ctypes.byref(ms),
+                                  None) == INVALID
+    assert L.nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(nabla._Sta(FAKE + 2, 3, 3, 3)), ctypes.byref(ms),
+                                  None) == INVALID
+    assert L.nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(nabla._Sta(FAKE, 3, 0, 3)), ctypes.byref(ms),
+                                  None) == INVALID
+    assert b"window" in L.nabla_last_error()
+    assert L.nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(sta), ctypes.byref(mask_struct(bits=None)),
+                                  None) == INVALID
+    assert L.nabla_build_sta_mask(ctypes.byref(shape(block=32)), ctypes.byref(sta), ctypes.byref(ms), None) == UNSUPPORTED

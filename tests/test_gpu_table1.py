@@ -1,0 +1,80 @@
+"""GPU parity of the Table 1 configurations ("∇NABLA: Neighborhood Adaptive
+Block-Level Attention", §4.1, Table 1) on the padded Wan 720p layout
+(21 x 48 x 80 tokens = 80,640, tiles 21 x 6 x 10), through the C ABI:
+
+* STA-only masks (nabla_build_sta_mask) equal the oracle's window mask bit for
+  bit, and the two STA rows reproduce the sparsity Table 1 prints;
+* NABLA and NABLA + STA masks match the oracle outside the 1e-5 band;
+* attention under GPU-built Table 1 masks matches the oracle on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_nabla_b200 as nabla
+import synth
+from oracle import nabla_oracle as orc
+from tests import gpu_util as gu
+from tests.test_oracle_pins import _read_golden
+
+pytestmark = pytest.mark.gpu
+
+W6 = synth.WORKLOADS[6]
+HEADS = [0, 39]
+
+
+@pytest.fixture(scope="module")
+def inputs():
+    x = synth.make_inputs(W6, heads=HEADS)
+    return x
+
+
+@pytest.mark.parametrize("window", [(18, 40, 40), (18, 24, 24), (11, 40, 40), (11, 24, 24), (1, 8, 8)])
+def test_sta_only_mask_matches_oracle(window, inputs):
+    tiles = synth.sta_tiles(window)
+    coords = inputs["coords"]
+    q_shape = (1, len(HEADS), W6.S, W6.D)
+    mask = nabla.build_sta_mask(q_shape, coords.cuda(), tiles)
+    torch.cuda.synchronize()
+    G = orc.bits_to_mask(gu.gpu_bits(mask), W6.nb)
+    want = orc.sta_mask(coords.numpy(), tiles)
+    assert (G == want[None, None]).all()
+    gu.check_lists(mask, W6.nb)
+    printed = {tuple(int(v) for v in c[1]): float(c[2][0]) for c in _read_golden("sta_table1.txt")}
+    if tiles in printed:
+        assert round(100.0 * (1.0 - G.mean()), 2) == printed[tiles]
+
+
+@pytest.mark.parametrize("name,thr,window", [c for c in synth.TABLE1 if c[1] is not None and c[1] < 1.0])
+def test_nabla_table1_masks_match_oracle(name, thr, window, inputs):
+    q, k = inputs["q"].cuda(), inputs["k"].cuda()
+    tiles = synth.sta_tiles(window) if window else None
+    coords = inputs["coords"]
+    mask = nabla.build_mask(q, k, thr, sta_coords=coords.cuda() if tiles else None, sta_window=tiles)
+    torch.cuda.synchronize()
+    M, C, stam = gu.oracle_mask(inputs["q"], inputs["k"], thr, coords.numpy() if tiles else None, tiles)
+    bad, band, diff = gu.compare_mask(mask, M, C, thr, stam)
+    assert bad == 0, (name, bad, band, diff)
+    gu.check_lists(mask, W6.nb, check_transpose=False)
+
+
+@pytest.mark.parametrize("name", ["NABLA(0.2)+STA(11,24,24)", "STA(18,40,40)"])
+def test_attention_under_table1_masks_sampled_rows(name, inputs):
+    _, thr, window = next(c for c in synth.TABLE1 if c[0] == name)
+    q, k, v = (inputs[n].cuda() for n in ("q", "k", "v"))
+    coords = inputs["coords"].cuda()
+    tiles = synth.sta_tiles(window)
+    if thr is None:
+        mask = nabla.build_sta_mask(tuple(q.shape), coords, tiles)
+    else:
+        mask = nabla.build_mask(q, k, thr, sta_coords=coords, sta_window=tiles)
+    ws = nabla.workspace(q)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    G = orc.bits_to_mask(gu.gpu_bits(mask), W6.nb)
+    rng = np.random.default_rng(6)
+    rows = np.unique(np.concatenate([[0, 63, 64, 3839, 3840, W6.S - 1], rng.integers(0, W6.S, size=30)]))
+    for hi in range(len(HEADS)):
+        Or, Lr = orc.masked_attention_rows(inputs["q"], inputs["k"], inputs["v"], G, 0, hi, rows)
+        gu.assert_close(o[0, hi, rows], Or, "bf16", f"{name} head {HEADS[hi]}")
+        assert np.abs(lse[0, hi, rows].cpu().numpy() - Lr).max() < 1e-3
