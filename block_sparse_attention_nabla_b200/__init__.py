@@ -183,6 +183,23 @@ def workspace(q: torch.Tensor, want_bwd: bool = False) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=q.device)
 
 
+def _sta_struct(sta_coords: torch.Tensor | None, sta_window, S: int):
+    """The C struct for an STA window, or None.  The kernels read nb x 3 int32
+    coordinates, so anything else is refused here rather than read past."""
+    if sta_coords is None:
+        return None
+    if sta_window is None:
+        raise NablaError("sta_window is required with sta_coords")
+    nb = num_blocks(S)
+    if tuple(sta_coords.shape) != (nb, 3):
+        raise NablaError(f"sta_coords must have shape [nb, 3] = [{nb}, 3] (got {list(sta_coords.shape)})")
+    if len(sta_window) != 3:
+        raise NablaError("sta_window must be (wT, wH, wW) in tiles")
+    if sta_coords.dtype != torch.int32 or not sta_coords.is_cuda or not sta_coords.is_contiguous():
+        raise NablaError("sta_coords must be a contiguous int32 CUDA tensor [nb, 3]")
+    return _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+
+
 def build_mask(q: torch.Tensor, k: torch.Tensor, thr: float, sta_coords: torch.Tensor | None = None,
                sta_window: tuple | None = None, out: Mask | None = None, ws: torch.Tensor | None = None,
                transpose: bool = True) -> Mask:
@@ -191,13 +208,7 @@ def build_mask(q: torch.Tensor, k: torch.Tensor, thr: float, sta_coords: torch.T
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
     ws = ws if ws is not None else workspace(q)
-    sta = None
-    if sta_coords is not None:
-        if sta_window is None:
-            raise NablaError("sta_window is required with sta_coords")
-        if sta_coords.dtype != torch.int32 or not sta_coords.is_cuda or not sta_coords.is_contiguous():
-            raise NablaError("sta_coords must be a contiguous int32 CUDA tensor [nb, 3]")
-        sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
     _check(lib().nabla_build_mask(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), ctypes.c_float(thr),
                                   ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
@@ -214,11 +225,7 @@ def build_mask_topk(q: torch.Tensor, k: torch.Tensor, topk: int, sta_coords: tor
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
     ws = workspace(q) if ws is None else ws
-    sta = None
-    if sta_coords is not None:
-        if sta_window is None:
-            raise NablaError("sta_window is required with sta_coords")
-        sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
     _check(lib().nabla_build_mask_topk(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), int(topk),
                                        ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
@@ -236,11 +243,7 @@ def build_mask_noalloc(q: torch.Tensor, k: torch.Tensor, thr: float,
     sh = _shape_of(q)
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
-    sta = None
-    if sta_coords is not None:
-        if sta_window is None:
-            raise NablaError("sta_window is required with sta_coords")
-        sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
     _check(lib().nabla_build_mask_noalloc(ctypes.byref(sh), q.data_ptr(), k.data_ptr(),
                                           ctypes.c_float(thr),
@@ -255,9 +258,9 @@ def build_sta_mask(q_shape, sta_coords: torch.Tensor, sta_window: tuple, dtype=t
     keeps key block j iff j lies in the window (in tiles) centred on i."""
     B, H, S, D = q_shape
     sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
-    if sta_coords.dtype != torch.int32 or not sta_coords.is_cuda or not sta_coords.is_contiguous():
-        raise NablaError("sta_coords must be a contiguous int32 CUDA tensor [nb, 3]")
-    sta = _Sta(sta_coords.data_ptr(), *[int(w) for w in sta_window])
+    if sta_coords is None:
+        raise NablaError("sta_coords is required")
+    sta = _sta_struct(sta_coords, sta_window, S)
     out = out or Mask.empty(B, H, S, sta_coords.device, transpose)
     ms = out.as_struct()
     _check(lib().nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(sta), ctypes.byref(ms), _stream()),

@@ -194,3 +194,17 @@ def test_build_sta_mask_argument_errors(L):
     assert L.nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(sta), ctypes.byref(mask_struct(bits=None)),
                                   None) == INVALID
     assert L.nabla_build_sta_mask(ctypes.byref(shape(block=32)), ctypes.byref(sta), ctypes.byref(ms), None) == UNSUPPORTED
+
+
+def test_binding_refuses_sta_coordinates_of_the_wrong_shape():
+    import torch
+    nb = nabla.num_blocks(1000)
+    with pytest.raises(nabla.NablaError, match=r"\[nb, 3\]"):
+        nabla._sta_struct(torch.zeros(nb - 1, 3, dtype=torch.int32), (3, 3, 3), 1000)
+    with pytest.raises(nabla.NablaError, match=r"\[nb, 3\]"):
+        nabla._sta_struct(torch.zeros(nb, 2, dtype=torch.int32), (3, 3, 3), 1000)
+    with pytest.raises(nabla.NablaError, match="sta_window"):
+        nabla._sta_struct(torch.zeros(nb, 3, dtype=torch.int32), None, 1000)
+    with pytest.raises(nabla.NablaError, match="CUDA"):     # right shape, but a host tensor
+        nabla._sta_struct(torch.zeros(nb, 3, dtype=torch.int32), (3, 3, 3), 1000)
+    assert nabla._sta_struct(None, None, 1000) is None
