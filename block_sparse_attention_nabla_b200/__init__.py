@@ -132,6 +132,13 @@ def _same(ref: torch.Tensor, *ts: torch.Tensor) -> None:
             raise NablaError("tensors must be contiguous")
 
 
+def _check_f32(t: torch.Tensor, shape: tuple, device, name: str) -> None:
+    if tuple(t.shape) != tuple(shape) or t.dtype != torch.float32 or t.device != torch.device(device) \
+            or not t.is_contiguous():
+        raise NablaError(f"{name} must be a contiguous float32 tensor {list(shape)} on {device} "
+                         f"(got {list(t.shape)} {t.dtype} {t.device})")
+
+
 def num_blocks(S: int) -> int:
     return -(-S // BLOCK)
 
@@ -145,6 +152,25 @@ class Mask:
     work: torch.Tensor           # int32 [B * H * npairs, 2]
     cnt_t: torch.Tensor | None = None
     idx_t: torch.Tensor | None = None
+
+    def check(self, B: int, H: int, S: int, device, need_bits: bool = True, need_transpose: bool = False) -> None:
+        """Refuses tensors that do not have this problem's shapes: the kernels
+        index them by the shape alone."""
+        nb = num_blocks(S)
+        W, npairs = -(-nb // 32), -(-nb // 2)
+        want = {"cnt": (B, H, nb), "idx": (B, H, nb, nb), "work": (B * H * npairs, 2)}
+        if need_bits:
+            want["bits"] = (B, H, nb, W)
+        if need_transpose or self.cnt_t is not None or self.idx_t is not None:
+            want["cnt_t"], want["idx_t"] = (B, H, nb), (B, H, nb, nb)
+        for name, shape in want.items():
+            t = getattr(self, name)
+            if t is None:
+                raise NablaError(f"mask.{name} is required")
+            if (tuple(t.shape) != shape or t.dtype != torch.int32 or t.device != torch.device(device)
+                    or not t.is_contiguous()):
+                raise NablaError(f"mask.{name} must be a contiguous int32 tensor {list(shape)} on {device} "
+                                 f"(got {list(t.shape)} {t.dtype} {t.device})")
 
     def as_struct(self) -> _Mask:
         return _Mask(_ptr(self.bits), _ptr(self.cnt), _ptr(self.idx), _ptr(self.cnt_t),
@@ -207,6 +233,7 @@ def build_mask(q: torch.Tensor, k: torch.Tensor, thr: float, sta_coords: torch.T
     sh = _shape_of(q)
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
+    out.check(sh.B, sh.H, sh.S, q.device)
     ws = ws if ws is not None else workspace(q)
     sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
@@ -224,6 +251,7 @@ def build_mask_topk(q: torch.Tensor, k: torch.Tensor, topk: int, sta_coords: tor
     sh = _shape_of(q)
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
+    out.check(sh.B, sh.H, sh.S, q.device)
     ws = workspace(q) if ws is None else ws
     sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
@@ -243,6 +271,7 @@ def build_mask_noalloc(q: torch.Tensor, k: torch.Tensor, thr: float,
     sh = _shape_of(q)
     _same(q, k)
     out = out or Mask.empty(sh.B, sh.H, sh.S, q.device, transpose)
+    out.check(sh.B, sh.H, sh.S, q.device)
     sta = _sta_struct(sta_coords, sta_window, sh.S)
     ms = out.as_struct()
     _check(lib().nabla_build_mask_noalloc(ctypes.byref(sh), q.data_ptr(), k.data_ptr(),
@@ -262,6 +291,7 @@ def build_sta_mask(q_shape, sta_coords: torch.Tensor, sta_window: tuple, dtype=t
         raise NablaError("sta_coords is required")
     sta = _sta_struct(sta_coords, sta_window, S)
     out = out or Mask.empty(B, H, S, sta_coords.device, transpose)
+    out.check(B, H, S, sta_coords.device)
     ms = out.as_struct()
     _check(lib().nabla_build_sta_mask(ctypes.byref(sh), ctypes.byref(sta), ctypes.byref(ms), _stream()),
            "nabla_build_sta_mask")
@@ -276,6 +306,7 @@ def mask_from_bits(bits: torch.Tensor, q_shape, dtype=torch.bfloat16, out: Mask 
     bits = bits.to(torch.int32).contiguous()
     out = out or Mask.empty(B, H, S, bits.device, transpose)
     out.bits = bits
+    out.check(B, H, S, bits.device)
     if ws is None:
         ws = torch.empty(workspace_size(q_shape, dtype), dtype=torch.uint8, device=bits.device)
     ms = out.as_struct()
@@ -292,6 +323,7 @@ def block_mass(q: torch.Tensor, k: torch.Tensor, out: torch.Tensor | None = None
     _same(q, k)
     nb = num_blocks(sh.S)
     out = torch.empty(sh.B, sh.H, nb, nb, dtype=torch.float32, device=q.device) if out is None else out
+    _check_f32(out, (sh.B, sh.H, nb, nb), q.device, "out")
     ws = torch.zeros(256, dtype=torch.uint8, device=q.device) if ws is None else ws
     _check(lib().nabla_block_mass(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), out.data_ptr(), ws.data_ptr(),
                                   ws.numel(), _stream()), "nabla_block_mass")
@@ -302,6 +334,12 @@ def mask_recall(mass: torch.Tensor, mask: Mask, q_shape, dtype=torch.bfloat16) -
     """Kept token-level mass of every query block under `mask`, float [B, H, nb]."""
     B, H, S, D = q_shape
     sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    nb = num_blocks(S)
+    _check_f32(mass, (B, H, nb, nb), mass.device, "mass")
+    if mask.bits is None or tuple(mask.bits.shape) != (B, H, nb, -(-nb // 32)) or mask.bits.dtype != torch.int32 \
+            or mask.bits.device != mass.device or not mask.bits.is_contiguous():
+        raise NablaError(f"mask.bits must be a contiguous int32 tensor [{B}, {H}, {nb}, {-(-nb // 32)}] "
+                         f"on {mass.device}")
     rec = torch.empty(mass.shape[:-1], dtype=torch.float32, device=mass.device)
     _check(lib().nabla_mask_recall(ctypes.byref(sh), mass.data_ptr(), mask.bits.data_ptr(), rec.data_ptr(),
                                    _stream()), "nabla_mask_recall")
@@ -318,6 +356,7 @@ def fractal_reorder(x: torch.Tensor, T: int, H: int, W: int, P: int = 8, inverse
     if S != T * H * W:
         raise NablaError(f"x has {S} tokens, T * H * W = {T * H * W}")
     out = torch.empty_like(x) if out is None else out
+    _same(x, out)
     row_bytes = x[0, 0].numel() * x.element_size()
     _check(lib().nabla_fractal_reorder(x.data_ptr(), out.data_ptr(), B, T, H, W, P, row_bytes,
                                        1 if inverse else 0, _stream()), "nabla_fractal_reorder")
@@ -330,6 +369,9 @@ def attn_fwd(q, k, v, mask: Mask, o=None, lse=None, ws=None):
     _same(q, k, v)
     o = o if o is not None else torch.empty_like(q)
     lse = lse if lse is not None else torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    _same(q, o)
+    _check_f32(lse, tuple(q.shape[:3]), q.device, "lse")
+    mask.check(sh.B, sh.H, sh.S, q.device)
     ws = ws if ws is not None else workspace(q)
     ms = mask.as_struct()
     _check(lib().nabla_attn_fwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
@@ -346,6 +388,8 @@ def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None, dq=None, dk=None, dv=None
     dk = dk if dk is not None else torch.empty_like(k)
     dv = dv if dv is not None else torch.empty_like(v)
     _same(q, dq, dk, dv)
+    _check_f32(lse, tuple(q.shape[:3]), q.device, "lse")
+    mask.check(sh.B, sh.H, sh.S, q.device, need_transpose=True)
     ws = ws if ws is not None else workspace(q, want_bwd=True)
     ms = mask.as_struct()
     _check(lib().nabla_attn_bwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),

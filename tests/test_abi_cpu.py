@@ -208,3 +208,21 @@ def test_binding_refuses_sta_coordinates_of_the_wrong_shape():
     with pytest.raises(nabla.NablaError, match="CUDA"):     # right shape, but a host tensor
         nabla._sta_struct(torch.zeros(nb, 3, dtype=torch.int32), (3, 3, 3), 1000)
     assert nabla._sta_struct(None, None, 1000) is None
+
+
+def test_binding_refuses_masks_and_outputs_of_another_shape():
+    import torch
+    m = nabla.Mask.empty(1, 2, 1000, "cpu", transpose=False)
+    m.check(1, 2, 1000, "cpu")                                  # its own shape
+    with pytest.raises(nabla.NablaError, match="mask.cnt"):
+        m.check(1, 2, 2000, "cpu")                              # built for fewer blocks
+    with pytest.raises(nabla.NablaError, match="mask.cnt_t is required"):
+        m.check(1, 2, 1000, "cpu", need_transpose=True)         # the backward needs the transposed lists
+    m.work = m.work[:-1]
+    with pytest.raises(nabla.NablaError, match="mask.work"):
+        m.check(1, 2, 1000, "cpu")
+    with pytest.raises(nabla.NablaError, match="lse"):
+        nabla._check_f32(torch.zeros(1, 2, 999), (1, 2, 1000), "cpu", "lse")
+    with pytest.raises(nabla.NablaError, match="lse"):
+        nabla._check_f32(torch.zeros(1, 2, 1000, dtype=torch.float64), (1, 2, 1000), "cpu", "lse")
+    nabla._check_f32(torch.zeros(1, 2, 1000), (1, 2, 1000), "cpu", "lse")
