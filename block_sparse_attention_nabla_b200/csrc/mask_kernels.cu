@@ -530,6 +530,17 @@ cudaError_t set_smem(Kern k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+int num_sms();
+
+// Grid of at most `want` CTAs that all fit on the GPU at once.
+template <typename Kern>
+int resident_grid(Kern kern, int threads, long long want) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  return (int)std::min<long long>(want, (long long)num_sms() * per_sm);
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -548,17 +559,20 @@ cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa,
                         float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st) {
   const long long per = d.BH() * d.nb;
   const long long warps = 2 * per;
-  const int grid = (int)std::min<long long>((warps + 7) / 8, (long long)num_sms() * 8);
+  // One wave of resident CTAs walking the blocks (grid-stride), instead of
+  // more CTAs than fit at once and a partial last wave.
+  auto launch = [&](auto kern, const auto* qq, const auto* kk) {
+    const int grid = resident_grid(kern, 256, (warps + 7) / 8);
+    kern<<<grid, 256, 0, st>>>(qq, kk, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
+  };
   if (d.dtype == NABLA_BF16) {
-    if (d.D == 128)
-      pool_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
-    else
-      pool_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
+    const auto* qq = (const __nv_bfloat16*)q;
+    const auto* kk = (const __nv_bfloat16*)k;
+    if (d.D == 128) launch(pool_kernel<__nv_bfloat16, 128>, qq, kk);
+    else launch(pool_kernel<__nv_bfloat16, 64>, qq, kk);
   } else {
-    if (d.D == 128)
-      pool_kernel<float, 128><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
-    else
-      pool_kernel<float, 64><<<grid, 256, 0, st>>>((const float*)q, (const float*)k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
+    if (d.D == 128) launch(pool_kernel<float, 128>, (const float*)q, (const float*)k);
+    else launch(pool_kernel<float, 64>, (const float*)q, (const float*)k);
   }
   return cudaGetLastError();
 }

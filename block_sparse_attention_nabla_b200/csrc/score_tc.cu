@@ -15,8 +15,8 @@
 //
 // One CTA computes one 128 x 128 tile of L: warp 0 streams the four operand
 // sub-chunks (32 dimensions = one 128-byte swizzle row) with TMA, warp 1 owns
-// TMEM and issues the MMAs, then all four warps write the tile (one row per
-// thread) to the logits buffer.
+// TMEM and issues the MMAs, then all four warps write the tile to the logits
+// buffer through shared memory in coalesced row segments.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -107,30 +107,45 @@ __global__ void __launch_bounds__(128) score_gemm_kernel(
     }
     if (ok) mma_commit(done);
   }
-  // epilogue: thread r writes row m0 + r of the tile
+  // epilogue: each warp moves its 32 rows out of TMEM in 32 x 32 chunks
+  // through a shared-memory tile of its own (the operand stage is free once
+  // the MMAs are done; 16-byte chunk k of row r sits at k ^ (r & 7), so the
+  // writes and reads are conflict-free), so that every global store writes
+  // whole 128-byte row segments instead of 32 rows' 16-byte pieces.
   __syncwarp();
   const bool w = mbar_wait(done, 0, abort_flag, limit_ns);
   if (__all_sync(0xffffffffu, w)) {
     tc_fence_after();
-    const int m = m0 + warp * 32 + lane;
     const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-    float* lrow = L + ((long long)bh * nb + m) * ldl;
-#pragma unroll
+    uint8_t* tile = smem + warp * 4096;  // [32 rows][128 B]
+    const int rsub = lane >> 3, q = lane & 7;
+#pragma unroll 1
     for (int c0 = 0; c0 < 128; c0 += 32) {
       uint32_t v[32];
       tmem_ld32(taddr + c0, v);
       tmem_ld_wait();
-      if (m < nb) {
-        if (n0 + c0 + 32 <= nb) {
+      __syncwarp();  // the previous chunk's reads of the tile are done
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(lrow + n0 + c0 + e) =
-                make_float4(__uint_as_float(v[e]) * scale, __uint_as_float(v[e + 1]) * scale,
-                            __uint_as_float(v[e + 2]) * scale, __uint_as_float(v[e + 3]) * scale);
-        } else {
+      for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float4*>(tile + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+            make_float4(__uint_as_float(v[4 * k]) * scale, __uint_as_float(v[4 * k + 1]) * scale,
+                        __uint_as_float(v[4 * k + 2]) * scale, __uint_as_float(v[4 * k + 3]) * scale);
+      __syncwarp();
+      const int col = n0 + c0 + 4 * q;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (n0 + c0 + e < nb) lrow[n0 + c0 + e] = __uint_as_float(v[e]) * scale;
+      for (int k = 0; k < 8; ++k) {
+        const int r = 4 * k + rsub;  // row of the warp's 32; lanes 8 rsub .. 8 rsub + 7 cover its 128 bytes
+        const float4 x = *reinterpret_cast<const float4*>(tile + r * 128 + ((q ^ (r & 7)) << 4));
+        const int m = m0 + warp * 32 + r;
+        if (m < nb && col < nb) {
+          float* dst = L + ((long long)bh * nb + m) * ldl + col;
+          if (col + 4 <= nb) {
+            *reinterpret_cast<float4*>(dst) = x;
+          } else {
+            dst[0] = x.x;
+            if (col + 1 < nb) dst[1] = x.y;
+            if (col + 2 < nb) dst[2] = x.z;
+          }
         }
       }
     }
