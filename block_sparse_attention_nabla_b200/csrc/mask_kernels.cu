@@ -489,30 +489,65 @@ __global__ void __launch_bounds__(1024) work_kernel(const uint32_t* __restrict__
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
   const long long bh = blockIdx.x;
   const uint32_t* rb = bits + bh * nb * W;
-  for (int p = warp; p < npairs; p += nwarp) {
-    int c = 0;
-    const bool has_b = 2 * p + 1 < nb;
+  // costs, four pairs in flight per warp (the bitmask words come from L2)
+  for (int p0 = 4 * warp; p0 < npairs; p0 += 4 * nwarp) {
+    int c[4] = {0, 0, 0, 0};
     for (int w = lane; w < W; w += 32) {
-      const uint32_t a = rb[(long long)(2 * p) * W + w];
-      const uint32_t b = has_b ? rb[(long long)(2 * p + 1) * W + w] : 0u;
-      c += __popc(a | b);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = p0 + u;
+        if (p < npairs) {
+          const uint32_t a = rb[(long long)(2 * p) * W + w];
+          const uint32_t b = 2 * p + 1 < nb ? rb[(long long)(2 * p + 1) * W + w] : 0u;
+          c[u] += __popc(a | b);
+        }
+      }
     }
-    c = warp_sum_i(c);
-    if (lane == 0) keys[p] = ((unsigned long long)(nb - c) << 32) | (unsigned)p;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int cu = warp_sum_i(c[u]);
+      if (lane == 0 && p0 + u < npairs) keys[p0 + u] = ((unsigned long long)(nb - cu) << 32) | (unsigned)(p0 + u);
+    }
   }
   for (int p = npairs + tid; p < p2; p += blockDim.x) keys[p] = ~0ull;
   __syncthreads();
-  for (int kk = 2; kk <= p2; kk <<= 1) {
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < p2; i += blockDim.x) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], b = keys[ixj];
-          const bool up = (i & kk) == 0;
-          if ((a > b) == up) { keys[i] = b; keys[ixj] = a; }
+  // ascending bitonic sort of keys[0, p2) (distinct keys: the pair index is
+  // in the low word)
+  if (p2 <= (int)blockDim.x) {
+    // one key per thread in a register: exchanges within a warp by shuffle,
+    // across warps through shared memory
+    unsigned long long key = tid < p2 ? keys[tid] : ~0ull;
+    for (int kk = 2; kk <= p2; kk <<= 1) {
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        unsigned long long other;
+        if (jj >= 32) {
+          __syncthreads();
+          keys[tid] = key;
+          __syncthreads();
+          other = keys[tid ^ jj];
+        } else {
+          other = __shfl_xor_sync(kFull, key, jj);
         }
+        const bool up = (tid & kk) == 0, lower = (tid & jj) == 0;
+        key = (lower == up) ? (key < other ? key : other) : (key < other ? other : key);
       }
-      __syncthreads();
+    }
+    __syncthreads();
+    keys[tid] = key;
+    __syncthreads();
+  } else {
+    for (int kk = 2; kk <= p2; kk <<= 1) {
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        for (int i = tid; i < p2; i += blockDim.x) {
+          const int ixj = i ^ jj;
+          if (ixj > i) {
+            const unsigned long long a = keys[i], b = keys[ixj];
+            const bool up = (i & kk) == 0;
+            if ((a > b) == up) { keys[i] = b; keys[ixj] = a; }
+          }
+        }
+        __syncthreads();
+      }
     }
   }
   for (int r = tid; r < npairs; r += blockDim.x) {
@@ -619,7 +654,8 @@ cudaError_t launch_transpose_lists(const Dims& d, const uint32_t* bits, int32_t*
 cudaError_t launch_work_list(const Dims& d, const uint32_t* bits, int32_t* work, cudaStream_t st) {
   int p2 = 1;
   while (p2 < d.npairs) p2 <<= 1;
-  const size_t smem = sizeof(unsigned long long) * p2;
+  // one key per thread in the register sort (p2 <= 1024), p2 keys otherwise
+  const size_t smem = sizeof(unsigned long long) * std::max(p2, 1024);
   cudaError_t e = set_smem(work_kernel, smem);
   if (e != cudaSuccess) return e;
   work_kernel<<<(unsigned)d.BH(), 1024, smem, st>>>(bits, d.nb, d.W, d.npairs, p2, work);
