@@ -152,14 +152,15 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, cons
 // order like their bit patterns), taken on the top 16 bits: the cut-off
 // bucket is the smallest 16-bit prefix p with sum_{prefix(e_k) > p} e_k <=
 // thr * s.  Entries above the bucket are kept, entries below dropped, and the
-// entries of the bucket (relative width <= 2^-7, typically a handful) are
-// ranked by their fp64 logits (ties: higher block index first, as a stable
-// ascending sort leaves them; fp32 cannot order entries closer than its
-// rounding error) and kept in rank order while the mass above them stays
-// <= thr * s.  Then the STA window is OR-ed in and bits / cnt / idx are
+// entries of the bucket (relative width <= 2^-7: a handful at a thousand
+// blocks per row, up to ~100 at 8,192) are ranked by their fp64 logits (ties:
+// higher block index first, as a stable ascending sort leaves them; fp32
+// cannot order entries closer than its rounding error) and kept in rank order
+// while the mass above them stays <= thr * s; a bucket of more than
+// kMaxCand entries is decided in fp32 instead.  Then the STA window is OR-ed in and bits / cnt / idx are
 // written.  The row's values live in registers (NPL per lane, nb <= 32 NPL),
 // else in the logits buffer.
-constexpr int kMaxCand = 32;
+constexpr int kMaxCand = 128;
 
 struct SelectCtx {
   const double* qa_h;
@@ -171,6 +172,7 @@ struct SelectCtx {
   int hT, hH, hW;
   int (*cand_j)[kMaxCand];
   float (*cand_e)[kMaxCand];
+  double (*cand_lg)[kMaxCand];
 };
 
 // fp64 logits Qa_row . Ka_j (unscaled: a positive factor keeps the order) of
@@ -321,28 +323,72 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
       cut32 = l2;
       mode = 2;
     } else {
-      const bool act = lane < ncand;
-      const int cj = act ? c.cand_j[warp][lane] : 0;
-      const float ce = act ? c.cand_e[warp][lane] : 0.f;
-      const double lg = candidate_logits<D>(c.qa_h + (long long)row * D, c.ka_h, c.cand_j[warp], ncand, lane);
-      float mass = above;
-      for (int b2 = 0; b2 < ncand; ++b2) {
-        const double lb = __shfl_sync(kFull, lg, b2);
-        const int jb = __shfl_sync(kFull, cj, b2);
-        const float eb = __shfl_sync(kFull, ce, b2);
-        if (lb > lg || (lb == lg && jb > cj)) mass += tk ? 1.f : eb;
-      }
-      const bool kp = act && mass <= limit;
-      // hand each candidate's decision to the lane that owns its block
-      const uint32_t kmask = __ballot_sync(kFull, kp);
-      for (int b2 = 0; b2 < ncand; ++b2) {
-        const int jb = __shfl_sync(kFull, cj, b2);
-        if ((jb & 31) == lane) {
-          const bool kb = (kmask >> b2) & 1u;
-          if constexpr (NPL > 0) {
-            if (kb) keepbits |= 1ull << (jb >> 5);
-          } else {
-            Lr[jb] = kb ? 2.f : 0.f;  // 2 sits in a bucket above any e <= 1
+      if (ncand <= 32) {
+        // one candidate per lane: fp64 logits and ranking through shuffles
+        const bool act = lane < ncand;
+        const int cj = act ? c.cand_j[warp][lane] : 0;
+        const float ce = act ? c.cand_e[warp][lane] : 0.f;
+        const double lg = candidate_logits<D>(c.qa_h + (long long)row * D, c.ka_h, c.cand_j[warp], ncand, lane);
+        float mass = above;
+        for (int b2 = 0; b2 < ncand; ++b2) {
+          const double lb = __shfl_sync(kFull, lg, b2);
+          const int jb = __shfl_sync(kFull, cj, b2);
+          const float eb = __shfl_sync(kFull, ce, b2);
+          if (lb > lg || (lb == lg && jb > cj)) mass += tk ? 1.f : eb;
+        }
+        const bool kp = act && mass <= limit;
+        // hand each candidate's decision to the lane that owns its block
+        const uint32_t kmask = __ballot_sync(kFull, kp);
+        for (int b2 = 0; b2 < ncand; ++b2) {
+          const int jb = __shfl_sync(kFull, cj, b2);
+          if ((jb & 31) == lane) {
+            const bool kb = (kmask >> b2) & 1u;
+            if constexpr (NPL > 0) {
+              if (kb) keepbits |= 1ull << (jb >> 5);
+            } else {
+              Lr[jb] = kb ? 2.f : 0.f;  // 2 sits in a bucket above any e <= 1
+            }
+          }
+        }
+      } else {
+        // larger buckets (long rows): the same ranking with the candidates'
+        // logits in shared memory, 32 candidates at a time
+        // fp64 logits of the candidates, 32 at a time (lane b of a group
+        // returns candidate b's), kept in shared memory
+        const double* qrow = c.qa_h + (long long)row * D;
+        for (int c0 = 0; c0 < ncand; c0 += 32) {
+          const int nc = min(32, ncand - c0);
+          const double lg = candidate_logits<D>(qrow, c.ka_h, c.cand_j[warp] + c0, nc, lane);
+          if (lane < nc) c.cand_lg[warp][c0 + lane] = lg;
+        }
+        __syncwarp();
+        // a candidate is kept iff the weight above the bucket plus that of the
+        // candidates ranked above it is <= limit
+        for (int c0 = 0; c0 < ncand; c0 += 32) {
+          const int ci = c0 + lane;
+          const bool act = ci < ncand;
+          const int cj = act ? c.cand_j[warp][ci] : 0;
+          const double lg = act ? c.cand_lg[warp][ci] : 0.0;
+          float mass = above;
+          for (int b2 = 0; b2 < ncand; ++b2) {
+            const double lb = c.cand_lg[warp][b2];
+            const int jb = c.cand_j[warp][b2];
+            if (lb > lg || (lb == lg && jb > cj)) mass += tk ? 1.f : c.cand_e[warp][b2];
+          }
+          const bool kp = act && mass <= limit;
+          // hand each candidate's decision to the lane that owns its block
+          const uint32_t kmask = __ballot_sync(kFull, kp);
+          const int nc = min(32, ncand - c0);
+          for (int b2 = 0; b2 < nc; ++b2) {
+            const int jb = c.cand_j[warp][c0 + b2];
+            if ((jb & 31) == lane) {
+              const bool kb = (kmask >> b2) & 1u;
+              if constexpr (NPL > 0) {
+                if (kb) keepbits |= 1ull << (jb >> 5);
+              } else {
+                Lr[jb] = kb ? 2.f : 0.f;  // 2 sits in a bucket above any e <= 1
+              }
+            }
           }
         }
       }
@@ -387,12 +433,13 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
     int hW, uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
   __shared__ int cand_j[8][kMaxCand];
   __shared__ float cand_e[8][kMaxCand];
+  __shared__ double cand_lg[8][kMaxCand];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long grow = (long long)blockIdx.x * 8 + warp;  // (b * H + h) * nb + i
   if (grow >= rows) return;
   const long long bh = grow / nb;
   const int row = (int)(grow - bh * nb);
-  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, topk, coords, hT, hH, hW, cand_j, cand_e};
+  SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, topk, coords, hT, hH, hW, cand_j, cand_e, cand_lg};
   float* Lr = const_cast<float*>(L) + grow * ldl;
   uint32_t* brow = bits + grow * W;
   int32_t* irow = idx + grow * nb;

@@ -132,7 +132,7 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q,
  * largest entries of softmax(Qa Ka^T / sqrt(D)) instead of the CDF set (topk
  * >= 1, clipped to nb; entries with equal values ranked as the stable
  * ascending sort leaves them, the higher block index first; a row whose cut
- * falls inside more than 32 entries of one 2^-7-wide value bucket keeps every
+ * falls inside more than 128 entries of one 2^-7-wide value bucket keeps every
  * entry tied in fp32 with the cut-off).  STA union, outputs, workspace and
  * errors as nabla_build_mask. */
 NABLA_API nabla_status nabla_build_mask_topk(const nabla_shape* shape, const void* q, const void* k,

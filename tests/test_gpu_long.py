@@ -1,0 +1,54 @@
+"""GPU parity at long sequences, through the C ABI: the selection's 64-word
+register path (1,281 to 2,048 blocks per row), its shared-memory path (more
+than 2,048 blocks: the row stays in the logits buffer and the cut-off is
+found by binary search), the work list's shared-memory sort (more than 1,024
+query-block pairs), and the largest problem the library accepts (8,192
+blocks, S = 524,288 tokens), where the forward is checked on sampled rows.
+Masks follow Algorithm 1 of "∇NABLA: Neighborhood Adaptive Block-Level
+Attention" (§3.1.2); attention is Eq. 4 (§2.2)."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_nabla_b200 as nabla
+import synth
+from oracle import nabla_oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("nblocks,tail", [(1500, 64), (2101, 17)])
+def test_mask_and_lists_long_rows(nblocks, tail):
+    S = (nblocks - 1) * 64 + tail
+    x = synth.make_random_qkv(1, 1, S, 128, "bf16", seed=nblocks)
+    q, k = x["q"].cuda(), x["k"].cuda()
+    thr = 0.8
+    mask = nabla.build_mask(q, k, thr)
+    torch.cuda.synchronize()
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], thr)
+    bad, band, diff = gu.compare_mask(mask, M, C, thr)
+    assert bad == 0, (bad, band, diff)
+    gu.check_lists(mask, x["nb"])
+
+
+def test_largest_supported_problem_mask_and_forward():
+    S = 8192 * 64
+    x = synth.make_random_qkv(1, 1, S, 128, "bf16", seed=8192)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    thr = 0.5
+    ws = nabla.workspace(q)
+    mask = nabla.build_mask(q, k, thr, ws=ws)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], thr)
+    bad, band, diff = gu.compare_mask(mask, M, C, thr)
+    assert bad == 0, (bad, band, diff)
+    gu.check_lists(mask, x["nb"])
+    G = orc.bits_to_mask(gu.gpu_bits(mask), x["nb"])
+    rng = np.random.default_rng(8192)
+    rows = np.unique(np.concatenate([[0, 63, 64, S - 64, S - 1], rng.integers(0, S, size=20)]))
+    Or, Lr = orc.masked_attention_rows(x["q"], x["k"], x["v"], G, 0, 0, rows)
+    gu.assert_close(o[0, 0, rows], Or, "bf16", "largest problem")
+    assert np.abs(lse[0, 0, rows].cpu().numpy() - Lr).max() < 1e-3
