@@ -52,3 +52,46 @@ def test_largest_supported_problem_mask_and_forward():
     Or, Lr = orc.masked_attention_rows(x["q"], x["k"], x["v"], G, 0, 0, rows)
     gu.assert_close(o[0, 0, rows], Or, "bf16", "largest problem")
     assert np.abs(lse[0, 0, rows].cpu().numpy() - Lr).max() < 1e-3
+
+
+@pytest.mark.parametrize("nblocks,topk", [(1500, 700), (2101, 1000)])
+def test_topk_long_rows(nblocks, topk):
+    """The fixed-budget comparator on long rows: the k-th largest entry's
+    bucket is ranked by fp64 logits as in the CDF rule."""
+    from tests.test_gpu_mask import _topk_check
+    S = nblocks * 64 - 5
+    x = synth.make_random_qkv(1, 1, S, 128, "bf16", seed=nblocks + topk)
+    q, k = x["q"].cuda(), x["k"].cuda()
+    mask = nabla.build_mask_topk(q, k, topk)
+    torch.cuda.synchronize()
+    M, X = gu.oracle_topk(x["q"], x["k"], topk)
+    _topk_check(mask, M, X, x["nb"], topk)
+
+
+def test_backward_long_rows_sparse_mask():
+    """Backward with more than 2,048 blocks (long column and row lists), under a
+    sparse external mask that keeps the fp64 oracle affordable: each query
+    block keeps its own block and six random others."""
+    S = 2101 * 64 - 47
+    nb = -(-S // 64)
+    x = synth.make_random_qkv(1, 1, S, 128, "bf16", seed=2101, with_grad=True)
+    rng = np.random.default_rng(2101)
+    M = np.zeros((1, 1, nb, nb), dtype=bool)
+    for i in range(nb):
+        M[0, 0, i, rng.choice(nb, size=6, replace=False)] = True
+        M[0, 0, i, i] = True
+    M[0, 0, :, nb - 1] |= rng.random(nb) < 0.01      # some rows reach the ragged last block
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    o, lse = nabla.attn_fwd(q, k, v, mask)
+    ws = nabla.workspace(q, want_bwd=True)
+    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    gu.check_lists(mask, nb)
+    O, _ = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, "bf16", "forward")
+    dQ, dK, dV = orc.masked_attention_bwd(x["q"], x["k"], x["v"], x["do"], M)
+    gu.assert_close(dq, dQ, "bf16", "dQ", grad=True)
+    gu.assert_close(dk, dK, "bf16", "dK", grad=True)
+    gu.assert_close(dv, dV, "bf16", "dV", grad=True)
