@@ -1,0 +1,51 @@
+"""GPU edge cases through the C ABI, against the fp64 oracle: logits far
+outside the usual range (softmax rows that are one-hot in fp32, most
+exponentials underflowing), and STA windows wider than the tile grid.  Masks
+follow Algorithm 1 and the STA union of "∇NABLA: Neighborhood Adaptive
+Block-Level Attention" (§3.1.2-3.1.3); attention is Eq. 4 (§2.2)."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_nabla_b200 as nabla
+import synth
+from oracle import nabla_oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("scale", [8.0, 30.0])
+def test_extreme_logits_mask_and_forward(scale):
+    x = synth.make_random_qkv(1, 2, 1000, 128, "bf16", seed=int(scale))
+    for n in ("q", "k"):
+        x[n] = (x[n].float() * scale).to(torch.bfloat16)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    thr = 0.8
+    ws = nabla.workspace(q)
+    mask = nabla.build_mask(q, k, thr, ws=ws)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], thr)
+    bad, band, diff = gu.compare_mask(mask, M, C, thr)
+    assert bad == 0, (bad, band, diff)
+    gu.check_lists(mask, x["nb"])
+    G = orc.bits_to_mask(gu.gpu_bits(mask), x["nb"])
+    O, L = orc.masked_attention(x["q"], x["k"], x["v"], G)
+    gu.assert_close(o, O, "bf16", f"scale {scale}")
+    assert torch.isfinite(o.float()).all()
+    # the LSE comes from fp32 logits of magnitude up to ~1e3 here: allow 1e-4
+    # of that magnitude on top of the usual 1e-3
+    assert np.abs(lse.cpu().numpy() - L).max() < 1e-4 * max(1.0, float(np.abs(L).max())) + 1e-3
+
+
+def test_sta_window_wider_than_the_grid_keeps_everything():
+    w = synth.WORKLOADS[6]
+    coords = torch.from_numpy(synth.block_coords(w.T, w.Hl, w.Wl, w.P))
+    mask = nabla.build_sta_mask((1, 1, w.S, w.D), coords.cuda(), (99, 999, 999))
+    torch.cuda.synchronize()
+    G = orc.bits_to_mask(gu.gpu_bits(mask), w.nb)
+    assert G.all()
+    assert (orc.sta_mask(coords.numpy(), (99, 999, 999)) == G[0, 0]).all()
+    gu.check_lists(mask, w.nb)
