@@ -249,11 +249,23 @@ def masked_attention_rows(Q, K, V, M: np.ndarray, b: int, h: int, rows, N: int =
     return O, LSE
 
 
-def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK):
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """x rounded to fp32, then to bfloat16 (the top 16 bits of the fp32
+    pattern, rounding to nearest with ties to even), returned as fp64."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, o_format: str | None = None):
     """Gradients of masked_attention with the mask held constant: with
     P = softmax(Q K_sel^T / sqrt(D)) per query block,
       dV_sel += P^T dO,  dP = dO V_sel^T,  dS = P * (dP - rowsum(P * dP)),
       dQ = dS K_sel / sqrt(D),  dK_sel += dS^T Q / sqrt(D).
+    rowsum(P * dP) equals rowsum(dO * O).  o_format="bf16" takes that row sum
+    with O rounded to bfloat16 (round to nearest even) first: the output a
+    forward stores in bf16, which is all a backward that is handed O can use;
+    the default is the exact (textbook) gradient.
     Returns (dQ, dK, dV) fp64 [B, H, S, D]."""
     Q, K, V, dO = as_f64(Q), as_f64(K), as_f64(V), as_f64(dO)
     B, H, S, D = Q.shape
@@ -273,7 +285,12 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK):
                 g = dO[b, h, rows]
                 dV[b, h, keys] += P.T @ g
                 dP = g @ V[b, h, keys].T
-                dS = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+                if o_format == "bf16":
+                    O_rows = round_bf16(P @ V[b, h, keys])
+                    delta = (g * O_rows).sum(axis=-1, keepdims=True)
+                else:
+                    delta = (P * dP).sum(axis=-1, keepdims=True)
+                dS = P * (dP - delta)
                 dQ[b, h, rows] = dS @ K[b, h, keys] * scale
                 dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
     return dQ, dK, dV

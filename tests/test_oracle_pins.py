@@ -403,3 +403,40 @@ def test_block_mass_rows_equal_the_full_map():
     K = rng.standard_normal((2, 2, 300, 8))
     A = orc.block_mass(Q, K)
     assert np.allclose(orc.block_mass_rows(Q, K, 1, 0, [0, 4, 2]), A[1, 0, [0, 4, 2]], atol=1e-14)
+
+
+def test_round_bf16_ties_to_even_and_matches_torch():
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties go to the even pattern (1)
+    # 1 + 3 * 2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6: even is 1 + 2^-6
+    x = np.array([1.0, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 1 + 2.0 ** -7, 3.0e38, 1e-30])
+    want = np.array([1.0, 1.0, 1 + 2.0 ** -6, -1.0, 1 + 2.0 ** -7])
+    got = orc.round_bf16(x)
+    assert (got[:5] == want).all()
+    rng = np.random.default_rng(3)
+    y = rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000)
+    ref = torch.from_numpy(y.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(orc.round_bf16(y), ref)
+
+
+def test_backward_with_bf16_output_reduces_to_exact_when_o_is_bf16():
+    # every key carries the same bf16 value row v, so O = v exactly and the
+    # row sum taken with the rounded O equals the exact one
+    rng = np.random.default_rng(4)
+    S, D = 150, 16
+    Q = rng.standard_normal((1, 1, S, D))
+    K = rng.standard_normal((1, 1, S, D))
+    v = orc.round_bf16(rng.standard_normal(D))
+    V = np.broadcast_to(v, (1, 1, S, D)).copy()
+    dO = rng.standard_normal((1, 1, S, D))
+    nb = orc.num_blocks(S)
+    M = rng.random((1, 1, nb, nb)) < 0.6
+    M[0, 0, np.arange(nb), np.arange(nb)] = True
+    exact = orc.masked_attention_bwd(Q, K, V, dO, M)
+    rounded = orc.masked_attention_bwd(Q, K, V, dO, M, o_format="bf16")
+    for a, b in zip(exact, rounded):
+        assert np.abs(a - b).max() < 1e-12
+    # with generic values the rounded-O row sum does change the gradient
+    V2 = rng.standard_normal((1, 1, S, D))
+    e2 = orc.masked_attention_bwd(Q, K, V2, dO, M)[0]
+    r2 = orc.masked_attention_bwd(Q, K, V2, dO, M, o_format="bf16")[0]
+    assert np.abs(e2 - r2).max() > 1e-6
