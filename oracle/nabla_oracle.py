@@ -34,6 +34,9 @@ Readings where the paper is silent (listed with reasons in the design notes):
 * STA window: |dt| <= wT // 2, |dy| <= wH // 2, |dx| <= wW // 2 in tile units,
   truncated at the grid edge (no shifting of the window);
 * the mask is a constant of the backward pass (no gradient through pooling);
+* optionally (o_format="bf16") the backward takes rowsum(dO * O) with O
+  rounded to bfloat16, the output a bf16 forward stores and hands on, instead
+  of the exact O of the textbook gradient;
 * edge patches of a frame whose sides are not multiples of P keep their valid
   tokens, row-major.
 
