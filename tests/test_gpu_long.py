@@ -95,3 +95,21 @@ def test_backward_long_rows_sparse_mask():
     gu.assert_close(dq, dQ, "bf16", "dQ", grad=True)
     gu.assert_close(dk, dK, "bf16", "dK", grad=True)
     gu.assert_close(dv, dV, "bf16", "dV", grad=True)
+
+
+@pytest.mark.parametrize("nblocks", [2101, 8192])
+def test_block_mass_long_rows(nblocks):
+    """The block-fidelity pass on long rows (its per-row partial sums take
+    16 nb bytes of shared memory: one CTA per SM at the largest size)."""
+    S = nblocks * 64 - (5 if nblocks < 8192 else 0)
+    x = synth.make_random_qkv(1, 1, S, 128, "bf16", seed=nblocks + 7)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    A = nabla.block_mass(x["q"].cuda(), x["k"].cuda(), ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    nb = x["nb"]
+    blocks = [0, 1, nb - 1] + list(np.random.default_rng(nblocks).integers(0, nb, 3))
+    got = A[0, 0, blocks].cpu().numpy()
+    assert np.abs(got.sum(-1) - 1).max() <= 1e-3
+    ref = orc.block_mass_rows(x["q"], x["k"], 0, 0, blocks)
+    assert np.abs(got - ref).max() <= 1e-4
