@@ -46,6 +46,14 @@ def test_fwd_small_bf16(S, D, thr):
     _fwd_parity(x, M, "bf16")
 
 
+@pytest.mark.parametrize("S,D", [(1000, 128), (130, 64), (37, 128)])
+def test_fwd_small_fp32(S, D):
+    # the fp32 inputs run on the CUDA cores: ragged tails at both head sizes
+    x = synth.make_random_qkv(2, 2, S, D, "fp32", seed=5 * S + D)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.7)
+    _fwd_parity(x, M, "fp32")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_fwd_edge_masks(dtype):
     # empty rows, a full row, only the ragged tail block, a random pattern
@@ -141,6 +149,13 @@ def test_bwd_small_bf16(S, D):
     x = synth.make_random_qkv(1, 2, S, D, "bf16", seed=S, with_grad=True)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
     _bwd_parity(x, M, "bf16")
+
+
+@pytest.mark.parametrize("S,D", [(1000, 128), (130, 64)])
+def test_bwd_small_fp32(S, D):
+    x = synth.make_random_qkv(1, 2, S, D, "fp32", seed=7 * S + D, with_grad=True)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
+    _bwd_parity(x, M, "fp32")
 
 
 def test_bwd_pretraining_workload_two_heads():
