@@ -8,13 +8,16 @@
 // tile, so every MMA runs at M = 128.  The unit visits the union of the two
 // blocks' kept key blocks in ascending order; rows whose own block did not keep
 // a visited key block see it as -inf.  Units come from the mask builder's work
-// list (grouped by head so a head's K and V stay in L2, most expensive first),
-// assigned round-robin to a persistent grid of two CTAs per SM: one thread
-// issuing tcgen05 MMAs cannot keep the tensor core busy with these tile
-// shapes, two can.
+// list (grouped by head so a head's K and V stay in L2, most expensive first)
+// and are drawn in list order by a persistent grid of two CTAs per SM: each
+// CTA takes the next unit (a global counter) when it is ready for one, so the
+// CTAs finish together; one thread issuing tcgen05 MMAs cannot keep the
+// tensor core busy with these tile shapes, two can.
 //
 // Warp roles (224 threads per CTA):
-//   warp 0      Q and K producer: TMA of the unit's Q tile and of the K tiles
+//   warp 0      Q and K producer: draws the next unit and hands its index to
+//               the other roles through a 4-slot ring; TMA of the unit's Q tile
+//               and of the K tiles
 //               of its key blocks (3-deep ring; a slot is refilled as soon as
 //               its S = Q K^T completes); it walks the OR of the pair's two
 //               bitmask rows (the softmax threads walk the same rows to learn
@@ -50,6 +53,8 @@ constexpr int kThreads = 224;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kOCol = 128;
 constexpr float kRescaleLog2 = 8.0f;
+// Units in flight between the producer that draws them and the other roles.
+constexpr int kUnitRing = 4;
 // Bound of the teardown waits for this CTA's own copies and MMAs in flight;
 // independent of the (tunable) limit of the pipeline waits.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
@@ -66,15 +71,16 @@ struct FwdLayout {
   static constexpr uint32_t v_off = k_off + kKStages * kKVBytes;
   static constexpr uint32_t bar_off = v_off + kVStages * kKVBytes;
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2],
-  // p_full[2], o_done, o_final, drain
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 3;
-  static constexpr uint32_t misc_off = bar_off + kNumBars * 8;
-  static constexpr uint32_t bytes = misc_off + 16;
+  // p_full[2], o_done, o_final, drain, unit_full[R], unit_empty[R]
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 3 + 2 * kUnitRing;
+  static constexpr uint32_t misc_off = bar_off + kNumBars * 8;   // TMEM slot, abort flag
+  static constexpr uint32_t ids_off = misc_off + 16;             // unit indices [R]
+  static constexpr uint32_t bytes = ids_off + 4 * kUnitRing;
 };
 
 struct Bars {
   uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done,
-      *o_final, *drain;
+      *o_final, *drain, *unit_full, *unit_empty;
 };
 
 // Walks the key blocks of one unit in ascending order: the set bits of the OR
@@ -136,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                   const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ bits,
                   const int32_t* __restrict__ work, int n_units, int S, int nb, int W, int npairs,
                   float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                  int32_t* __restrict__ status, uint64_t limit_ns) {
+                  int32_t* __restrict__ unit_ctr, int32_t* __restrict__ status, uint64_t limit_ns) {
   using L = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The 128-byte swizzle atoms must start on 1024-byte boundaries.
@@ -157,8 +163,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   b.o_done = b.p_full + 2;
   b.o_final = b.o_done + 1;
   b.drain = b.o_final + 1;
+  b.unit_full = b.drain + 1;
+  b.unit_empty = b.unit_full + kUnitRing;
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
+  int32_t* unit_ids = (int32_t*)(smem + L::ids_off);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -180,6 +189,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     mbar_init(b.o_done, 1);
     mbar_init(b.o_final, 1);
     mbar_init(b.drain, 1);
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(b.unit_full + s, 1);
+      mbar_init(b.unit_empty + s, 2 + 128);  // V producer, MMA issuer, softmax threads
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -199,9 +212,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (warp == 0) {
     // ---------------------------------------------------- Q and K producer
     if (lane == 0) {
-      uint32_t q_iter = 0, g = 0;
+      uint32_t q_iter = 0, g = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      while (ok) {
+        // draw the next unit of the work list (-1: none left) and hand its
+        // index to the other roles through the ring
+        const uint32_t us = ku % kUnitRing;
+        if (ku >= kUnitRing && !(ok = mbar_wait(b.unit_empty + us, (ku / kUnitRing - 1) & 1, abort_flag, limit_ns)))
+          break;
+        const int drawn = atomicAdd(unit_ctr, 1);
+        const int u = drawn < n_units ? drawn : -1;
+        unit_ids[us] = u;
+        mbar_arrive(b.unit_full + us);
+        ++ku;
+        if (u < 0) break;
         const int unit = work[2 * u];
         const int bh = unit / npairs, p = unit - bh * npairs;
         if (q_iter > 0 && !(ok = mbar_wait(b.q_empty, (q_iter - 1) & 1, abort_flag, limit_ns))) break;
@@ -233,9 +257,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   } else if (warp == 6) {
     // ------------------------------------------------------------ V producer
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      while (ok) {
+        const uint32_t us = ku % kUnitRing;
+        if (!(ok = mbar_wait(b.unit_full + us, (ku / kUnitRing) & 1, abort_flag, limit_ns))) break;
+        const int u = unit_ids[us];
+        mbar_arrive(b.unit_empty + us);
+        ++ku;
+        if (u < 0) break;
         const int unit = work[2 * u];
         const int bh = unit / npairs, p = unit - bh * npairs;
         const uint32_t* ra = bits + ((long long)bh * nb + 2 * p) * W;
@@ -279,7 +309,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mma_commit(b.o_done);
         return true;
       };
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      uint32_t ku = 0;
+      while (ok) {
+        const uint32_t us = ku % kUnitRing;
+        if (!(ok = mbar_wait(b.unit_full + us, (ku / kUnitRing) & 1, abort_flag, limit_ns))) break;
+        const int u = unit_ids[us];
+        mbar_arrive(b.unit_empty + us);
+        ++ku;
+        if (u < 0) break;
         const uint32_t n = (uint32_t)work[2 * u + 1];
         if (!(ok = mbar_wait(b.q_full, q_iter & 1, abort_flag, limit_ns))) break;
         ++q_iter;
@@ -316,7 +353,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int my_flag = row < 64 ? 1 : 2;
     uint32_t g_iter = 0, u_local = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
+    uint32_t ku = 0;
+    while (ok) {
+      const uint32_t us = ku % kUnitRing;
+      const bool wu = mbar_wait(b.unit_full + us, (ku / kUnitRing) & 1, abort_flag, limit_ns);
+      if (!__all_sync(0xffffffffu, wu)) { ok = false; break; }
+      const int u = unit_ids[us];
+      mbar_arrive(b.unit_empty + us);
+      ++ku;
+      if (u < 0) break;
       const int unit = work[2 * u];
       const uint32_t n = (uint32_t)work[2 * u + 1];
       const int bh = unit / npairs, p = unit - bh * npairs;
@@ -448,6 +493,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (valid && lse) lse[(long long)bh * S + qrow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
       g_iter += n;
+      ++u_local;
     }
   }
 
@@ -480,7 +526,8 @@ cudaError_t run(const Dims& d, const void* q, const void* k, const void* v, cons
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   kern<<<grid, kThreads, FwdLayout<D>::bytes, st>>>(tq, tk, tv, bits, work, n_units, d.S, d.nb, d.W,
                                                     d.npairs, scale_log2, (__nv_bfloat16*)o, lse,
-                                                    ws_header + kWsStatus, wait_limit_ns());
+                                                    ws_header + kWsUnitCounter, ws_header + kWsStatus,
+                                                    wait_limit_ns());
   return cudaGetLastError();
 }
 

@@ -64,7 +64,7 @@ inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
 }
 
 // Header words (int32 index into the workspace).
-enum : int { kWsStatus = 0, kWsTileCounter = 1 };
+enum : int { kWsStatus = 0, kWsUnitCounter = 1 };  // both zeroed at the start of every call
 
 uint64_t wait_limit_ns();
 
