@@ -41,8 +41,8 @@ THR = 0.8
 # reported only while the source is unchanged.  Filled from the summaries
 # under profiles/.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_tc_720p_h4.md: 374.2 MB at 4 heads, scaled x10 to 40 heads
-    "attn_fwd_tc.cu": ("c7b4383b2fad3e53a1051a0755b29b9f12b9bc679065ff3f17f00f3b87e443a2", 3.742e9),
+    # profiles/attn_fwd_tc_720p_h4.md: 304.9 MB at 4 heads, scaled x10 to 40 heads
+    "attn_fwd_tc.cu": ("88c3d65e11d641849bfd132cdf6c2d53eb8eb451264329b32b75d248b9a050ee", 3.049e9),
 }
 
 
