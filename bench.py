@@ -271,12 +271,13 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
             "gpu_launches_per_step": 9}
 
 
-def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
+def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int, with_sta: bool = True,
+                  inputs: str = "same inputs as the main line") -> dict:
     """The sparsity sweep at the 720p shape (thresholds 0.5 ... 1.0, the last
-    the dense path) and the threshold-0.8 mask OR-ed with the STA window of
-    3 x 3 x 3 tiles: per case the kept fraction, mask-build and attention
-    ms/call and the attention TFLOP/s on kept tiles (CUDA events on the
-    launching stream)."""
+    the dense path) and, with_sta, the threshold-0.8 mask OR-ed with the STA
+    window of 3 x 3 x 3 tiles: per case the kept fraction, mask-build and
+    attention ms/call and the attention TFLOP/s on kept tiles (CUDA events on
+    the launching stream)."""
     import torch
     B, H, S, D = q.shape
     ws = nabla.workspace(q)
@@ -285,7 +286,7 @@ def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
     lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
     stream = torch.cuda.current_stream()
     rows = []
-    cases = [(t, False) for t in (0.5, 0.7, 0.8, 0.9, 0.95, 1.0)] + [(0.8, True)]
+    cases = [(t, False) for t in (0.5, 0.7, 0.8, 0.9, 0.95, 1.0)] + ([(0.8, True)] if with_sta else [])
     for thr, sta in cases:
         kw = dict(sta_coords=coords, sta_window=(3, 3, 3)) if sta else {}
 
@@ -317,8 +318,23 @@ def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int) -> dict:
     dense = next(r for r in rows if r["thr"] == 1.0)
     for r in rows:
         r["speedup_vs_dense"] = dense["attn_ms"] / r["attn_ms"]
-    return {"workload": f"720p shape B={B} H={H} S={S} D={D} bf16, same inputs as the main line",
+    return {"workload": f"720p shape B={B} H={H} S={S} D={D} bf16, {inputs}",
             "steps": steps, "cases": rows}
+
+
+def measure_sweep_sigma06(nabla, dev, warmup: int, steps: int) -> dict:
+    """The same sweep on the 720p inputs drawn with block means and locality
+    anchors of standard deviation 0.6 (same seed: the same noise, block
+    structure scaled by 1.2), whose masks are as sparse as Table 1's NABLA
+    rows (about 92 % at thr 0.7, 82 % at thr 0.8)."""
+    import synth
+    w = synth.WORKLOADS[7]
+    x = synth.make_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    out = measure_sweep(nabla, q, k, v, None, warmup, steps, with_sta=False,
+                        inputs=f"{w.name}: block means and anchors of std {w.sigma}, seed {w.seed}")
+    del q, k, v
+    return out
 
 
 # Table 1 of the pages (§4.1): sparsity and whole-model inference time of
@@ -489,6 +505,8 @@ def main() -> None:
                     help="run only the fractal-reorder leg and print its object (profiling; not a bench line)")
     ap.add_argument("--only-table1", action="store_true",
                     help="run only the Table 1 configurations (padded 720p layout) and print their JSON")
+    ap.add_argument("--only-sweep", action="store_true",
+                    help="run only the two threshold sweeps and print their JSON (not a bench line)")
     ap.add_argument("--only-fidelity", action="store_true",
                     help="run only the block-fidelity leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
@@ -518,6 +536,18 @@ def main() -> None:
         torch.cuda.set_device(0)
         print(json.dumps(measure_table1(nabla, torch.device("cuda", 0), max(1, args.warmup), max(1, args.steps),
                                         args.heads)), flush=True)
+        return
+    if args.only_sweep:
+        torch.cuda.set_device(0)
+        dev0 = torch.device("cuda", 0)
+        ws_ = synth.WORKLOADS[WORKLOAD_ID]
+        xs = synth.make_inputs(ws_)
+        qs, ks, vs = (xs[n].to(dev0) for n in ("q", "k", "v"))
+        first = measure_sweep(nabla, qs, ks, vs, xs["coords"].to(dev0).int().contiguous(), max(1, args.warmup),
+                              max(1, args.steps))
+        del qs, ks, vs
+        print(json.dumps({"sweep": first, "sweep_sigma06": measure_sweep_sigma06(
+            nabla, dev0, max(1, args.warmup), max(1, args.steps))}), flush=True)
         return
     if args.only_fidelity:
         torch.cuda.set_device(0)
@@ -625,6 +655,10 @@ def main() -> None:
     if world == 1 and not args.no_sweep:
         sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
 
+    sweep06 = None
+    if world == 1 and not args.no_sweep:
+        sweep06 = measure_sweep_sigma06(nabla, dev, 1, 2)
+
     table1 = None
     if world == 1 and not args.no_sweep:
         table1 = measure_table1(nabla, dev, 1, 2)
@@ -650,6 +684,7 @@ def main() -> None:
             "e2e": e2e,
             "training": training,
             "sweep": sweep,
+            "sweep_sigma06": sweep06,
             "table1": table1,
             "fractal_reorder": reorder,
             "fidelity": fidelity,

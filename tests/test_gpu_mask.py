@@ -75,6 +75,16 @@ def test_mask_720p_full_size(sta):
         gu.check_lists(mask, w.nb, check_transpose=False)
 
 
+@pytest.mark.parametrize("thr", [0.5, 0.8, 0.95])
+def test_mask_720p_sigma06_sparse_masks(thr):
+    # block means of std 0.6: 1.6 % of tiles kept at thr 0.5, 18 % at 0.8
+    w = synth.WORKLOADS[7]
+    x, mask, M, C, _ = _run(w, heads=list(range(0, 40, 5)), thr=thr)
+    bad, band, diff = gu.compare_mask(mask, M, C, thr)
+    assert bad == 0, (bad, band, diff)
+    gu.check_lists(mask, w.nb, check_transpose=(thr == 0.5))
+
+
 def test_mask_sta_only_window_matches_oracle():
     # thr tiny: the NABLA part keeps only each row's top block, STA adds its window.
     w = synth.WORKLOADS[3].scaled(H=2)
