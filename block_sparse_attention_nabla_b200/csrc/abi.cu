@@ -321,7 +321,7 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(check_tensor(dk, "dk"));
   NABLA_TRY(check_tensor(dv, "dv"));
   NABLA_TRY(check_i32(lse, "lse"));
-  NABLA_TRY(check_mask_out(mask, false));
+  NABLA_TRY(check_mask_out(mask, true));
   if (!mask->cnt_t) return fail(NABLA_ERR_INVALID_ARG, "backward needs mask.cnt_t and mask.idx_t");
   NABLA_TRY(check_ws(d, true, workspace, workspace_bytes));
   cudaStream_t st = (cudaStream_t)stream;
@@ -329,7 +329,7 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(reset_status(workspace, st));
   char* ws = (char*)workspace;
   if (d.dtype == NABLA_BF16 && d.D == 128)
-    NABLA_CUDA(launch_attn_bwd_tc(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t, mask->idx_t,
+    NABLA_CUDA(launch_attn_bwd_tc(d, q, k, v, o, dout, lse, mask->bits, mask->cnt, mask->idx, mask->cnt_t,
                                   (float*)(ws + L.lse2p), (float*)(ws + L.deltap), dq, dk, dv,
                                   (int32_t*)ws, st),
                "tensor-core attention backward");

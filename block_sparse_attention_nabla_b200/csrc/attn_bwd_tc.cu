@@ -9,18 +9,22 @@
 //     dK = dS^T Q / sqrt(D)                 dQ = dS K / sqrt(D)
 //
 // The LSE of the forward makes every tile independent, so no online softmax
-// is needed and both orientations of a tile are equally cheap.  That lets a
-// step stack ANY two kept blocks of a list into one M = 128 operand: no tile
-// outside the mask is ever computed.
+// is needed and both orientations of a tile are equally cheap.  dQ stacks any
+// two kept blocks of a row list into one M = 128 operand (no tile outside the
+// mask is computed); dK / dV pairs neighbouring key blocks as the forward
+// pairs query blocks, so that P^T and dS^T can stay in TMEM as MMA operands,
+// and computes the union of the pair's columns (rows of a key block that did
+// not keep a visited query block get P = dS = 0).
 //
-//   dkdv_tc_kernel  one unit = one key block j; a step takes the next two
-//                   query blocks of j's column list (i0, i1):
-//                     S  = [Q_i0; Q_i1] K_j^T     (M = 128 queries, N = 64)
-//                     dP = [dO_i0; dO_i1] V_j^T
-//                     P, dS per query row (one thread per row), written to
-//                     shared memory as bf16
-//                     dV^T += [dO_i0; dO_i1]^T P   (M = D, N = 64, K = 128)
-//                     dK^T += [Q_i0; Q_i1]^T dS
+//   dkdv_tc_kernel  one unit = two key blocks (j0, j1) stacked into 128 key
+//                   rows; a step takes the next query block i of the union
+//                   of their two bitmask columns:
+//                     S^T  = [K_j0; K_j1] Q_i^T   (M = 128 keys, N = 64)
+//                     dP^T = [V_j0; V_j1] dO_i^T
+//                     P^T, dS^T per key row (one thread per row and half of
+//                     the columns), written back into TMEM as bf16
+//                     dV += P^T dO_i, dK += dS^T Q_i   (M = 128, N = D, A from
+//                     TMEM: only Q_i and dO_i come from shared memory)
 //   dq_tc_kernel    one unit = one query block i; a step takes the next two
 //                   key blocks of i's row list (j0, j1):
 //                     S^T  = [K_j0; K_j1] Q_i^T    (M = 128 keys, N = 64)
@@ -28,25 +32,26 @@
 //                     dS^T per key row, to shared memory as bf16
 //                     dQ^T += [K_j0; K_j1]^T dS^T  (M = D, N = 64, K = 128)
 //
-// Every MMA has N = 64, where one issuing thread reaches about a third of the
-// tensor core's rate; each kernel therefore issues its independent MMA
-// streams from separate warps (S, dP, dV, dK: four issuers; S^T, dP^T, dQ^T:
-// three), which together keep the tensor core fed.  One CTA per SM, persistent
-// over the units.  The step's stages form a chain (load -> S, dP -> P, dS ->
-// accumulate -> slot free), so every hand-off is buffered to let consecutive
-// steps overlap: S and dP double-buffered in TMEM (256 columns, plus the
-// accumulators), P and dS double-buffered in shared memory, and TMA rings for
-// the stepped operands (dkdv: 2 stages of Q + dO; dq: 3 stages of K, and 2 of
-// V, which is free as soon as dP^T completes).
+// Each kernel issues its independent MMA streams from separate warps (S^T,
+// dP^T, dV, dK: four issuers; S^T, dP^T, dQ^T: three), which together keep
+// the tensor core fed at these N = 64 / 128 shapes.  One CTA per SM,
+// persistent over the units.  The step's stages form a chain (load -> S, dP
+// -> P, dS -> accumulate -> slot free), so every hand-off is buffered to let
+// consecutive steps overlap: S and dP double-buffered in TMEM (256 columns,
+// plus the accumulators), P^T / dS^T in TMEM over them (dkdv) or dS^T
+// double-buffered in shared memory (dq), and TMA rings for the stepped
+// operands (dkdv: 4 stages of Q_i + dO_i; dq: 3 stages of K, and 2 of V,
+// which is free as soon as dP^T completes).
 //
 // Warp roles (dkdv: 13 warps; dq: 12 warps):
 //   warp 0       TMA producer (fixed operands per unit, stepped operands per
-//                step, and the rows' 1/ln2-scaled LSE and Delta);
+//                step, and the rows' 1/ln2-scaled LSE and Delta; in dkdv the
+//                whole warp scans the bitmask columns for the steps);
 //   warps 1..    MMA issuers (one thread each), warp 1 also owns TMEM;
 //   last eight   elementwise warps: a thread owns one row (TMEM lane) and half
-//                of its 64 columns: P and dS; then the epilogue (a thread owns
-//                one column d of a transposed accumulator, half of its keys or
-//                queries).
+//                of its 64 columns: P and dS; then the epilogue (dkdv: a
+//                thread writes its key row of dV or of dK; dq: a thread owns
+//                one column d of dQ^T and half of its queries).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -75,21 +80,24 @@ constexpr uint32_t kTile128 = 128 * kRowBytes;   // 128 rows x 64 columns
 constexpr uint32_t kFixed = 2 * kTile64;         // 64 rows x D = 128 (two column halves)
 constexpr uint32_t kStacked = 2 * kTile128;      // 128 rows x D = 128
 
-// Shared-memory plan of dkdv_tc_kernel (byte offsets; every tile 1024-aligned).
+// Shared-memory plan of dkdv_tc_kernel (byte offsets; every tile 1024-aligned):
+// the unit's stacked K and V pairs (128 rows x D, the A operands of S^T and
+// dP^T) and kDkdvStages stages of one query block each: Q_i, dO_i (64 rows x
+// D), LSE2 and Delta of its 64 rows, and the step record (query block,
+// membership flags, steps of the unit).
+constexpr int kDkdvStages = 4;
 struct DkdvSmem {
-  static constexpr uint32_t k_off = 0;
-  static constexpr uint32_t v_off = kFixed;
-  static constexpr uint32_t kStage = 2 * kStacked + 1024;  // Q pair, dO pair, LSE2[128], Delta[128]
-  static constexpr uint32_t stage0 = 2 * kFixed;
-  static constexpr uint32_t p0 = stage0 + 2 * kStage;      // P[2]
-  static constexpr uint32_t ds0 = p0 + 2 * kTile128;       // dS[2]
-  static constexpr uint32_t bar_off = ds0 + 2 * kTile128;
-  static constexpr int kBars = 17;
+  static constexpr uint32_t kp_off = 0;
+  static constexpr uint32_t vp_off = kStacked;
+  static constexpr uint32_t kStage = 2 * kFixed + 1024;
+  static constexpr uint32_t stats = 2 * kFixed;       // within a stage: LSE2[64], Delta[64]
+  static constexpr uint32_t record = 2 * kFixed + 512;  // within a stage: i, flags, n
+  static constexpr uint32_t stage0 = 2 * kStacked;
+  static constexpr uint32_t bar_off = stage0 + kDkdvStages * kStage;
+  static constexpr int kBars = 2 + 2 * kDkdvStages + 2 + 2 + 2 + 3;
   static constexpr uint32_t misc_off = bar_off + kBars * 8;
   static constexpr uint32_t bytes = misc_off + 16;
   static __host__ __device__ constexpr uint32_t stage(uint32_t s) { return stage0 + s * kStage; }
-  static __host__ __device__ constexpr uint32_t p(uint32_t b) { return p0 + b * kTile128; }
-  static __host__ __device__ constexpr uint32_t ds(uint32_t b) { return ds0 + b * kTile128; }
 };
 
 // Shared-memory plan of dq_tc_kernel.
@@ -110,7 +118,7 @@ struct DqSmem {
   static __host__ __device__ constexpr uint32_t ds(uint32_t b) { return ds0 + b * kTile128; }
 };
 
-static_assert(DkdvSmem::stage(1) % 1024 == 0 && DkdvSmem::p0 % 1024 == 0 && DkdvSmem::ds0 % 1024 == 0,
+static_assert(DkdvSmem::vp_off % 1024 == 0 && DkdvSmem::stage(1) % 1024 == 0 && DkdvSmem::kStage % 1024 == 0,
               "tile alignment");
 static_assert(DqSmem::k0 % 1024 == 0 && DqSmem::v0 % 1024 == 0 && DqSmem::ds0 % 1024 == 0, "tile alignment");
 static_assert(DkdvSmem::bytes <= 227 * 1024 && DqSmem::bytes <= 227 * 1024, "shared memory");
@@ -158,33 +166,47 @@ __device__ __forceinline__ void p_ds_pairs(const uint32_t (&sr)[32], const uint3
 }
 
 // ============================================================== dK and dV
+// One unit = the key blocks (j0, j1) = (2 jp, 2 jp + 1) of one (b, h), stacked
+// into 128 key rows; its steps are the query blocks i that kept j0 or j1 (the
+// union of the two columns of the bitmask, ascending), one per step:
+//   S^T  = [K_j0; K_j1] Q_i^T     dP^T = [V_j0; V_j1] dO_i^T   (M = 128, N = 64)
+//   P^T, dS^T per key row, written back into TMEM (bf16) over S^T and dP^T
+//   dV  += P^T dO_i                dK  += dS^T Q_i              (M = 128, N = D,
+//                                                               A from TMEM)
+// so shared memory serves only the step's Q_i and dO_i to the tensor core
+// (plus the unit's fixed K and V pairs).  Rows of a key block that query block
+// i did not keep get P = dS = 0.
+// TMEM: [0, 128) S^T / dP^T buffer 0, [128, 256) buffer 1 (S^T in the first 64
+// columns, dP^T in the next 64; the bf16 P^T and dS^T of the 32 query columns
+// an elementwise warp owns go into the first 16 of its own 32 columns), then
+// dV [256, 384) and dK [384, 512).
 template <int D>
 __global__ void __launch_bounds__(kDkdvThreads, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const float* __restrict__ lse2p, const float* __restrict__ deltap,
-                   const int32_t* __restrict__ cnt_t, const int32_t* __restrict__ idx_t, int n_units, int S,
-                   int nb, float scale, float scale_log2, __nv_bfloat16* __restrict__ dk,
+                   const uint32_t* __restrict__ bits, const int32_t* __restrict__ cnt_t, int n_units,
+                   int npairs, int S, int nb, int W, float scale, float scale_log2, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, int32_t* __restrict__ status, uint64_t limit_ns) {
   static_assert(D == 128, "the tensor-core backward is built for D = 128");
   using L = DkdvSmem;
+  constexpr int KS = kDkdvStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) atomicCAS(status, 0, (int32_t)NABLA_ERR_UNSUPPORTED);
     return;
   }
   uint64_t* bars = (uint64_t*)(smem + L::bar_off);
-  uint64_t* fixed_full = bars;        // K_j, V_j landed
-  uint64_t* fixed_empty = bars + 1;   // S and dP of the unit done with them
-  uint64_t* in_full = bars + 2;       // [2] Q / dO pair + stats landed
-  uint64_t* in_empty = bars + 4;      // [2] dV and dK of the step done with them
-  uint64_t* s_full = bars + 6;        // [2] S and dP in TMEM
-  uint64_t* s_free = bars + 8;        // [2] S and dP read out of TMEM
-  uint64_t* pd_full = bars + 10;      // [2] P and dS written
-  uint64_t* pd_empty = bars + 12;     // [2] dV and dK done with P and dS
-  uint64_t* acc_full = bars + 14;
-  uint64_t* acc_empty = bars + 15;
-  uint64_t* drain = bars + 16;
+  uint64_t* fixed_full = bars;             // K and V pairs landed
+  uint64_t* fixed_empty = bars + 1;        // S^T and dP^T of the unit done with them
+  uint64_t* in_full = bars + 2;            // [KS] Q_i, dO_i, stats, record landed
+  uint64_t* in_empty = bars + 2 + KS;      // [KS] dV and dK of the step done with them
+  uint64_t* s_full = bars + 2 + 2 * KS;    // [2] S^T and dP^T in TMEM
+  uint64_t* pd_full = s_full + 2;          // [2] P^T and dS^T written to TMEM
+  uint64_t* pd_empty = s_full + 4;         // [2] dV and dK done with P^T and dS^T
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* acc_empty = s_full + 7;
+  uint64_t* drain = s_full + 8;
   uint32_t* tmem_slot = (uint32_t*)(smem + L::misc_off);
   volatile int* abort_flag = (volatile int*)(smem + L::misc_off + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -192,13 +214,14 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(fixed_full, 1);
     mbar_init(fixed_empty, 2);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(in_full + s, 1);
       mbar_init(in_empty + s, 2);
-      mbar_init(s_full + s, 2);
-      mbar_init(s_free + s, kEwThreads);
-      mbar_init(pd_full + s, kEwThreads);
-      mbar_init(pd_empty + s, 2);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 2);
+      mbar_init(pd_full + b, kEwThreads);
+      mbar_init(pd_empty + b, 2);
     }
     mbar_init(acc_full, 2);
     mbar_init(acc_empty, kEwThreads);
@@ -219,83 +242,119 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
+  // A unit without steps (neither key block kept by any query block) is
+  // skipped by the producer and the S^T / dP^T issuers; the dV / dK issuers and
+  // the epilogue still run it (zeros).  Every role decides it the same way.
+  auto unit_empty = [&](int bh, int j0) -> bool {
+    const int32_t* c = cnt_t + (long long)bh * nb;
+    return c[j0] + (j0 + 1 < nb ? c[j0 + 1] : 0) == 0;
+  };
+  auto record = [&](uint32_t s) -> const int* { return (const int*)(smem + L::stage(s) + L::record); };
 
   if (warp == 0) {
     // -------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      uint32_t g = 0, fixed_it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int n = cnt_t[u];
-        if (n == 0) continue;
-        const int bh = u / nb, j = u - bh * nb;
-        const int32_t* list = idx_t + (long long)u * nb;
-        int nx0 = list[0], nx1 = n > 1 ? list[1] : nx0;  // the next step's pair, read one step early
-        if (fixed_it > 0 && !(ok = mbar_wait(fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns))) break;
-        mbar_expect_tx(fixed_full, 2 * kFixed);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tma_load_3d(smem + L::k_off + h * kTile64, &tm_k, fixed_full, h * 64, j * 64, bh);
-          tma_load_3d(smem + L::v_off + h * kTile64, &tm_v, fixed_full, h * 64, j * 64, bh);
-        }
-        ++fixed_it;
-        for (int t = 0; 2 * t < n; ++t, ++g) {
-          const int i0 = nx0, i1 = nx1;
-          if (2 * t + 2 < n) {
-            nx0 = list[2 * t + 2];
-            nx1 = 2 * t + 3 < n ? list[2 * t + 3] : nx0;
-          }
-          const uint32_t s = g & 1, use = g >> 1;
-          if (use > 0 && !(ok = mbar_wait(in_empty + s, (use - 1) & 1, abort_flag, limit_ns))) break;
-          uint8_t* st = smem + L::stage(s);
-          mbar_expect_tx(in_full + s, 2 * kStacked + 1024);
+    // The whole warp scans the unit's two bitmask columns (j0 is even, so
+    // both bits sit in one word of every row), 32 query blocks per ballot;
+    // lane 0 issues the copies.
+    uint32_t g = 0, fixed_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int bh = u / npairs, j0 = 2 * (u - bh * npairs);
+      if (unit_empty(bh, j0)) continue;
+      const bool has1 = j0 + 1 < nb;
+      const int j1 = has1 ? j0 + 1 : j0;  // a lone last block is loaded twice; its rows are masked
+      const uint32_t fmask = has1 ? 3u : 1u;
+      const uint32_t* col = bits + (long long)bh * nb * W + (j0 >> 5);
+      const int sh = j0 & 31;
+      auto flags_of = [&](int i) -> uint32_t { return i < nb ? (col[(long long)i * W] >> sh) & fmask : 0u; };
+      int n = 0;
+      for (int i0 = 0; i0 < nb; i0 += 32) n += __popc(__ballot_sync(0xffffffffu, flags_of(i0 + lane) != 0u));
+      if (lane == 0) {
+        if (fixed_it > 0) ok = mbar_wait(fixed_empty, (fixed_it - 1) & 1, abort_flag, limit_ns);
+        if (ok) {
+          mbar_expect_tx(fixed_full, 2 * kStacked);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tma_load_3d(st + h * kTile128, &tm_q, in_full + s, h * 64, i0 * 64, bh);
-            tma_load_3d(st + h * kTile128 + kTile64, &tm_q, in_full + s, h * 64, i1 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128, &tm_do, in_full + s, h * 64, i0 * 64, bh);
-            tma_load_3d(st + kStacked + h * kTile128 + kTile64, &tm_do, in_full + s, h * 64, i1 * 64, bh);
+            tma_load_3d(smem + L::kp_off + h * kTile128, &tm_k, fixed_full, h * 64, j0 * 64, bh);
+            tma_load_3d(smem + L::kp_off + h * kTile128 + kTile64, &tm_k, fixed_full, h * 64, j1 * 64, bh);
+            tma_load_3d(smem + L::vp_off + h * kTile128, &tm_v, fixed_full, h * 64, j0 * 64, bh);
+            tma_load_3d(smem + L::vp_off + h * kTile128 + kTile64, &tm_v, fixed_full, h * 64, j1 * 64, bh);
           }
-          const long long r0 = ((long long)bh * nb + i0) * 64, r1 = ((long long)bh * nb + i1) * 64;
-          bulk_load(st + 2 * kStacked, lse2p + r0, 256, in_full + s);
-          bulk_load(st + 2 * kStacked + 256, lse2p + r1, 256, in_full + s);
-          bulk_load(st + 2 * kStacked + 512, deltap + r0, 256, in_full + s);
-          bulk_load(st + 2 * kStacked + 768, deltap + r1, 256, in_full + s);
         }
       }
-      // Let every copy issued land before the CTA exits.
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++fixed_it;
+      for (int i0 = 0; i0 < nb && ok; i0 += 32) {
+        const uint32_t f = flags_of(i0 + lane);
+        uint32_t m = __ballot_sync(0xffffffffu, f != 0u);
+        while (m != 0u && ok) {
+          const int l = __ffs(m) - 1;
+          m &= m - 1u;
+          const int i = i0 + l;
+          const int fl = __shfl_sync(0xffffffffu, (int)f, l);
+          if (lane == 0) {
+            const uint32_t s = g % KS, use = g / KS;
+            if (use > 0) ok = mbar_wait(in_empty + s, (use - 1) & 1, abort_flag, limit_ns);
+            if (ok) {
+              uint8_t* st = smem + L::stage(s);
+              int* rec = (int*)(st + L::record);
+              rec[0] = i;
+              rec[1] = fl;
+              rec[2] = n;
+              mbar_expect_tx(in_full + s, 2 * kFixed + 512);  // also releases the record
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                tma_load_3d(st + h * kTile64, &tm_q, in_full + s, h * 64, i * 64, bh);
+                tma_load_3d(st + kFixed + h * kTile64, &tm_do, in_full + s, h * 64, i * 64, bh);
+              }
+              const long long r0 = ((long long)bh * nb + i) * 64;
+              bulk_load(st + L::stats, lse2p + r0, 256, in_full + s);
+              bulk_load(st + L::stats + 256, deltap + r0, 256, in_full + s);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++g;
+        }
+      }
+    }
+    // Let every copy issued land before the CTA exits.
+    if (lane == 0) {
       if (fixed_it > 0) mbar_wait(fixed_full, (fixed_it - 1) & 1, nullptr, kDrainLimitNs);
-      for (uint32_t i = (g > 2 ? g - 2 : 0); i < g; ++i)
-        mbar_wait(in_full + (i & 1), (i >> 1) & 1, nullptr, kDrainLimitNs);
+      for (uint32_t i = (g > (uint32_t)KS ? g - KS : 0); i < g; ++i)
+        mbar_wait(in_full + i % KS, (i / KS) & 1, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1 || warp == 2) {
-    // ---------------------------------------- S and dP issuers (one each)
+    // ---------------------------------------- S^T and dP^T issuers (one each)
     if (lane == 0) {
       const bool is_s = warp == 1;
       constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t fixed_base = sbase + (is_s ? L::k_off : L::v_off);
+      const uint32_t a_base = sbase + (is_s ? L::kp_off : L::vp_off);
       const uint32_t col = is_s ? 0u : 64u;
       uint32_t g = 0, fixed_it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int n = cnt_t[u];
-        if (n == 0) continue;
+        const int bh = u / npairs, j0 = 2 * (u - bh * npairs);
+        if (unit_empty(bh, j0)) continue;
         if (!(ok = mbar_wait(fixed_full, fixed_it & 1, abort_flag, limit_ns))) break;
         ++fixed_it;
-        const int steps = (n + 1) >> 1;
-        for (int t = 0; t < steps; ++t, ++g) {
-          const uint32_t s = g & 1;
-          if (!(ok = mbar_wait(in_full + s, (g >> 1) & 1, abort_flag, limit_ns))) break;
-          if (g >= 2 && !(ok = mbar_wait(s_free + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
+        int n = -1;  // read from the first step's record
+        for (int t = 0; n < 0 || t < n; ++t, ++g) {
+          const uint32_t s = g % KS, b = g & 1;
+          if (!(ok = mbar_wait(in_full + s, (g / KS) & 1, abort_flag, limit_ns))) break;
+          if (n < 0) n = record(s)[2];
+          // buffer b is free once dV and dK of step g - 2 have read P^T / dS^T
+          if (g >= 2 && !(ok = mbar_wait(pd_empty + b, ((g >> 1) - 1) & 1, abort_flag, limit_ns))) break;
           tc_fence_after();
-          const uint32_t a_base = sbase + L::stage(s) + (is_s ? 0u : kStacked);
+          const uint32_t b_base = sbase + L::stage(s) + (is_s ? 0u : kFixed);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + s * 128 + col, kmajor_desc(a_base, kTile128, kk), kmajor_desc(fixed_base, kTile64, kk),
-                   idesc, kk > 0 ? 1u : 0u);
-          mma_commit(s_full + s);
+            mma_ss(tmem + b * 128 + col, kmajor_desc(a_base, kTile128, kk), kmajor_desc(b_base, kTile64, kk), idesc,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(s_full + b);
         }
-        if (ok) mma_commit(fixed_empty);
+        if (!ok) break;
+        mma_commit(fixed_empty);
       }
       mma_commit(drain);
     }
@@ -303,29 +362,33 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
     // ---------------------------------------- dV and dK issuers (one each)
     if (lane == 0) {
       const bool is_v = warp == 3;
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
-      const uint32_t acc = tmem + kAccCol0 + (is_v ? 0u : 64u);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t acc = tmem + kAccCol0 + (is_v ? 0u : 128u);
+      const uint32_t src = is_v ? 0u : 64u;  // P^T lives over S^T, dS^T over dP^T
       uint32_t g = 0, u_local = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
-        const int steps = (cnt_t[u] + 1) >> 1;
+        const int bh = u / npairs, j0 = 2 * (u - bh * npairs);
         // The epilogue of the previous unit must have read the accumulators
         // (and seen its acc_full phase) before this unit overwrites or signals.
         if (u_local > 0 && !(ok = mbar_wait(acc_empty, (u_local - 1) & 1, abort_flag, limit_ns))) break;
-        for (int t = 0; t < steps; ++t, ++g) {
-          const uint32_t pb = g & 1;
-          if (!(ok = mbar_wait(pd_full + pb, (g >> 1) & 1, abort_flag, limit_ns))) break;
+        int n = unit_empty(bh, j0) ? 0 : -1;
+        for (int t = 0; n < 0 || t < n; ++t, ++g) {
+          const uint32_t s = g % KS, b = g & 1;
+          if (!(ok = mbar_wait(pd_full + b, (g >> 1) & 1, abort_flag, limit_ns))) break;
+          if (n < 0) n = record(s)[2];
           tc_fence_after();
-          // A = the stacked dO (for dV) or Q (for dK) tile read MN-major: M = D
-          // in two 64-column atoms, K = the 128 stacked query rows.
-          const uint32_t a_base = sbase + L::stage(g & 1) + (is_v ? kStacked : 0u);
-          const uint32_t b_base = sbase + (is_v ? L::p(pb) : L::ds(pb));
+          // B = dO_i (for dV) or Q_i (for dK), MN-major: K = the 64 query
+          // rows, N = D in two 64-column atoms.  A = the 16 packed columns of
+          // each elementwise half: query steps kk = 0, 1 in the first half's,
+          // 2, 3 in the second's.
+          const uint32_t b_base = sbase + L::stage(s) + (is_v ? kFixed : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(acc, mnmajor_desc(a_base, kTile128, kk), mnmajor_desc(b_base, kTile128, kk), idesc,
-                   (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(pd_empty + pb);
-          mma_commit(in_empty + (g & 1));
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(acc, tmem + b * 128 + src + (kk >> 1) * 32 + (kk & 1) * 8,
+                   desc_sw128(b_base + kk * 16 * kRowBytes, kTile64, 1024), idesc, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(pd_empty + b);
+          mma_commit(in_empty + s);
         }
         if (!ok) break;
         mma_commit(acc_full);
@@ -333,65 +396,76 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       mma_commit(drain);
     }
   } else {
-    // ------------------------------------- elementwise (P, dS) + epilogue
-    const int half = (warp - 5) >> 2;   // which 32 of the 64 columns
+    // -------------------------------- elementwise (P^T, dS^T) + epilogue
+    const int half = (warp - 5) >> 2;   // which 32 of the 64 query columns
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // TMEM lane: query row of S / dP; column d of dV^T / dK^T
+    const int r = quarter * 32 + lane;  // TMEM lane = key row of the pair
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool upper = r >= 64;         // key block j1 (else j0); warp-uniform
     uint32_t g = 0, u_local = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_local) {
-      const int n = cnt_t[u];
-      const int bh = u / nb, j = u - bh * nb;
-      const int kv_lim = j == nb - 1 ? S - j * 64 : 64;
-      const int steps = (n + 1) >> 1;
-      for (int t = 0; t < steps; ++t, ++g) {
-        const uint32_t s = g & 1;
-        const bool w1 = mbar_wait(s_full + s, (g >> 1) & 1, abort_flag, limit_ns);
-        const bool w2 = w1 && mbar_wait(in_full + s, (g >> 1) & 1, abort_flag, limit_ns);
+      const int bh = u / npairs, j0 = 2 * (u - bh * npairs);
+      const int j = j0 + (upper ? 1 : 0);
+      const bool row_ok = j < nb && j * 64 + (r & 63) < S;
+      const int my_flag = upper ? 2 : 1;
+      int n = unit_empty(bh, j0) ? 0 : -1;
+      for (int t = 0; n < 0 || t < n; ++t, ++g) {
+        const uint32_t s = g % KS, b = g & 1;
+        const bool w1 = mbar_wait(s_full + b, (g >> 1) & 1, abort_flag, limit_ns);
+        const bool w2 = w1 && mbar_wait(in_full + s, (g / KS) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
         tc_fence_after();
+        const int* rec = record(s);
+        const int fl = rec[1];
+        if (n < 0) n = rec[2];
         uint32_t sr[32], dr[32];
-        tmem_ld32(lane_base + s * 128 + half * 32, sr);
-        tmem_ld32(lane_base + s * 128 + 64 + half * 32, dr);
+        tmem_ld32(lane_base + b * 128 + half * 32, sr);
+        tmem_ld32(lane_base + b * 128 + 64 + half * 32, dr);
         tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(s_free + s);  // the S / dP buffer may be overwritten now
-        const float* st = (const float*)(smem + L::stage(s) + 2 * kStacked);
-        const float lse2 = st[r], delta = st[128 + r];
-        const bool row_ok = r < 64 || 2 * t + 1 < n;
+        const float* stc = (const float*)(smem + L::stage(s) + L::stats) + half * 32;
+        const bool mine = row_ok && (fl & my_flag) != 0;
         uint32_t pw[16], dw[16];
-        p_ds_pairs(sr, dr, scale_log2, nullptr, nullptr, lse2, delta, half * 32, row_ok ? kv_lim : 0, pw, dw);
-        // P / dS of two steps back must have been consumed.
-        const bool w3 = g < 2 || mbar_wait(pd_empty + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns);
-        if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
-        store_half_row_sw128(smem + L::p(s), r, half, pw);
-        store_half_row_sw128(smem + L::ds(s), r, half, dw);
-        fence_proxy_async_smem();
-        mbar_arrive(pd_full + s);
+        p_ds_pairs(sr, dr, scale_log2, stc, stc + 64, 0.f, 0.f, 0, mine ? 32 : 0, pw, dw);
+        // into this warp's own S^T / dP^T columns, which it has read
+        tmem_st16(lane_base + b * 128 + half * 32, pw);
+        tmem_st16(lane_base + b * 128 + 64 + half * 32, dw);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(pd_full + b);
       }
       if (!ok) break;
-      // epilogue: thread r owns column d = r of dV^T (half 0) or dK^T (half 1)
+      // epilogue: thread r owns key row r of the pair; half 0 writes its dV
+      // row, half 1 its dK row (times 1 / sqrt(D))
       const bool w4 = mbar_wait(acc_full, u_local & 1, abort_flag, limit_ns);
       if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
       tc_fence_after();
-      const long long row0 = (long long)bh * S + (long long)j * 64;
       __nv_bfloat16* out = half == 0 ? dv : dk;
       const float mul = half == 0 ? 1.f : scale;
+      const long long orow = (long long)bh * S + (long long)j * 64 + (r & 63);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t a[32];
-        if (steps > 0) {
-          tmem_ld32(lane_base + kAccCol0 + half * 64 + h * 32, a);
+        if (n > 0) {
+          tmem_ld32(lane_base + kAccCol0 + half * 128 + c0, a);
           tmem_ld_wait();
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) a[c] = 0u;
         }
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(out + orow * D + c0);
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (h * 32 + c < kv_lim)
-            out[(row0 + h * 32 + c) * D + r] = __float2bfloat16_rn(__uint_as_float(a[c]) * mul);
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * v4 + 2 * e;
+              w[e] = pack_bf16x2(__uint_as_float(a[c]) * mul, __uint_as_float(a[c + 1]) * mul);
+            }
+            dst[v4] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
@@ -721,9 +795,9 @@ __global__ void __launch_bounds__(256) bwd_stats_kernel(const __nv_bfloat16* __r
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, const float* lse, const int32_t* cnt, const int32_t* idx,
-                               const int32_t* cnt_t, const int32_t* idx_t, float* lse2p, float* deltap,
-                               void* dq, void* dk, void* dv, int32_t* ws_header, cudaStream_t st) {
+                               const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
+                               const int32_t* idx, const int32_t* cnt_t, float* lse2p, float* deltap, void* dq,
+                               void* dk, void* dv, int32_t* ws_header, cudaStream_t st) {
   if (d.dtype != NABLA_BF16 || d.D != 128) return cudaErrorInvalidValue;
   const long long rows = d.BH() * d.nb * 64;
   bwd_stats_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
@@ -735,14 +809,15 @@ cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, cons
       !make_map_bf16(&tdo, dout, d, 64))
     return cudaErrorInvalidValue;
   const int n_units = (int)(d.BH() * d.nb);
+  const int n_pairs = (int)(d.BH() * d.npairs);
   const int grid = std::min(n_units, sm_count());
   const float scale = 1.0f / sqrtf(128.0f), scale_log2 = 1.4426950408889634f * scale;
   auto k1 = dkdv_tc_kernel<128>;
   e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DkdvSmem::bytes);
   if (e != cudaSuccess) return e;
-  k1<<<grid, kDkdvThreads, DkdvSmem::bytes, st>>>(tq, tk, tv, tdo, lse2p, deltap, cnt_t, idx_t, n_units, d.S, d.nb,
-                                          scale, scale_log2, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv,
-                                          ws_header + kWsStatus, wait_limit_ns());
+  k1<<<std::min(n_pairs, sm_count()), kDkdvThreads, DkdvSmem::bytes, st>>>(
+      tq, tk, tv, tdo, lse2p, deltap, bits, cnt_t, n_pairs, d.npairs, d.S, d.nb, d.W, scale, scale_log2,
+      (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, ws_header + kWsStatus, wait_limit_ns());
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto k2 = dq_tc_kernel<128>;

@@ -120,9 +120,9 @@ cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, cons
 
 // bf16, D = 128 only.  lse2p / deltap: workspace [B*H][nb*64] fp32 each.
 cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, const float* lse, const int32_t* cnt, const int32_t* idx,
-                               const int32_t* cnt_t, const int32_t* idx_t, float* lse2p, float* deltap,
-                               void* dq, void* dk, void* dv, int32_t* ws_header, cudaStream_t st);
+                               const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
+                               const int32_t* idx, const int32_t* cnt_t, float* lse2p, float* deltap, void* dq,
+                               void* dk, void* dv, int32_t* ws_header, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 

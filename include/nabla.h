@@ -205,8 +205,10 @@ NABLA_API nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, c
 
 /* Backward of nabla_attn_fwd with the mask held constant (no gradient flows
  * into the mask builder).  o and lse are the forward's outputs, dout the
- * upstream gradient; mask needs cnt, idx, cnt_t and idx_t.  Writes dq, dk, dv
- * [B, H, S, D] in shape->dtype.  The result is deterministic (no atomics). */
+ * upstream gradient; mask needs bits, cnt, idx, cnt_t and idx_t, all of the
+ * same mask (the bf16 path walks cnt / idx for dQ and bits / cnt_t for dK and
+ * dV; the fp32 path the four lists).  Writes dq, dk, dv [B, H, S, D] in
+ * shape->dtype.  The result is deterministic (no atomics). */
 NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                             const void* o, const void* dout, const float* lse,
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
