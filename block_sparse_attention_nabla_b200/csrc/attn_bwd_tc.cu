@@ -145,23 +145,36 @@ __device__ __forceinline__ void store_half_row_sw128(uint8_t* tile, int row, int
         make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 
-// P and dS of 32 columns of one row: s, dp raw accumulator words; lse2 and
-// delta per column (arrays) or per row (scalars broadcast by the caller).
-__device__ __forceinline__ void p_ds_pairs(const uint32_t (&sr)[32], const uint32_t (&dr)[32], float scale_log2,
-                                           const float* lse2c, const float* deltac, float lse2r, float deltar,
-                                           int col0, int col_lim, uint32_t* pw, uint32_t* dw) {
+// P and dS of 32 columns of one row: s, dp raw accumulator words; lse2c and
+// deltac the 1/ln2-scaled LSE and the Delta of the 32 columns (16-byte
+// aligned shared memory, read four at a time).  keep == false (a row outside
+// the mask or the sequence) gives P = dS = 0 without evaluating anything.
+__device__ __forceinline__ void p_ds_cols(const uint32_t (&sr)[32], const uint32_t (&dr)[32], float scale_log2,
+                                          const float* lse2c, const float* deltac, bool keep, uint32_t* pw,
+                                          uint32_t* dw) {
+  if (!keep) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const int c0 = 2 * c, c1 = 2 * c + 1;
-    const float l0 = lse2c ? lse2c[c0] : lse2r, l1 = lse2c ? lse2c[c1] : lse2r;
-    const float e0 = deltac ? deltac[c0] : deltar, e1 = deltac ? deltac[c1] : deltar;
-    float p0 = ex2(fmaf(__uint_as_float(sr[c0]), scale_log2, -l0));
-    float p1 = ex2(fmaf(__uint_as_float(sr[c1]), scale_log2, -l1));
-    if (col0 + c0 >= col_lim) p0 = 0.f;
-    if (col0 + c1 >= col_lim) p1 = 0.f;
-    const float d0 = p0 * (__uint_as_float(dr[c0]) - e0), d1 = p1 * (__uint_as_float(dr[c1]) - e1);
-    if (pw) pw[c] = pack_bf16x2(p0, p1);
-    dw[c] = pack_bf16x2(d0, d1);
+    for (int c = 0; c < 16; ++c) {
+      if (pw) pw[c] = 0u;
+      dw[c] = 0u;
+    }
+    return;
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 l4 = reinterpret_cast<const float4*>(lse2c)[q];
+    const float4 e4 = reinterpret_cast<const float4*>(deltac)[q];
+    const float l[4] = {l4.x, l4.y, l4.z, l4.w}, e[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c0 = 4 * q + 2 * h, c1 = c0 + 1;
+      const float p0 = ex2(fmaf(__uint_as_float(sr[c0]), scale_log2, -l[2 * h]));
+      const float p1 = ex2(fmaf(__uint_as_float(sr[c1]), scale_log2, -l[2 * h + 1]));
+      const float d0 = p0 * (__uint_as_float(dr[c0]) - e[2 * h]);
+      const float d1 = p1 * (__uint_as_float(dr[c1]) - e[2 * h + 1]);
+      if (pw) pw[2 * q + h] = pack_bf16x2(p0, p1);
+      dw[2 * q + h] = pack_bf16x2(d0, d1);
+    }
   }
 }
 
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
         const float* stc = (const float*)(smem + L::stage(s) + L::stats) + half * 32;
         const bool mine = row_ok && (fl & my_flag) != 0;
         uint32_t pw[16], dw[16];
-        p_ds_pairs(sr, dr, scale_log2, stc, stc + 64, 0.f, 0.f, 0, mine ? 32 : 0, pw, dw);
+        p_ds_cols(sr, dr, scale_log2, stc, stc + 64, mine, pw, dw);
         // into this warp's own S^T / dP^T columns, which it has read
         tmem_st16(lane_base + b * 128 + half * 32, pw);
         tmem_st16(lane_base + b * 128 + 64 + half * 32, dw);
@@ -714,7 +727,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const int pos = 2 * t + (r >= 64 ? 1 : 0);  // list position of this row's key block
         const bool row_ok = pos < n && !(ends_in_tail && pos == n - 1 && (r & 63) >= tail_keys);
         uint32_t dw[16];
-        p_ds_pairs(sr, dr, scale_log2, lse2c, deltac, 0.f, 0.f, 0, row_ok ? 32 : 0, nullptr, dw);
+        p_ds_cols(sr, dr, scale_log2, lse2c, deltac, row_ok, nullptr, dw);
         const bool w3 = g < 2 || mbar_wait(pd_empty + s, ((g >> 1) - 1) & 1, abort_flag, limit_ns);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
         store_half_row_sw128(smem + L::ds(s), r, half, dw);
