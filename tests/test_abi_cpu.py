@@ -122,6 +122,9 @@ def test_attention_argument_errors(L):
     full = mask_struct(cnt_t=FAKE, idx_t=FAKE)
     assert bwd(m=full, dv=None) == INVALID
     assert bwd(m=full, wsb=1000) == WORKSPACE
+    # the tensor-core dK / dV walks the bitmask columns: bits are required
+    assert bwd(m=mask_struct(cnt_t=FAKE, idx_t=FAKE, bits=None)) == INVALID
+    assert b"bits" in L.nabla_last_error()
 
 
 def test_mask_from_bits_and_status_argument_errors(L):
