@@ -1,0 +1,302 @@
+"""Random-interleaving models of two mbarrier protocols of the tensor-core
+kernels (host only; no GPU code runs).
+
+Every role of a kernel is a Python generator that yields the waits and
+arrivals it performs; the scheduler runs any runnable role (or completes any
+outstanding asynchronous operation) at random.  A run fails on
+
+* a deadlock (nothing runnable, roles unfinished);
+* a parity alias: mbarrier waits test the parity of a phase, so a waiter for
+  phase k must proceed while the barrier has completed exactly k + 1 phases;
+  a barrier two phases ahead would make the wait hang on the hardware;
+* a broken hand-off: a buffer overwritten while a reader still needs it, or
+  read before its producer wrote it.
+
+Models:
+
+* ``unit_ring`` -- attn_fwd_tc.cu: the producer warp draws unit ids from a
+  counter shared by all CTAs and hands each to three consumer roles through a
+  ring of R slots (full / empty barriers); -1 ends every role.
+* ``dkdv_pair`` -- attn_bwd_tc.cu, dkdv_tc_kernel: producer (the unit's fixed
+  K / V pair, one stage per step with its record), the S^T and dP^T issuers,
+  the dV and dK issuers (tcgen05 commits arrive once the issuing thread's
+  earlier MMAs are done, so each issuer is an in-order engine), the
+  elementwise group and its epilogue, TMA copies landing at any time.
+
+``mutation`` plants one mistake in the protocol (not in a kernel); the tests
+require each to be caught.
+"""
+from __future__ import annotations
+
+import random
+
+
+class ProtocolError(Exception):
+    pass
+
+
+class _Bar:
+    def __init__(self, count: int):
+        self.count, self.arrived, self.done = count, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        if self.arrived == self.count:
+            self.arrived = 0
+            self.done += 1
+
+
+def _run(roles: dict, bars: dict, engines: dict, execute, rnd: random.Random):
+    """Interleave `roles` (generators of ("wait", bar, phase) / ("arrive", bar))
+    and the asynchronous `engines` (queues of operations run by `execute`)."""
+    pending = {r: None for r in roles}
+    done = set()
+    while True:
+        runnable = []
+        for r, gen in roles.items():
+            if r in done:
+                continue
+            if pending[r] is None:
+                try:
+                    pending[r] = next(gen)
+                except StopIteration:
+                    done.add(r)
+                    continue
+            op = pending[r]
+            if op[0] == "arrive":
+                runnable.append(("role", r))
+            else:
+                bar = bars[op[1]]
+                if bar.done > op[2] + 1:
+                    raise ProtocolError(f"parity alias: {r} waits {op[1]} phase {op[2]}, done {bar.done}")
+                if bar.done > op[2]:
+                    runnable.append(("role", r))
+        runnable += [("engine", e) for e, q in engines.items() if q]
+        if not runnable:
+            if len(done) == len(roles):
+                return
+            raise ProtocolError(f"deadlock: {[pending[r] for r in roles if r not in done]}")
+        kind, x = rnd.choice(runnable)
+        if kind == "engine":
+            execute(x, engines[x].pop(0))
+        else:
+            op = pending[x]
+            pending[x] = None
+            if op[0] == "arrive":
+                bars[op[1]].arrive()
+
+
+def unit_ring(n_units: int, n_cta: int, seed: int, R: int = 4, mutation: str | None = None) -> None:
+    rnd = random.Random(seed)
+    counter = [0]
+    roles, bars, logs = {}, {}, []
+    consumers = ("v_producer", "mma", "softmax")
+    for c in range(n_cta):
+        for s in range(R):
+            bars[(c, "full", s)] = _Bar(1)
+            bars[(c, "empty", s)] = _Bar(len(consumers) - (1 if mutation == "empty_count" else 0))
+        slots = [None] * R
+        log = {r: [] for r in ("producer",) + consumers}
+        logs.append(log)
+
+        def producer(c=c, slots=slots, log=log):
+            k = 0
+            while True:
+                s = k % R
+                if k >= R and mutation != "no_empty_wait":
+                    yield ("wait", (c, "empty", s), k // R - 1)
+                u = counter[0]
+                counter[0] += 1
+                slots[s] = u if u < n_units else -1
+                log["producer"].append(slots[s])
+                yield ("arrive", (c, "full", s))
+                if u >= n_units:
+                    return
+                k += 1
+
+        def consumer(name, c=c, slots=slots, log=log):
+            k = 0
+            while True:
+                s = k % R
+                yield ("wait", (c, "full", s), k // R)
+                u = slots[s]
+                log[name].append(u)
+                yield ("arrive", (c, "empty", s))
+                if u < 0:
+                    return
+                k += 1
+
+        roles[(c, "producer")] = producer()
+        for name in consumers:
+            roles[(c, name)] = consumer(name)
+    _run(roles, bars, {}, None, rnd)
+    drawn = []
+    for log in logs:
+        for name in consumers:
+            if log[name] != log["producer"]:
+                raise ProtocolError(f"{name} saw {log[name]}, producer handed {log['producer']}")
+        drawn += [u for u in log["producer"] if u >= 0]
+    if sorted(drawn) != list(range(n_units)):
+        raise ProtocolError("units lost or drawn twice")
+
+
+def dkdv_pair(units: list, seed: int, KS: int = 4, mutation: str | None = None) -> None:
+    """units: the number of steps of each unit this CTA runs (0 = no query
+    block kept either key block)."""
+    rnd = random.Random(seed)
+    bars = {"fixed_full": _Bar(1), "fixed_empty": _Bar(2), "acc_full": _Bar(2), "acc_empty": _Bar(1),
+            "drain": _Bar(4)}
+    for s in range(KS):
+        bars[f"in_full{s}"] = _Bar(1)
+        bars[f"in_empty{s}"] = _Bar(2)
+    for b in range(2):
+        bars[f"s_full{b}"] = _Bar(2)
+        bars[f"pd_full{b}"] = _Bar(1)
+        bars[f"pd_empty{b}"] = _Bar(1 if mutation == "pd_empty_count" else 2)
+    st = {"stage": [None] * KS, "stage_readers": [set() for _ in range(KS)], "record": [None] * KS,
+          "buf": [dict(S=None, dP=None, P=None, readers=set()) for _ in range(2)],
+          "kv": None, "kv_readers": set(), "acc": {"dV": None, "dK": None}, "epilogue_done": -1}
+    engines = {e: [] for e in ("S", "dP", "dV", "dK", "tma")}
+
+    def producer():
+        g = fixed = 0
+        for u, n in enumerate(units):
+            if n == 0:
+                continue
+            if fixed > 0:
+                yield ("wait", "fixed_empty", fixed - 1)
+            engines["tma"].append(("kv", u))
+            fixed += 1
+            for t in range(n):
+                s, use = g % KS, g // KS
+                if use > 0:
+                    yield ("wait", f"in_empty{s}", use - 1)
+                if st["stage_readers"][s]:
+                    raise ProtocolError(f"record of step {g} written while {st['stage_readers'][s]} read stage {s}")
+                st["record"][s] = (u, t, n, g)
+                engines["tma"].append(("stage", g, s))
+                g += 1
+
+    def s_issuer(name):
+        g = fixed = 0
+        for u, n in enumerate(units):
+            if n == 0:
+                continue
+            yield ("wait", "fixed_full", fixed)
+            fixed += 1
+            steps, t = -1, 0
+            while steps < 0 or t < steps:
+                s, b = g % KS, g & 1
+                yield ("wait", f"in_full{s}", g // KS)
+                rec = st["record"][s]
+                if rec[3] != g:
+                    raise ProtocolError(f"{name} read the record of step {rec[3]} at step {g}")
+                steps = rec[2] if steps < 0 else steps
+                if g >= 2 and mutation != "no_buffer_wait":
+                    yield ("wait", f"pd_empty{b}", (g >> 1) - 1)
+                st["stage_readers"][s].add((name, g))
+                st["kv_readers"].add((name, u))
+                engines[name].append(("mma", g, s, b, u))
+                engines[name].append(("commit", f"s_full{b}"))
+                t += 1
+                g += 1
+            engines[name].append(("commit", "fixed_empty"))
+        engines[name].append(("commit", "drain"))
+
+    def acc_issuer(name):
+        g = 0
+        for u, n in enumerate(units):
+            if u > 0 and mutation != "no_acc_wait":
+                yield ("wait", "acc_empty", u - 1)
+            steps, t = (0 if n == 0 else -1), 0
+            while steps < 0 or t < steps:
+                s, b = g % KS, g & 1
+                yield ("wait", f"pd_full{b}", g >> 1)
+                rec = st["record"][s]
+                if rec[3] != g:
+                    raise ProtocolError(f"{name} read the record of step {rec[3]} at step {g}")
+                steps = rec[2] if steps < 0 else steps
+                st["stage_readers"][s].add((name, g))
+                st["buf"][b]["readers"].add((name, g))
+                engines[name].append(("mma", g, s, b, u, t))
+                engines[name].append(("commit", f"pd_empty{b}"))
+                if mutation != "no_stage_release":
+                    engines[name].append(("commit", f"in_empty{s}"))
+                t += 1
+                g += 1
+            engines[name].append(("commit", "acc_full"))
+        engines[name].append(("commit", "drain"))
+
+    def elementwise():
+        g = 0
+        for u, n in enumerate(units):
+            steps, t = (0 if n == 0 else -1), 0
+            while steps < 0 or t < steps:
+                s, b = g % KS, g & 1
+                yield ("wait", f"s_full{b}", g >> 1)
+                yield ("wait", f"in_full{s}", g // KS)
+                rec = st["record"][s]
+                if rec[3] != g:
+                    raise ProtocolError(f"elementwise read the record of step {rec[3]} at step {g}")
+                steps = rec[2] if steps < 0 else steps
+                buf = st["buf"][b]
+                if buf["S"] != g or buf["dP"] != g:
+                    raise ProtocolError(f"elementwise read S {buf['S']} / dP {buf['dP']} at step {g}")
+                if st["stage"][s] != g:
+                    raise ProtocolError(f"elementwise read stats of step {st['stage'][s]} at step {g}")
+                buf["P"] = g
+                yield ("arrive", f"pd_full{b}")
+                t += 1
+                g += 1
+            yield ("wait", "acc_full", u)
+            want = (u, steps - 1) if steps > 0 else None
+            if steps > 0 and (st["acc"]["dV"] != want or st["acc"]["dK"] != want):
+                raise ProtocolError(f"epilogue of unit {u} read accumulators {st['acc']}")
+            st["epilogue_done"] = u
+            yield ("arrive", "acc_empty")
+
+    def execute(e, op):
+        if op[0] == "commit":
+            bars[op[1]].arrive()
+            return
+        if e == "tma":
+            if op[0] == "kv":
+                live = [x for x in st["kv_readers"] if x[1] != op[1]]
+                if live:
+                    raise ProtocolError(f"K / V pair overwritten while {live} read it")
+                st["kv"] = op[1]
+                bars["fixed_full"].arrive()
+            else:
+                _, g, s = op
+                live = [x for x in st["stage_readers"][s] if x[1] != g]
+                if live:
+                    raise ProtocolError(f"stage {s} overwritten for step {g} while {live} read it")
+                st["stage"][s] = g
+                bars[f"in_full{s}"].arrive()
+            return
+        if e in ("S", "dP"):
+            _, g, s, b, u = op
+            buf = st["buf"][b]
+            if st["stage"][s] != g or st["kv"] != u:
+                raise ProtocolError(f"{e} of step {g} read stage {st['stage'][s]} / K-V {st['kv']}")
+            if g >= 2 and (any(x[1] == g - 2 for x in buf["readers"]) or buf["P"] != g - 2):
+                raise ProtocolError(f"{e} of step {g} overwrote buffer {b} before step {g - 2} was done with it")
+            buf[e] = g
+            st["stage_readers"][s].discard((e, g))
+            st["kv_readers"].discard((e, u))
+            return
+        _, g, s, b, u, t = op
+        buf = st["buf"][b]
+        if buf["P"] != g or st["stage"][s] != g:
+            raise ProtocolError(f"{e} of step {g} read P of {buf['P']} / stage {st['stage'][s]}")
+        if t == 0 and st["epilogue_done"] < u - 1:
+            raise ProtocolError(f"{e} overwrote the accumulator before the epilogue of unit {u - 1}")
+        st["acc"][e] = (u, t)
+        buf["readers"].discard((e, g))
+        st["stage_readers"][s].discard((e, g))
+
+    roles = {"producer": producer(), "S": s_issuer("S"), "dP": s_issuer("dP"), "dV": acc_issuer("dV"),
+             "dK": acc_issuer("dK"), "elementwise": elementwise()}
+    _run(roles, bars, engines, execute, rnd)
+    if bars["drain"].done != 1:
+        raise ProtocolError("teardown barrier did not complete")

@@ -1,0 +1,50 @@
+"""The barrier protocols of the forward's unit ring and of the dK / dV
+pipeline, checked in random-interleaving models (host only).  Each planted
+mistake must be caught within the sampled traces."""
+import random
+
+import pytest
+
+from tests import protocol_models as pm
+
+
+def _dkdv_traces(n, KS, mutation=None):
+    rng = random.Random(7)
+    failures = 0
+    for seed in range(n):
+        units = [rng.choice([0, 0, 1, 2, 3, 5, 8]) for _ in range(rng.randint(1, 6))]
+        try:
+            pm.dkdv_pair(units, seed, KS=KS, mutation=mutation)
+        except pm.ProtocolError:
+            failures += 1
+    return failures
+
+
+@pytest.mark.parametrize("KS", [2, 3, 4])
+def test_dkdv_pair_protocol_holds(KS):
+    assert _dkdv_traces(400, KS) == 0
+
+
+@pytest.mark.parametrize("mutation", ["pd_empty_count", "no_buffer_wait", "no_stage_release", "no_acc_wait"])
+def test_dkdv_pair_protocol_mutants_are_caught(mutation):
+    assert _dkdv_traces(200, 4, mutation) > 0
+
+
+def _ring_traces(n, mutation=None):
+    rng = random.Random(2)
+    failures = 0
+    for seed in range(n):
+        try:
+            pm.unit_ring(rng.randint(0, 30), rng.randint(1, 4), seed, mutation=mutation)
+        except pm.ProtocolError:
+            failures += 1
+    return failures
+
+
+def test_unit_ring_protocol_holds():
+    assert _ring_traces(1500) == 0
+
+
+@pytest.mark.parametrize("mutation", ["empty_count", "no_empty_wait"])
+def test_unit_ring_mutants_are_caught(mutation):
+    assert _ring_traces(400, mutation) > 0
