@@ -340,7 +340,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (t >= 1) ok = issue_pv(g - 1);
         }
         if (ok && n >= 1) ok = issue_pv(g_iter + n - 1);
-        if (ok) mma_commit(b.o_final);
+        // only a unit with tiles signals its O: for one without, the issuer
+        // runs ahead of the softmax threads, and two such signals in a row
+        // could put o_final two phases past a waiter
+        if (ok && n >= 1) mma_commit(b.o_final);
         mma_commit(b.q_empty);
         g_iter += n;
       }
@@ -351,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int row = quarter * 32 + lane;  // row of the 128-row tile == TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int my_flag = row < 64 ? 1 : 2;
-    uint32_t g_iter = 0, u_local = 0;
+    uint32_t g_iter = 0, finals = 0;  // finals: units with tiles, i.e. o_final phases
     bool ok = true;
     uint32_t ku = 0;
     while (ok) {
@@ -461,11 +464,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_arrive(b.p_full + sb);
       }
       if (!ok) break;
-      // epilogue: o_final completes once per unit, after its last P V (at
-      // once for a unit without tiles)
-      const bool w4 = mbar_wait(b.o_final, u_local & 1, abort_flag, limit_ns);
-      if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
-      tc_fence_after();
+      // epilogue: o_final completes once per unit with tiles, after its
+      // last P V; a unit without tiles writes O = 0 and LSE = -inf at once
+      if (n >= 1) {
+        const bool w4 = mbar_wait(b.o_final, finals & 1, abort_flag, limit_ns);
+        if (!__all_sync(0xffffffffu, w4)) { ok = false; break; }
+        ++finals;
+        tc_fence_after();
+      }
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool valid = qrow < S;
       __nv_bfloat16* orow = out + ((long long)bh * S + qrow) * D;
@@ -493,7 +499,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (valid && lse) lse[(long long)bh * S + qrow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
       g_iter += n;
-      ++u_local;
     }
   }
 

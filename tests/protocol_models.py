@@ -1,4 +1,4 @@
-"""Random-interleaving models of two mbarrier protocols of the tensor-core
+"""Random-interleaving models of the mbarrier protocols of the tensor-core
 kernels (host only; no GPU code runs).
 
 Every role of a kernel is a Python generator that yields the waits and
@@ -22,6 +22,12 @@ Models:
   the dV and dK issuers (tcgen05 commits arrive once the issuing thread's
   earlier MMAs are done, so each issuer is an in-order engine), the
   elementwise group and its epilogue, TMA copies landing at any time.
+
+* ``fwd_pipeline`` -- attn_fwd_tc.cu after the unit ring: Q / K producer, V
+  producer, the MMA issuer, the softmax group with its O rescale and
+  epilogue.  Units without tiles do not signal O (mutation
+  "o_final_for_empty_units" restores the earlier protocol, in which two such
+  units in a row could leave o_final two phases past its waiter).
 
 ``mutation`` plants one mistake in the protocol (not in a kernel); the tests
 require each to be caught.
@@ -300,3 +306,153 @@ def dkdv_pair(units: list, seed: int, KS: int = 4, mutation: str | None = None) 
     _run(roles, bars, engines, execute, rnd)
     if bars["drain"].done != 1:
         raise ProtocolError("teardown barrier did not complete")
+
+
+def fwd_pipeline(units: list, seed: int, KS: int = 3, VS: int = 2, mutation: str | None = None) -> None:
+    """attn_fwd_tc.cu, one CTA after the unit ring: the Q / K producer, the V
+    producer, the single MMA issuer (S of tile g into TMEM buffer g & 1, then
+    P V of tile g - 1; its MMAs and commits complete in issue order), the
+    softmax group (P over S, a rescale of O that waits for P V of tile g - 1,
+    the epilogue) and TMA copies landing at any time.  units: tiles per unit."""
+    rnd = random.Random(seed)
+    bars = {"q_full": _Bar(1), "q_empty": _Bar(1), "o_done": _Bar(1), "o_final": _Bar(1)}
+    for s in range(KS):
+        bars[f"k_full{s}"] = _Bar(1)
+        bars[f"k_empty{s}"] = _Bar(1)
+    for s in range(VS):
+        bars[f"v_full{s}"] = _Bar(1)
+        bars[f"v_empty{s}"] = _Bar(1)
+    for b in range(2):
+        bars[f"s_full{b}"] = _Bar(1)
+        bars[f"p_full{b}"] = _Bar(1)
+    st = {"q": None, "q_readers": set(), "k": [None] * KS, "k_readers": [set() for _ in range(KS)],
+          "v": [None] * VS, "v_readers": [set() for _ in range(VS)],
+          "buf": [dict(S=None, P=None) for _ in range(2)], "pv_done": -1, "o_unit": None,
+          "epilogue_done": -1}
+    first = []  # global index of each unit's first tile
+    g = 0
+    for n in units:
+        first.append(g)
+        g += n
+    engines = {"mma": [], "tma": []}
+
+    def qk_producer():
+        g = q_it = 0
+        for u, n in enumerate(units):
+            if q_it > 0 and mutation != "no_q_wait":
+                yield ("wait", "q_empty", q_it - 1)
+            engines["tma"].append(("q", u))
+            q_it += 1
+            for _ in range(n):
+                s, use = g % KS, g // KS
+                if use > 0:
+                    yield ("wait", f"k_empty{s}", use - 1)
+                engines["tma"].append(("k", g, s))
+                g += 1
+
+    def v_producer():
+        g = 0
+        for n in units:
+            for _ in range(n):
+                s, use = g % VS, g // VS
+                if use > 0 and mutation != "no_v_wait":
+                    yield ("wait", f"v_empty{s}", use - 1)
+                engines["tma"].append(("v", g, s))
+                g += 1
+
+    def mma():
+        g = 0
+        for u, n in enumerate(units):
+            yield ("wait", "q_full", u)
+            for t in range(n):
+                s = g % KS
+                if mutation != "no_k_wait":
+                    yield ("wait", f"k_full{s}", g // KS)
+                st["q_readers"].add(("S", g))
+                st["k_readers"][s].add(g)
+                engines["mma"].append(("S", g, u))
+                engines["mma"].append(("commit", f"k_empty{s}"))
+                engines["mma"].append(("commit", f"s_full{g & 1}"))
+                if t >= 1:
+                    yield from _pv(g - 1, u)
+                g += 1
+            if n >= 1:
+                yield from _pv(g - 1, u)
+                engines["mma"].append(("commit", "o_final"))  # only units with tiles signal O
+            elif mutation == "o_final_for_empty_units":
+                engines["mma"].append(("commit", "o_final"))
+            engines["mma"].append(("commit", "q_empty"))
+
+    def _pv(h, u):
+        yield ("wait", f"p_full{h & 1}", h >> 1)
+        yield ("wait", f"v_full{h % VS}", h // VS)
+        st["v_readers"][h % VS].add(h)
+        engines["mma"].append(("PV", h, u))
+        engines["mma"].append(("commit", f"v_empty{h % VS}"))
+        engines["mma"].append(("commit", "o_done"))
+
+    def softmax():
+        g = finals = 0  # finals: o_final phases waited for (units with tiles)
+        for u, n in enumerate(units):
+            for t in range(n):
+                b = g & 1
+                yield ("wait", f"s_full{b}", g >> 1)
+                if st["buf"][b]["S"] != g:
+                    raise ProtocolError(f"softmax read S of tile {st['buf'][b]['S']} at tile {g}")
+                if t >= 1 and rnd.random() < 0.3:  # the running max grew: rescale O
+                    lag = 2 if mutation == "rescale_lag" else 1
+                    yield ("wait", "o_done", g - lag)
+                    if st["pv_done"] != g - 1:
+                        raise ProtocolError(f"O rescaled at tile {g} with P V done up to {st['pv_done']}")
+                st["buf"][b]["P"] = g
+                yield ("arrive", f"p_full{b}")
+                g += 1
+            if n > 0 or mutation == "o_final_for_empty_units":
+                yield ("wait", "o_final", finals)
+                finals += 1
+            if n > 0 and st["pv_done"] != first[u] + n - 1:
+                raise ProtocolError(f"epilogue of unit {u} read O with P V done up to {st['pv_done']}")
+            st["epilogue_done"] = u
+
+    def execute(e, op):
+        if op[0] == "commit":
+            bars[op[1]].arrive()
+            return
+        if op[0] == "q":
+            if st["q_readers"]:
+                raise ProtocolError(f"Q of unit {op[1]} landed while {st['q_readers']} read the previous one")
+            st["q"] = op[1]
+            bars["q_full"].arrive()
+        elif op[0] == "k":
+            _, g, s = op
+            if st["k_readers"][s]:
+                raise ProtocolError(f"K slot {s} refilled for tile {g} while tiles {st['k_readers'][s]} read it")
+            st["k"][s] = g
+            bars[f"k_full{s}"].arrive()
+        elif op[0] == "v":
+            _, g, s = op
+            if st["v_readers"][s]:
+                raise ProtocolError(f"V slot {s} refilled for tile {g} while tiles {st['v_readers'][s]} read it")
+            st["v"][s] = g
+            bars[f"v_full{s}"].arrive()
+        elif op[0] == "S":
+            _, g, u = op
+            buf = st["buf"][g & 1]
+            if st["q"] != u or st["k"][g % KS] != g:
+                raise ProtocolError(f"S of tile {g} read Q of unit {st['q']} / K of tile {st['k'][g % KS]}")
+            if g >= 2 and (buf["P"] != g - 2 or st["pv_done"] < g - 2):
+                raise ProtocolError(f"S of tile {g} overwrote buffer {g & 1} before P V of tile {g - 2}")
+            buf["S"] = g
+            st["q_readers"].discard(("S", g))
+            st["k_readers"][g % KS].discard(g)
+        else:
+            _, h, u = op
+            if st["buf"][h & 1]["P"] != h or st["v"][h % VS] != h:
+                raise ProtocolError(f"P V of tile {h} read P of {st['buf'][h & 1]['P']} / V of {st['v'][h % VS]}")
+            if h == first[u] and st["epilogue_done"] < u - 1:
+                raise ProtocolError(f"P V of tile {h} overwrote O before the epilogue of unit {u - 1}")
+            st["pv_done"] = h
+            st["v_readers"][h % VS].discard(h)
+
+    roles = {"qk_producer": qk_producer(), "v_producer": v_producer(), "mma": mma(), "softmax": softmax()}
+    _run(roles, bars, engines, execute, rnd)

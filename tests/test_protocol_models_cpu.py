@@ -48,3 +48,24 @@ def test_unit_ring_protocol_holds():
 @pytest.mark.parametrize("mutation", ["empty_count", "no_empty_wait"])
 def test_unit_ring_mutants_are_caught(mutation):
     assert _ring_traces(400, mutation) > 0
+
+
+def _fwd_traces(n, mutation=None):
+    rng = random.Random(11)
+    failures = 0
+    for seed in range(n):
+        units = [rng.choice([0, 1, 1, 2, 3, 5, 9]) for _ in range(rng.randint(1, 6))]
+        try:
+            pm.fwd_pipeline(units, seed, mutation=mutation)
+        except pm.ProtocolError:
+            failures += 1
+    return failures
+
+
+def test_forward_pipeline_protocol_holds():
+    assert _fwd_traces(600) == 0
+
+
+@pytest.mark.parametrize("mutation", ["no_q_wait", "no_v_wait", "no_k_wait", "rescale_lag", "o_final_for_empty_units"])
+def test_forward_pipeline_mutants_are_caught(mutation):
+    assert _fwd_traces(300, mutation) > 0
