@@ -38,10 +38,9 @@ THR = 0.8
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # one ncu capture, keyed by the SHA-256 of the kernel source it was taken on;
-# reported only while the source is unchanged.  Filled from the summaries
-# under profiles/.
+# reported only while the source is unchanged.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_tc_720p_h4.md: 304.9 MB at 4 heads, scaled x10 to 40 heads
+    # 4-head capture of the 720p shape at thr 0.8: 304.9 MB, scaled x10 to 40 heads
     "attn_fwd_tc.cu": ("88c3d65e11d641849bfd132cdf6c2d53eb8eb451264329b32b75d248b9a050ee", 3.049e9),
 }
 
@@ -144,7 +143,7 @@ def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def cpu_baseline(x: dict, thr: float, budget_s: float = 12.0) -> dict:
+def cpu_baseline(x: dict, thr: float, budget_s: float = 12.0, heads_total: int | None = None) -> dict:
     """The fp64 oracle, as it stands, on a bounded sample of the workload: the
     full mask of one head, then masked attention for as many query blocks of
     that head as fit in the time budget.  Value in the metric's unit (TFLOP/s on
@@ -177,7 +176,12 @@ def cpu_baseline(x: dict, thr: float, budget_s: float = 12.0) -> dict:
         step = min(step * 2, 64)
     flops = done_tiles * 4 * 64 * 64 * D
     mask_bytes = q.numel() * q.element_size() * 2
+    heads = heads_total or x["q"].shape[0] * x["q"].shape[1]
+    full_s = heads * (t_mask + spent / nblk * nb)
     return {"value": flops / spent / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "full_config_extrapolated_s": full_s,
+            "full_config_note": "one head's mask time plus its attention time per query block, scaled "
+                                "linearly to every query block and head of the problem",
             "sample": f"head 0 of {tuple(x['q'].shape)}: full fp64 mask ({t_mask:.2f} s, "
                       f"{mask_bytes / t_mask / 1e9:.3f} GB/s of Q+K), masked attention for {nblk} of {nb} "
                       f"query blocks ({done_tiles} kept tiles, {spent:.2f} s)",
@@ -197,7 +201,7 @@ def run_reference(args) -> None:
     vals = []
     t_all = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(cpu_baseline(x, THR, budget_s=budget))
+        vals.append(cpu_baseline(x, THR, budget_s=budget, heads_total=w.B * w.H))
     elapsed = time.perf_counter() - t_all
     v = statistics.median(r["value"] for r in vals)
     cb = dict(vals[-1])
@@ -269,6 +273,113 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
                              "frac": bwd_tflops / peaks["bf16_sus"],
                              "algorithmic": "kept tiles x 10*64*64*D flops per call (executed: 14*64*64*D)"},
             "gpu_launches_per_step": 9}
+
+
+def builder_bytes(B: int, H: int, S: int, D: int, elem: int, kept_tiles: int) -> int:
+    """Algorithmic bytes of one mask build: Q and K read once, and the bitmask,
+    the counts, the kept key-block indices and the work list written."""
+    nb = -(-S // 64)
+    W = -(-nb // 32)
+    return 2 * B * H * S * D * elem + B * H * nb * (W * 4 + 4) + kept_tiles * 4 + B * H * -(-nb // 2) * 8
+
+
+def oracle_sample_ms(x: dict, thr: float, budget_s: float) -> dict:
+    """The fp64 oracle, as it stands, on head 0 of inputs x: its full mask, then
+    masked attention for as many query blocks as fit in budget_s, extrapolated
+    to all heads and query blocks of the workload (labelled as such)."""
+    import numpy as np
+    from oracle import nabla_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count()
+    B, H, S, D = x["q"].shape
+    q, k, v = x["q"][:1, :1], x["k"][:1, :1], x["v"][:1, :1]
+    t0 = time.perf_counter()
+    M, _, _ = orc.nabla_mask(q, k, thr)
+    t_mask = time.perf_counter() - t0
+    nb = M.shape[-1]
+    order = np.random.default_rng(0).permutation(nb)
+    spent, done = 0.0, 0
+    step = 2
+    while spent < budget_s and done < nb:
+        sel = order[done:done + step]
+        Ms = np.zeros_like(M)
+        Ms[0, 0, sel] = M[0, 0, sel]
+        t0 = time.perf_counter()
+        orc.masked_attention(q, k, v, Ms)
+        spent += time.perf_counter() - t0
+        done += len(sel)
+        step = min(step * 2, 64)
+    attn_ms = spent / done * nb * B * H * 1e3
+    mask_ms = t_mask * B * H * 1e3
+    return {"mask_ms": mask_ms, "attn_ms": attn_ms, "cores": threads, "host_cpus": os.cpu_count(),
+            "sample": f"head 0: full fp64 mask ({t_mask:.2f} s), attention for {done} of {nb} query blocks "
+                      f"({spent:.2f} s); both extrapolated linearly to {B * H} heads"
+                      + ("" if done < nb or B * H > 1 else " (complete)")}
+
+
+def measure_config(nabla, dev, wid: int, warmup: int, steps: int, oracle_budget_s: float = 3.0) -> dict:
+    """One workload at every threshold it names: per threshold the kept
+    fraction, mask-build ms and GB/s (algorithmic bytes, builder_bytes), and
+    attention ms and TFLOP/s on kept tiles (CUDA events on the launching
+    stream), each as a fraction of the measured peaks; next to them the fp64
+    oracle's time for the same workload on the host's cores (bounded sample,
+    extrapolated)."""
+    import torch
+    import synth
+    w = synth.WORKLOADS[wid]
+    x = synth.make_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    B, H, S, D = q.shape
+    elem = q.element_size()
+    ws = nabla.workspace(q)
+    mask = nabla.Mask.empty(B, H, S, dev, transpose=False)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    peaks = _peaks()
+    rows = []
+    for thr in w.thresholds:
+        def one(ev=None):
+            if ev:
+                ev[0].record(stream)
+            nabla.build_mask(q, k, thr, out=mask, ws=ws, transpose=False)
+            if ev:
+                ev[1].record(stream)
+            nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+            if ev:
+                ev[2].record(stream)
+
+        for _ in range(max(warmup, 1)):
+            one()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in evs:
+            one(e)
+        torch.cuda.synchronize()
+        if nabla.workspace_status(ws) != 0:
+            raise SystemExit(f"device status word reports a timeout in the {w.name} leg")
+        kept = int(mask.cnt.to(torch.int64).sum().item())
+        nb = mask.cnt.shape[-1]
+        mask_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        tflops = kept * 4 * 64 * 64 * D / (attn_ms * 1e-3) / 1e12
+        gbs = builder_bytes(B, H, S, D, elem, kept) / (mask_ms * 1e-3) / 1e9
+        row = {"thr": thr, "kept_fraction": kept / (B * H * nb * nb), "kept_tiles": kept,
+               "mask_ms": mask_ms, "mask_gbs": gbs, "mask_frac_hbm": gbs / peaks["hbm"],
+               "attn_ms": attn_ms, "attn_tflops": tflops}
+        if w.dtype == "bf16":
+            row["attn_frac_bf16_sustained"] = tflops / peaks["bf16_sus"]
+        else:
+            # CUDA-core fp32 path: nominal fp32 FMA rate of 148 SMs x 128 lanes x 2 flops at 1.965 GHz
+            row["attn_frac_fp32_nominal"] = tflops / (148 * 128 * 2 * 1.965e9 / 1e12)
+        rows.append(row)
+    out = {"workload": f"{w.name}: B={B} H={H} S={S} D={D} {w.dtype}, {w.T}x{w.Hl}x{w.Wl} tokens",
+           "steps": steps, "cases": rows,
+           "oracle": oracle_sample_ms(x, w.thresholds[0], oracle_budget_s)}
+    del q, k, v
+    return out
 
 
 def measure_sweep(nabla, q, k, v, coords, warmup: int, steps: int, with_sta: bool = True,
@@ -359,7 +470,7 @@ def measure_table1(nabla, dev, warmup: int, steps: int, heads: int | None = None
         w = w.scaled(H=heads)
     x = synth.make_inputs(w)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
-    coords = x["coords"].to(dev).int().contiguous()
+    coords = nabla.sta_block_coords(w.T, w.Hl, w.Wl, w.P, w.S).to(dev)
     B, H, S, D = q.shape
     ws = nabla.workspace(q)
     mask = nabla.Mask.empty(B, H, S, dev, transpose=False)
@@ -543,7 +654,7 @@ def main() -> None:
         ws_ = synth.WORKLOADS[WORKLOAD_ID]
         xs = synth.make_inputs(ws_)
         qs, ks, vs = (xs[n].to(dev0) for n in ("q", "k", "v"))
-        first = measure_sweep(nabla, qs, ks, vs, xs["coords"].to(dev0).int().contiguous(), max(1, args.warmup),
+        first = measure_sweep(nabla, qs, ks, vs, nabla.sta_block_coords(ws_.T, ws_.Hl, ws_.Wl, ws_.P, ws_.S).to(dev0), max(1, args.warmup),
                               max(1, args.steps))
         del qs, ks, vs
         print(json.dumps({"sweep": first, "sweep_sigma06": measure_sweep_sigma06(
@@ -628,9 +739,7 @@ def main() -> None:
     ms_step = total_ms / args.steps
     value = job_tflops(world, flops, ms_step)
     attn_tflops = flops / (attn_avg * 1e-3) / 1e12
-    W = -(-nb // 32)
-    mask_bytes = 2 * q.numel() * q.element_size() + B * H * nb * (W * 4 + 4) + kept_tiles * 4 \
-        + B * H * -(-nb // 2) * 8
+    mask_bytes = builder_bytes(B, H, S, D, q.element_size(), kept_tiles)
     mask_gbs = mask_bytes / (mask_avg * 1e-3) / 1e9
     peaks = _peaks()
 
@@ -653,7 +762,7 @@ def main() -> None:
 
     sweep = None
     if world == 1 and not args.no_sweep:
-        sweep = measure_sweep(nabla, q, k, v, x["coords"].to(dev).int().contiguous(), 1, 2)
+        sweep = measure_sweep(nabla, q, k, v, nabla.sta_block_coords(w.T, w.Hl, w.Wl, w.P, w.S).to(dev), 1, 2)
 
     sweep06 = None
     if world == 1 and not args.no_sweep:
@@ -662,6 +771,11 @@ def main() -> None:
     table1 = None
     if world == 1 and not args.no_sweep:
         table1 = measure_table1(nabla, dev, 1, 2)
+
+    configs = None
+    if world == 1 and not args.no_sweep:
+        configs = {"tiny_fp32": measure_config(nabla, dev, 1, 3, 5),
+                   "fwd_480p": measure_config(nabla, dev, 2, 2, 5)}
 
     if rank == 0:
         line = {
@@ -681,7 +795,13 @@ def main() -> None:
                                       f"burst {peaks['bf16']}",
                          "traffic": _traffic("attn_fwd_tc.cu"),
                          "algorithmic": "kept tiles x 4*64*64*D flops per launch"},
+            "mask_roofline": {"bound": "hbm", "kernels": "pool + score GEMM + select + work list",
+                              "achieved": mask_gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                              "frac": mask_gbs / peaks["hbm"], "bytes_per_call": mask_bytes,
+                              "ms_per_call": mask_avg, "traffic": None,
+                              "algorithmic": "Q + K read once; bitmask, counts, kept indices, work list written"},
             "e2e": e2e,
+            "configs": configs,
             "training": training,
             "sweep": sweep,
             "sweep_sigma06": sweep06,
@@ -692,7 +812,8 @@ def main() -> None:
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR)
+            line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR,
+                                                heads_total=B * H)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -20,8 +20,8 @@ import torch
 
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
-           "selftest_wait_timeout", "build_mask_noalloc", "fractal_reorder", "build_mask_topk",
-           "block_mass", "mask_recall",
+           "selftest_wait_timeout", "build_mask_noalloc", "build_mask_noalloc_status", "fractal_reorder",
+           "build_mask_topk", "block_mass", "mask_recall", "sta_block_coords",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -31,7 +31,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc",
-           "nabla_build_sta_mask", "nabla_mask_from_bits", "nabla_attn_fwd",
+           "nabla_build_mask_noalloc_status", "nabla_build_sta_mask", "nabla_sta_block_coords",
+           "nabla_mask_from_bits", "nabla_attn_fwd",
            "nabla_attn_bwd", "nabla_block_mass", "nabla_mask_recall", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
            "nabla_last_error", "nabla_abi_version"]
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.nabla_mask_from_bits.argtypes = [SH, P, MK, P, SZ, P]
     L.nabla_build_sta_mask.argtypes = [SH, ST, MK, P]
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
+    L.nabla_build_mask_noalloc_status.argtypes = [ctypes.POINTER(I32), P]
+    L.nabla_sta_block_coords.argtypes = [I32, I32, I32, I32, I32, P]
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_fractal_reorder.argtypes = [P, P, I32, I32, I32, I32, I32, SZ, I32, P]
@@ -90,7 +93,7 @@ def lib() -> ctypes.CDLL:
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
-                 "nabla_build_sta_mask",
+                 "nabla_build_mask_noalloc_status", "nabla_build_sta_mask", "nabla_sta_block_coords",
                  "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_block_mass",
                  "nabla_mask_recall",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
@@ -278,6 +281,30 @@ def build_mask_noalloc(q: torch.Tensor, k: torch.Tensor, thr: float,
                                           ctypes.c_float(thr),
                                           ctypes.byref(sta) if sta is not None else None,
                                           ctypes.byref(ms), _stream()), "nabla_build_mask_noalloc")
+    return out
+
+
+def build_mask_noalloc_status() -> int:
+    """Status word of build_mask_noalloc's static scratch on the current device
+    (0 = ok, 4 = a bounded wait of the last call ran out); synchronises the
+    current stream."""
+    out = ctypes.c_int32(-1)
+    _check(lib().nabla_build_mask_noalloc_status(ctypes.byref(out), _stream()),
+           "nabla_build_mask_noalloc_status")
+    return out.value
+
+
+def sta_block_coords(T: int, H: int, W: int, P: int = 8, S: int | None = None) -> torch.Tensor:
+    """STA tile coordinates (t, y // P, x // P) of the first token of every
+    64-token block of a T x H x W latent in the token order of §3.1.1, as a CPU
+    int32 tensor [ceil(S / 64), 3] (S defaults to T * H * W).  Move it to the
+    device for the sta_coords argument of build_mask / build_sta_mask."""
+    S = T * H * W if S is None else int(S)
+    if S < 1:
+        raise NablaError(f"S must be >= 1 (got {S})")
+    out = torch.empty(num_blocks(S), 3, dtype=torch.int32)
+    _check(lib().nabla_sta_block_coords(int(T), int(H), int(W), int(P), S, out.data_ptr()),
+           "nabla_sta_block_coords")
     return out
 
 

@@ -1,6 +1,7 @@
 // extern "C" entry points of libnabla.so: argument validation, workspace
 // layout, kernel dispatch and error reporting.  Declarations and the contract
 // of every call are in include/nabla.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -30,38 +31,6 @@ nabla_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
-
-nabla_status check_shape(const nabla_shape* s) {
-  if (!s) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
-  if (s->B < 1 || s->H < 1 || s->S < 1 || s->D < 1)
-    return fail(NABLA_ERR_INVALID_ARG, "B, H, S, D must be >= 1 (got %d, %d, %d, %d)", s->B, s->H,
-                s->S, s->D);
-  if (s->block != kBlock)
-    return fail(NABLA_ERR_UNSUPPORTED, "block must be %d (got %d)", kBlock, s->block);
-  if (s->dtype != NABLA_BF16 && s->dtype != NABLA_FP32)
-    return fail(NABLA_ERR_INVALID_ARG, "dtype must be NABLA_BF16 or NABLA_FP32 (got %d)", s->dtype);
-  if (s->D != 64 && s->D != 128)
-    return fail(NABLA_ERR_UNSUPPORTED, "head dimension D must be 64 or 128 (got %d)", s->D);
-  const long long nb = (s->S + kBlock - 1) / kBlock;
-  if (nb > kMaxBlocks)
-    return fail(NABLA_ERR_UNSUPPORTED, "S = %d gives %lld blocks; at most %d are supported", s->S,
-                nb, kMaxBlocks);
-  if ((long long)s->B * s->H > (1ll << 30))
-    return fail(NABLA_ERR_UNSUPPORTED, "B * H too large");
-  return NABLA_OK;
-}
-
-nabla_status check_tensor(const void* p, const char* name) {
-  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
-  if (!aligned(p, 16)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
-  return NABLA_OK;
-}
-
-nabla_status check_i32(const void* p, const char* name) {
-  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
-  if (!aligned(p, 4)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);
-  return NABLA_OK;
-}
 
 nabla_status check_ws(const Dims& d, bool bwd, const void* ws, size_t bytes) {
   const size_t need = ws_layout(d, bwd).total;
@@ -97,6 +66,45 @@ nabla_status emit_derived(const Dims& d, const uint32_t* bits, const nabla_mask*
   return NABLA_OK;
 }
 
+nabla_status reset_status(void* ws, cudaStream_t st) {
+  NABLA_CUDA(cudaMemsetAsync(ws, 0, 256, st), "clear workspace header");
+  return NABLA_OK;
+}
+
+}  // namespace
+
+nabla_status check_shape(const nabla_shape* s) {
+  if (!s) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->H < 1 || s->S < 1 || s->D < 1)
+    return fail(NABLA_ERR_INVALID_ARG, "B, H, S, D must be >= 1 (got %d, %d, %d, %d)", s->B, s->H,
+                s->S, s->D);
+  if (s->block != kBlock)
+    return fail(NABLA_ERR_UNSUPPORTED, "block must be %d (got %d)", kBlock, s->block);
+  if (s->dtype != NABLA_BF16 && s->dtype != NABLA_FP32)
+    return fail(NABLA_ERR_INVALID_ARG, "dtype must be NABLA_BF16 or NABLA_FP32 (got %d)", s->dtype);
+  if (s->D != 64 && s->D != 128)
+    return fail(NABLA_ERR_UNSUPPORTED, "head dimension D must be 64 or 128 (got %d)", s->D);
+  const long long nb = (s->S + kBlock - 1) / kBlock;
+  if (nb > kMaxBlocks)
+    return fail(NABLA_ERR_UNSUPPORTED, "S = %d gives %lld blocks; at most %d are supported", s->S,
+                nb, kMaxBlocks);
+  if ((long long)s->B * s->H > (1ll << 30))
+    return fail(NABLA_ERR_UNSUPPORTED, "B * H too large");
+  return NABLA_OK;
+}
+
+nabla_status check_tensor(const void* p, const char* name) {
+  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 16)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return NABLA_OK;
+}
+
+nabla_status check_i32(const void* p, const char* name) {
+  if (!p) return fail(NABLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 4)) return fail(NABLA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);
+  return NABLA_OK;
+}
+
 nabla_status check_mask_out(const nabla_mask* m, bool need_bits) {
   if (!m) return fail(NABLA_ERR_INVALID_ARG, "mask is NULL");
   if (need_bits) NABLA_TRY(check_i32(m->bits, "mask.bits"));
@@ -108,12 +116,18 @@ nabla_status check_mask_out(const nabla_mask* m, bool need_bits) {
   return NABLA_OK;
 }
 
-nabla_status reset_status(void* ws, cudaStream_t st) {
-  NABLA_CUDA(cudaMemsetAsync(ws, 0, 256, st), "clear workspace header");
+nabla_status check_selection(float thr, int32_t topk, const nabla_sta* sta) {
+  if (topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
+  if (topk == 0 && !(thr > 0.f && thr <= 1.f))
+    return fail(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1] (got %g)", (double)thr);
+  if (sta && sta->block_coords) {
+    NABLA_TRY(check_i32(sta->block_coords, "sta.block_coords"));
+    if (sta->wT < 1 || sta->wH < 1 || sta->wW < 1)
+      return fail(NABLA_ERR_INVALID_ARG, "STA window sizes must be >= 1 (got %d, %d, %d)", sta->wT,
+                  sta->wH, sta->wW);
+  }
   return NABLA_OK;
 }
-
-}  // namespace
 
 void record_error(nabla_status, const char* fmt, ...) {
   char buf[512];
@@ -153,15 +167,7 @@ static nabla_status build_mask_impl(const nabla_shape* shape, const void* q, con
   const Dims d = make_dims(*shape);
   NABLA_TRY(check_tensor(q, "q"));
   NABLA_TRY(check_tensor(k, "k"));
-  if (topk == 0 && !(thr > 0.f && thr <= 1.f))
-    return fail(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1] (got %g)", (double)thr);
-  if (topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
-  if (sta && sta->block_coords) {
-    NABLA_TRY(check_i32(sta->block_coords, "sta.block_coords"));
-    if (sta->wT < 1 || sta->wH < 1 || sta->wW < 1)
-      return fail(NABLA_ERR_INVALID_ARG, "STA window sizes must be >= 1 (got %d, %d, %d)", sta->wT,
-                  sta->wH, sta->wW);
-  }
+  NABLA_TRY(check_selection(thr, topk, sta));
   NABLA_TRY(check_mask_out(out, true));
   NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
   cudaStream_t st = (cudaStream_t)stream;
@@ -362,6 +368,45 @@ nabla_status nabla_workspace_status(const void* workspace, int32_t* host_status,
   NABLA_CUDA(cudaMemcpyAsync(host_status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, st),
              "read status word");
   NABLA_CUDA(cudaStreamSynchronize(st), "synchronise stream");
+  return NABLA_OK;
+}
+
+// Tile coordinate of the first token of every 64-token block.  Inside a
+// frame of H_lat x W_lat tokens the P x P patches follow in row-major patch
+// order, each patch's tokens contiguous (an edge patch cut by the frame holds
+// only its valid tokens); frames follow in time order.  Patch row py starts at
+// token py * P * W_lat of its frame (every patch row above it is P tokens
+// high), and inside that row, whose patches are ph = min(P, H_lat - py * P)
+// tokens high, patch px starts at px * ph * P (every patch left of it is P
+// tokens wide).  The tile coordinate of any token of patch (py, px) of frame t
+// is (t, py, px).
+nabla_status nabla_sta_block_coords(int32_t T, int32_t H_lat, int32_t W_lat, int32_t P, int32_t S,
+                                    int32_t* coords_host) {
+  g_last_error.clear();
+  if (!coords_host) return fail(NABLA_ERR_INVALID_ARG, "coords_host is NULL");
+  if (T < 1 || H_lat < 1 || W_lat < 1 || P < 1 || S < 1)
+    return fail(NABLA_ERR_INVALID_ARG, "T, H_lat, W_lat, P and S must be >= 1 (got %d, %d, %d, %d, %d)", T,
+                H_lat, W_lat, P, S);
+  const long long frame = (long long)H_lat * W_lat;
+  const long long tokens = frame * T;
+  const long long nb = ((long long)S + kBlock - 1) / kBlock;
+  if (tokens > 0x7fffffffll)
+    return fail(NABLA_ERR_INVALID_ARG, "T * H_lat * W_lat = %lld tokens is beyond int32", tokens);
+  if ((nb - 1) * kBlock >= tokens)
+    return fail(NABLA_ERR_INVALID_ARG,
+                "S = %d gives %lld blocks, but block %lld would start past the %lld tokens of the latent", S,
+                nb, nb - 1, tokens);
+  const long long patch_row = (long long)P * W_lat;
+  for (long long i = 0; i < nb; ++i) {
+    const long long n = i * kBlock;
+    const long long t = n / frame, r = n - t * frame;
+    const long long py = r / patch_row, rr = r - py * patch_row;
+    const long long ph = std::min<long long>(P, H_lat - py * P);
+    const long long px = rr / (ph * P);
+    coords_host[3 * i] = (int32_t)t;
+    coords_host[3 * i + 1] = (int32_t)py;
+    coords_host[3 * i + 2] = (int32_t)px;
+  }
   return NABLA_OK;
 }
 

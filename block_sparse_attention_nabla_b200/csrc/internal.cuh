@@ -80,6 +80,15 @@ int sm_count();
 // empty message clears it); status is for the reader's benefit only.
 void record_error(nabla_status status, const char* fmt, ...);
 
+// Argument checks shared by the entry points (abi.cu).  Each returns NABLA_OK
+// or records a message and returns the error status the header documents.
+nabla_status check_shape(const nabla_shape* s);                  // sizes, block, dtype, D, nb, B * H
+nabla_status check_tensor(const void* p, const char* name);      // non-NULL, 16-byte aligned
+nabla_status check_i32(const void* p, const char* name);         // non-NULL, 4-byte aligned
+nabla_status check_mask_out(const nabla_mask* m, bool need_bits);  // required lists present, aligned
+// thr in (0, 1] (topk == 0) or topk >= 1, and an optional STA window.
+nabla_status check_selection(float thr, int32_t topk, const nabla_sta* sta);
+
 // ---------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 

@@ -9,9 +9,15 @@
 // word) comes from the static array below instead of a caller workspace.
 //
 // The array lives in every GPU that loads this library until the process
-// exits.  Every call shares it and it keeps the last call's contents, so calls
-// whose work overlaps on the GPU (different streams, or different host
-// threads on one device) race on it; callers serialise them.
+// exits.  The first call on a device loads the module that holds it (CUDA
+// loads modules lazily), which commits the 32 MiB on that device; callers make
+// that first call, or nabla_build_mask_noalloc_status, at start-up, before they
+// reserve the rest of the device memory.  The status word at the start of the
+// array reports a bounded wait that ran out in the score GEMM, and
+// nabla_build_mask_noalloc_status reads it back.  Every call shares the array
+// and it keeps the last call's contents, so calls whose work overlaps on the
+// GPU (different streams, or different host threads on one device) race on
+// it; callers serialise them.
 #include <mutex>
 
 #include "internal.cuh"
@@ -59,13 +65,6 @@ nabla_status scratch_on_current_device(void** out) {
   return NABLA_OK;
 }
 
-bool al(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
-
-nabla_status bad(nabla_status s, const char* what) {
-  record_error(s, "%s", what);
-  return s;
-}
-
 }  // namespace
 }  // namespace nabla
 
@@ -77,26 +76,13 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
                                                            const nabla_mask* out,
                                                            nabla_stream_t stream) {
   record_error(NABLA_OK, "");
-  if (!shape) return bad(NABLA_ERR_INVALID_ARG, "shape is NULL");
-  if (shape->B < 1 || shape->H < 1 || shape->S < 1)
-    return bad(NABLA_ERR_INVALID_ARG, "B, H and S must be >= 1");
-  if (shape->block != kBlock) return bad(NABLA_ERR_UNSUPPORTED, "block must be 64");
-  if (shape->dtype != NABLA_BF16 && shape->dtype != NABLA_FP32)
-    return bad(NABLA_ERR_INVALID_ARG, "dtype must be NABLA_BF16 or NABLA_FP32");
-  if (shape->D != 64 && shape->D != 128) return bad(NABLA_ERR_UNSUPPORTED, "D must be 64 or 128");
-  if ((shape->S + kBlock - 1) / kBlock > kMaxBlocks) return bad(NABLA_ERR_UNSUPPORTED, "S too large");
-  if (!q || !k || !al(q, 16) || !al(k, 16))
-    return bad(NABLA_ERR_INVALID_ARG, "q and k must be non-NULL and 16-byte aligned");
-  if (!(thr > 0.f && thr <= 1.f)) return bad(NABLA_ERR_INVALID_ARG, "thr must lie in (0, 1]");
-  if (sta && sta->block_coords &&
-      (!al(sta->block_coords, 4) || sta->wT < 1 || sta->wH < 1 || sta->wW < 1))
-    return bad(NABLA_ERR_INVALID_ARG, "STA coordinates must be 4-byte aligned and windows >= 1");
-  if (!out || !out->bits || !out->cnt || !out->idx || !out->work)
-    return bad(NABLA_ERR_INVALID_ARG, "mask.bits, cnt, idx and work are required");
-  if (!al(out->bits, 4) || !al(out->cnt, 4) || !al(out->idx, 4) || !al(out->work, 4))
-    return bad(NABLA_ERR_INVALID_ARG, "mask arrays must be 4-byte aligned");
-  if ((out->cnt_t == nullptr) != (out->idx_t == nullptr))
-    return bad(NABLA_ERR_INVALID_ARG, "mask.cnt_t and mask.idx_t must both be set or both NULL");
+  // the same checks, with the same messages, as nabla_build_mask
+  nabla_status chk = check_shape(shape);
+  if (chk == NABLA_OK) chk = check_tensor(q, "q");
+  if (chk == NABLA_OK) chk = check_tensor(k, "k");
+  if (chk == NABLA_OK) chk = check_selection(thr, 0, sta);
+  if (chk == NABLA_OK) chk = check_mask_out(out, true);
+  if (chk != NABLA_OK) return chk;
   const Dims d = make_dims(*shape);
   const WsLayout L = ws_layout(d, false);
   if (L.total > kNoAllocScratchBytes) {
@@ -127,6 +113,27 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);
   if (e != cudaSuccess) {
     record_error(NABLA_ERR_CUDA, "nabla_build_mask_noalloc launch failed: %s", cudaGetErrorString(e));
+    return NABLA_ERR_CUDA;
+  }
+  return NABLA_OK;
+}
+
+extern "C" NABLA_API nabla_status nabla_build_mask_noalloc_status(int32_t* host_status,
+                                                                  nabla_stream_t stream) {
+  record_error(NABLA_OK, "");
+  if (!host_status) {
+    record_error(NABLA_ERR_INVALID_ARG, "host_status is NULL");
+    return NABLA_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  const nabla_status st0 = scratch_on_current_device(&scratch);
+  if (st0 != NABLA_OK) return st0;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(host_status, (const int32_t*)scratch + kWsStatus, sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    record_error(NABLA_ERR_CUDA, "reading the static scratch's status word failed: %s", cudaGetErrorString(e));
     return NABLA_ERR_CUDA;
   }
   return NABLA_OK;

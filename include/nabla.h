@@ -24,7 +24,8 @@
  *   mask row; npairs = ceil(nb / 2) query-block pairs per (b, h).
  * - Every pointer argument is a device pointer unless stated otherwise.  The
  *   caller owns every buffer, including the workspace; the library allocates no
- *   device memory and keeps no global device state.
+ *   device memory and keeps no global device state, except the static scratch
+ *   of nabla_build_mask_noalloc (below).
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *   stream).  A returned NABLA_OK means the arguments were valid and the work
  *   was enqueued; device-side failures (a bounded wait that ran out) are
@@ -154,15 +155,30 @@ NABLA_API nabla_status nabla_build_mask_topk(const nabla_shape* shape, const voi
  *   NABLA_ERR_UNSUPPORTED and a message naming both sizes.
  *   The first call on a device looks up the array's device address with that
  *   device current (cudaGetSymbolAddress) and caches it; make that first call
- *   before any stream capture.  The caller still provides q, k and every mask
- *   output.
+ *   before any stream capture.  CUDA loads the library's modules lazily, so
+ *   that first call is also when the 32 MiB is committed on the device (and it
+ *   may synchronise the device): make it, or a call of
+ *   nabla_build_mask_noalloc_status, at start-up, before reserving the rest of
+ *   the device memory or serving requests.  The caller still provides q, k and
+ *   every mask output.  Argument checks and their messages are those of
+ *   nabla_build_mask.
  *   All calls share the array and it keeps the last call's contents (the
  *   status word is cleared at the start of every call): calls whose GPU work
- *   overlaps race on it, so serialise them.  The status word is not readable
- *   through nabla_workspace_status. */
+ *   overlaps race on it, so serialise them.  A bounded wait that ran out inside
+ *   the builder (NABLA_ERR_TIMEOUT) is recorded in the array's status word, which
+ *   nabla_build_mask_noalloc_status reads back (not nabla_workspace_status). */
 NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const void* q,
                                                 const void* k, float thr, const nabla_sta* sta,
                                                 const nabla_mask* out, nabla_stream_t stream);
+
+/* Reads the status word of nabla_build_mask_noalloc's static scratch on the
+ * current device into *host_status (a host pointer): NABLA_OK, or
+ * NABLA_ERR_TIMEOUT if a bounded wait of the most recent call on this device
+ * ran out (its mask is then incomplete).  Copies on `stream` and synchronises
+ * it, so call it after the build on the same stream.  Allocates nothing; the
+ * paper has no counterpart.  Errors: NABLA_ERR_INVALID_ARG for a NULL
+ * host_status, NABLA_ERR_CUDA if the copy fails. */
+NABLA_API nabla_status nabla_build_mask_noalloc_status(int32_t* host_status, nabla_stream_t stream);
 
 /* Sliding-tile (STA) mask alone, without the NABLA selection: the STA
  * configurations of Table 1 (§4.1) and the neighbourhood mask of §2.2 (Eq. 5).
@@ -180,6 +196,31 @@ NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const 
  * instance the result of nabla_sta_block_coords); they are not range-checked. */
 NABLA_API nabla_status nabla_build_sta_mask(const nabla_shape* shape, const nabla_sta* sta, const nabla_mask* out,
                                             nabla_stream_t stream);
+
+/* Host helper: the STA tile coordinate of every 64-token block of a latent
+ * video laid out in the token order of §3.1.1 (Figure 3: inside each frame the
+ * P x P spatial patches follow in row-major patch order, each patch's tokens
+ * contiguous; frames keep their time order), for the window test of §2.2 ("a
+ * fixed 3D window ... centered on the query tile") used by nabla_build_mask
+ * and nabla_build_sta_mask.
+ *   T, H_lat, W_lat  latent frames and frame height / width in tokens (>= 1);
+ *   P                patch side in tokens (>= 1; 8 in the paper, so a full
+ *                    patch is one 64-token block);
+ *   S                tokens in the sequence the mask is built for (>= 1):
+ *                    T * H_lat * W_lat, or that count padded at the end; every
+ *                    block must start inside the latent, i.e.
+ *                    64 * (ceil(S / 64) - 1) < T * H_lat * W_lat;
+ *   coords_host      HOST int32 [ceil(S / 64)][3], caller-owned, written with
+ *                    (t, y / P, x / P) of each block's first token.
+ * When H_lat or W_lat is not a multiple of P the pages are silent; the reading
+ * used: an edge patch cut by the frame holds only its valid tokens (row-major)
+ * as one run, so blocks there may straddle patches and take the tile of their
+ * first token.  Then copy the array to the device for nabla_sta.block_coords.
+ * Runs on the host only (no CUDA call).  Errors: NABLA_ERR_INVALID_ARG for a
+ * NULL pointer, a size < 1, more than 2^31 - 1 latent tokens, or a block that
+ * starts past the latent. */
+NABLA_API nabla_status nabla_sta_block_coords(int32_t T, int32_t H_lat, int32_t W_lat, int32_t P, int32_t S,
+                                              int32_t* coords_host);
 
 /* Builds cnt, idx, work (and cnt_t, idx_t if not NULL) of `out` from a
  * caller-supplied bitmask `bits` [B, H, nb, W] (padding bits must be zero);

@@ -23,7 +23,7 @@ arXiv 2507.13546v1):
   rule is compared with, and the per-block fidelity check of the pooling
   proxy (token-level attention mass inside the retained blocks).
 
-Readings where the paper is silent (listed with reasons in the design notes):
+Readings where the paper is silent (each with its reason):
 
 * sort direction: ascending, so that cvals >= 1 - thr keeps the largest
   entries and thr = 1 keeps every block;
@@ -367,6 +367,24 @@ def fractal_order(T: int, Hl: int, Wl: int, P: int = 8) -> np.ndarray:
                     for x in range(px, min(px + P, Wl)):
                         order.append((t * Hl + y) * Wl + x)
     return np.asarray(order, dtype=np.int64)
+
+
+def block_tile_coords(T: int, Hl: int, Wl: int, P: int = 8, S: int | None = None, N: int = BLOCK) -> np.ndarray:
+    """STA tile coordinate of every N-token block of the reordered sequence
+    (§3.1.1 token order; the window of §2.2 is centred on the query tile): the
+    (t, y // P, x // P) of the block's first token, read off the gather index
+    of fractal_order.  S (default T * Hl * Wl) sets the number of blocks,
+    ceil(S / N); every block must start at a latent token.  int64 [nb, 3]."""
+    order = fractal_order(T, Hl, Wl, P)
+    S = len(order) if S is None else S
+    nb = num_blocks(S, N)
+    out = np.empty((nb, 3), dtype=np.int64)
+    for i in range(nb):
+        r = int(order[i * N])            # raster index t * Hl * Wl + y * Wl + x
+        t, rem = divmod(r, Hl * Wl)
+        y, x = divmod(rem, Wl)
+        out[i] = (t, y // P, x // P)
+    return out
 
 
 def fractal_reorder(X, T: int, Hl: int, Wl: int, P: int = 8, inverse: bool = False) -> np.ndarray:

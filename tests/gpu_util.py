@@ -135,3 +135,14 @@ def oracle_topk(q, k, topk, coords=None, window=None):
         M |= sta[None, None]
         X &= ~sta[None, None]
     return M, X
+
+
+def lib_coords(w) -> torch.Tensor:
+    """Block tile coordinates of workload w from the library's host helper
+    (nabla_sta_block_coords), on the device, as the STA argument of the builders."""
+    return nabla.sta_block_coords(w.T, w.Hl, w.Wl, w.P, w.S).cuda()
+
+
+def oracle_coords(w) -> np.ndarray:
+    """The same coordinates from the oracle's restatement of the token order."""
+    return orc.block_tile_coords(w.T, w.Hl, w.Wl, w.P, w.S)

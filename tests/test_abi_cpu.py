@@ -42,7 +42,7 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 16
+    assert len(names) == 18
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
@@ -229,3 +229,58 @@ def test_binding_refuses_masks_and_outputs_of_another_shape():
     with pytest.raises(nabla.NablaError, match="lse"):
         nabla._check_f32(torch.zeros(1, 2, 1000, dtype=torch.float64), (1, 2, 1000), "cpu", "lse")
     nabla._check_f32(torch.zeros(1, 2, 1000), (1, 2, 1000), "cpu", "lse")
+
+
+# ------------------------------------------------ STA block coordinates (host)
+
+def _lib_coords(L, T, H, W, P, S):
+    import numpy as np
+    nb = -(-S // 64)
+    out = (ctypes.c_int32 * (3 * nb))()
+    st = L.nabla_sta_block_coords(T, H, W, P, S, ctypes.cast(out, ctypes.c_void_p))
+    return st, np.frombuffer(out, dtype=np.int32).reshape(nb, 3)
+
+
+@pytest.mark.parametrize("T,H,W,P,S", [
+    (21, 30, 52, 8, 32760),       # 480p latent
+    (21, 45, 80, 8, 75600),       # 720p latent
+    (21, 48, 80, 8, 80640),       # 720p with frames padded to 48 rows (Table 1 layout)
+    (4, 32, 32, 8, 4096),         # tiny case
+    (16, 32, 32, 8, 16384),       # pretraining shape
+    (3, 12, 20, 8, 768),          # 720 tokens padded to 12 blocks
+    (2, 7, 9, 4, 126),            # patches of 4, ragged on both sides
+])
+def test_sta_block_coords_matches_the_oracle(L, T, H, W, P, S):
+    from oracle import nabla_oracle as orc
+    st, got = _lib_coords(L, T, H, W, P, S)
+    assert st == OK, L.nabla_last_error()
+    assert (got == orc.block_tile_coords(T, H, W, P, S)).all()
+
+
+def test_sta_block_coords_binding_and_errors(L):
+    from oracle import nabla_oracle as orc
+    c = nabla.sta_block_coords(21, 45, 80)
+    assert c.dtype.is_floating_point is False and tuple(c.shape) == (1182, 3) and not c.is_cuda
+    assert (c.numpy() == orc.block_tile_coords(21, 45, 80, 8)).all()
+    buf = (ctypes.c_int32 * 30)()
+    assert L.nabla_sta_block_coords(1, 12, 12, 8, 144, None) == INVALID
+    assert L.nabla_sta_block_coords(0, 12, 12, 8, 144, ctypes.cast(buf, ctypes.c_void_p)) == INVALID
+    assert L.nabla_sta_block_coords(1, 12, 12, 0, 144, ctypes.cast(buf, ctypes.c_void_p)) == INVALID
+    # block 3 of S = 193 would start at token 192, past the 144 latent tokens
+    assert L.nabla_sta_block_coords(1, 12, 12, 8, 193, ctypes.cast(buf, ctypes.c_void_p)) == INVALID
+    assert b"past" in L.nabla_last_error()
+    assert L.nabla_sta_block_coords(1, 12, 12, 8, 192, ctypes.cast(buf, ctypes.c_void_p)) == OK
+    with pytest.raises(nabla.NablaError, match="S must be"):
+        nabla.sta_block_coords(1, 12, 12, 8, 0)
+
+
+def test_noalloc_entry_points_refuse_bad_arguments_like_the_workspace_builder(L):
+    ms = mask_struct()
+    for thr, q, sh, word in ((0.0, FAKE, shape(), b"thr"), (0.5, None, shape(), b"q is NULL"),
+                             (0.5, FAKE, shape(D=96), b"head dimension"),
+                             (0.5, FAKE, shape(S=64 * 8192 + 1), b"blocks")):
+        a = L.nabla_build_mask_noalloc(ctypes.byref(sh), q, FAKE, ctypes.c_float(thr), None, ctypes.byref(ms), None)
+        msg_a = L.nabla_last_error()
+        b = _build(L, sh=sh, q=q, thr=thr)
+        assert a == b and a != OK and word in msg_a and msg_a == L.nabla_last_error()
+    assert L.nabla_build_mask_noalloc_status(None, None) == INVALID

@@ -222,3 +222,41 @@ def test_forward_with_tiny_wait_limit_stops_cleanly():
     assert nabla.workspace_status(ws) == 0
     O, _ = orc.masked_attention(x["q"][:, :1], x["k"][:, :1], x["v"][:, :1], M[:, :1])
     gu.assert_close(o[:, :1], O, "bf16", "O after timeout")
+
+
+def test_forward_with_long_runs_of_empty_units():
+    """External mask whose query-block pairs are empty in long runs, with many
+    more units (16 heads x 32 pairs = 512) than CTAs (two per SM), so each CTA
+    draws several units and meets empty units back to back, and after units
+    with tiles.  Rows of an empty block get O = 0 and LSE = -inf; the rest
+    match the oracle (Eq. 4 of §2.2), and no bounded wait runs out."""
+    B, H, S = 1, 16, 4096
+    x = synth.make_random_qkv(B, H, S, 128, "bf16", seed=41)
+    nb = S // 64
+    rng = np.random.default_rng(41)
+    M = rng.random((B, H, nb, nb)) < 0.3
+    for h in range(H):
+        # runs of empty pairs: pairs [a, a + len) of this head keep nothing
+        a = int(rng.integers(0, 20))
+        M[0, h, 2 * a:2 * (a + 6 + h % 3)] = False
+        if h % 2:
+            M[0, h, 0:2] = False                       # the head's first pair
+        if h % 4 == 1:
+            M[0, h, nb - 6:] = False                   # its last three pairs
+        M[0, h, 2 * (a + 10), :] = False               # one empty block inside a non-empty pair
+    M[0, 3] = False                                    # one head with no tile at all
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    ws = nabla.workspace(q)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    O, L = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, "bf16", "long runs of empty units")
+    empty = ~M.any(-1)                                 # [B, H, nb] query blocks that keep nothing
+    rows = np.repeat(empty, 64, axis=-1)[..., :S]
+    assert rows.sum() > 0
+    assert (o.float().cpu().numpy()[rows] == 0).all()
+    assert np.isneginf(lse.cpu().numpy()[rows]).all()
+    lg = lse.cpu().numpy()[~rows]
+    assert np.abs(lg - L[~rows]).max() < 1e-3

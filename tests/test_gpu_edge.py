@@ -42,12 +42,12 @@ def test_extreme_logits_mask_and_forward(scale):
 
 def test_sta_window_wider_than_the_grid_keeps_everything():
     w = synth.WORKLOADS[6]
-    coords = torch.from_numpy(synth.block_coords(w.T, w.Hl, w.Wl, w.P))
+    coords = nabla.sta_block_coords(w.T, w.Hl, w.Wl, w.P)
     mask = nabla.build_sta_mask((1, 1, w.S, w.D), coords.cuda(), (99, 999, 999))
     torch.cuda.synchronize()
     G = orc.bits_to_mask(gu.gpu_bits(mask), w.nb)
     assert G.all()
-    assert (orc.sta_mask(coords.numpy(), (99, 999, 999)) == G[0, 0]).all()
+    assert (orc.sta_mask(gu.oracle_coords(w), (99, 999, 999)) == G[0, 0]).all()
     gu.check_lists(mask, w.nb)
 
 

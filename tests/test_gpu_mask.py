@@ -21,10 +21,10 @@ def _run(w, heads=None, thr=None, sta=False):
     x = synth.make_inputs(w, heads=heads)
     thr = w.thresholds[0] if thr is None else thr
     q, k = x["q"].cuda(), x["k"].cuda()
-    coords = x["coords"].cuda() if sta else None
+    coords = gu.lib_coords(w) if sta else None
     mask = nabla.build_mask(q, k, thr, sta_coords=coords, sta_window=w.sta_window if sta else None)
     torch.cuda.synchronize()
-    M, C, stam = gu.oracle_mask(x["q"], x["k"], thr, x["coords"].numpy() if sta else None,
+    M, C, stam = gu.oracle_mask(x["q"], x["k"], thr, gu.oracle_coords(w) if sta else None,
                                 w.sta_window if sta else None)
     return x, mask, M, C, stam
 
@@ -142,9 +142,9 @@ def test_topk_720p_two_heads_at_the_cdf_budget(sta):
     q, k = x["q"].cuda(), x["k"].cuda()
     cdf = nabla.build_mask(q, k, 0.8)
     topk = int(round(cdf.cnt.float().mean().item()))
-    coords = x["coords"].cuda().int().contiguous() if sta else None
+    coords = gu.lib_coords(w) if sta else None
     mask = nabla.build_mask_topk(q, k, topk, sta_coords=coords, sta_window=w.sta_window if sta else None)
     torch.cuda.synchronize()
-    M, X = gu.oracle_topk(x["q"], x["k"], topk, x["coords"].numpy() if sta else None,
+    M, X = gu.oracle_topk(x["q"], x["k"], topk, gu.oracle_coords(w) if sta else None,
                           w.sta_window if sta else None)
     _topk_check(mask, M, X, w.nb, topk, sta)

@@ -31,12 +31,11 @@ def inputs():
 @pytest.mark.parametrize("window", [(18, 40, 40), (18, 24, 24), (11, 40, 40), (11, 24, 24), (1, 8, 8)])
 def test_sta_only_mask_matches_oracle(window, inputs):
     tiles = synth.sta_tiles(window)
-    coords = inputs["coords"]
     q_shape = (1, len(HEADS), W6.S, W6.D)
-    mask = nabla.build_sta_mask(q_shape, coords.cuda(), tiles)
+    mask = nabla.build_sta_mask(q_shape, gu.lib_coords(W6), tiles)
     torch.cuda.synchronize()
     G = orc.bits_to_mask(gu.gpu_bits(mask), W6.nb)
-    want = orc.sta_mask(coords.numpy(), tiles)
+    want = orc.sta_mask(gu.oracle_coords(W6), tiles)
     assert (G == want[None, None]).all()
     gu.check_lists(mask, W6.nb)
     printed = {tuple(int(v) for v in c[1]): float(c[2][0]) for c in _read_golden("sta_table1.txt")}
@@ -48,10 +47,9 @@ def test_sta_only_mask_matches_oracle(window, inputs):
 def test_nabla_table1_masks_match_oracle(name, thr, window, inputs):
     q, k = inputs["q"].cuda(), inputs["k"].cuda()
     tiles = synth.sta_tiles(window) if window else None
-    coords = inputs["coords"]
-    mask = nabla.build_mask(q, k, thr, sta_coords=coords.cuda() if tiles else None, sta_window=tiles)
+    mask = nabla.build_mask(q, k, thr, sta_coords=gu.lib_coords(W6) if tiles else None, sta_window=tiles)
     torch.cuda.synchronize()
-    M, C, stam = gu.oracle_mask(inputs["q"], inputs["k"], thr, coords.numpy() if tiles else None, tiles)
+    M, C, stam = gu.oracle_mask(inputs["q"], inputs["k"], thr, gu.oracle_coords(W6) if tiles else None, tiles)
     bad, band, diff = gu.compare_mask(mask, M, C, thr, stam)
     assert bad == 0, (name, bad, band, diff)
     gu.check_lists(mask, W6.nb, check_transpose=False)
@@ -61,7 +59,7 @@ def test_nabla_table1_masks_match_oracle(name, thr, window, inputs):
 def test_attention_under_table1_masks_sampled_rows(name, inputs):
     _, thr, window = next(c for c in synth.TABLE1 if c[0] == name)
     q, k, v = (inputs[n].cuda() for n in ("q", "k", "v"))
-    coords = inputs["coords"].cuda()
+    coords = gu.lib_coords(W6)
     tiles = synth.sta_tiles(window)
     if thr is None:
         mask = nabla.build_sta_mask(tuple(q.shape), coords, tiles)

@@ -26,12 +26,20 @@ def _all_pins():
         checks.append(lambda c=case: pins.test_fractal_order_hand_cases(c))
     for args in [(3, 30, 52, 8), (2, 45, 80, 8), (1, 7, 9, 4), (4, 8, 8, 8)]:
         checks.append(lambda a=args: pins.test_fractal_order_is_a_framewise_bijection_with_contiguous_patches(*a))
+    for case in pins._read_golden("block_coords_cases.txt"):
+        checks.append(lambda c=case: pins.test_block_tile_coords_hand_cases(c))
+    for args in [(21, 6, 10), (4, 4, 4), (16, 4, 4)]:
+        checks.append(lambda a=args: pins.test_block_tile_coords_full_patch_grids_are_the_tile_grid(*a))
+    for args in [(21, 30, 52), (21, 45, 80), (3, 12, 20)]:
+        checks.append(lambda a=args: pins.test_block_tile_coords_invariants(*a))
     for name in dir(pins):
         fn = getattr(pins, name)
         if name.startswith("test_") and callable(fn) and name not in (
                 "test_cdf_hand_cases", "test_sta_reproduces_table1_sparsity", "test_fractal_order_hand_cases",
                 "test_topk_hand_cases",
-                "test_fractal_order_is_a_framewise_bijection_with_contiguous_patches"):
+                "test_fractal_order_is_a_framewise_bijection_with_contiguous_patches",
+                "test_block_tile_coords_hand_cases", "test_block_tile_coords_full_patch_grids_are_the_tile_grid",
+                "test_block_tile_coords_invariants"):
             checks.append(fn)
     return checks
 
@@ -158,6 +166,21 @@ def _mass_unscaled(Q, K, N=64):
     return _ORIG_MASS(orc.as_f64(Q) * np.sqrt(D), K, N)
 
 
+def _coords_variant(last_token=False, xy_swapped=False):
+    def f(T, Hl, Wl, P=8, S=None, N=64):
+        order = orc.fractal_order(T, Hl, Wl, P)
+        S = len(order) if S is None else S
+        nb = -(-S // N)
+        out = np.empty((nb, 3), dtype=np.int64)
+        for i in range(nb):
+            r = int(order[min(i * N + N - 1, len(order) - 1)] if last_token else order[i * N])
+            t, rem = divmod(r, Hl * Wl)
+            y, x = divmod(rem, Wl)
+            out[i] = (t, x // P, y // P) if xy_swapped else (t, y // P, x // P)
+        return out
+    return f
+
+
 MUTANTS = {
     "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
     "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
@@ -184,6 +207,8 @@ MUTANTS = {
     "fractal_tokens_column_major": ("fractal_order", _fractal_variant(col_major_tokens=True)),
     "fractal_patches_column_major": ("fractal_order", _fractal_variant(col_major_patches=True)),
     "fractal_edge_patches_last": ("fractal_order", _fractal_variant(edges_last=True)),
+    "block_coords_of_last_token": ("block_tile_coords", _coords_variant(last_token=True)),
+    "block_coords_x_and_y_swapped": ("block_tile_coords", _coords_variant(xy_swapped=True)),
 }
 
 

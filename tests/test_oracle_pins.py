@@ -326,6 +326,40 @@ def test_fractal_reorder_inverse_restores_raster_order():
     assert np.array_equal(orc.fractal_reorder(Y, 3, 9, 11, 4, inverse=True), X)
 
 
+@pytest.mark.parametrize("case", _read_golden("block_coords_cases.txt"))
+def test_block_tile_coords_hand_cases(case):
+    T, H, W, P, S = (int(v) for v in case[0])
+    got = orc.block_tile_coords(T, H, W, P, S)
+    assert got.shape == (-(-S // 64), 3)
+    for part in case[1:]:
+        i, t, y, x = (int(v) for v in part)
+        assert got[i].tolist() == [t, y, x], (i, got[i])
+
+
+@pytest.mark.parametrize("T,Hy,Wx", [(21, 6, 10), (4, 4, 4), (16, 4, 4)])
+def test_block_tile_coords_full_patch_grids_are_the_tile_grid(T, Hy, Wx):
+    """When the frame sides are multiples of P = 8 every 64-token block is one
+    whole 8 x 8 patch, so the blocks enumerate the tile grid time-major and
+    patch-row-major (Table 1's padded 720p layout: 21 x 6 x 10 tiles)."""
+    got = orc.block_tile_coords(T, 8 * Hy, 8 * Wx, 8)
+    assert (got == orc.sta_grid_coords(T, Hy, Wx)).all()
+
+
+@pytest.mark.parametrize("T,H,W", [(21, 30, 52), (21, 45, 80), (3, 12, 20)])
+def test_block_tile_coords_invariants(T, H, W):
+    """Coordinates stay inside the tile grid, never decrease in time, and each
+    block's tile is the tile of its first token in the reordered sequence."""
+    got = orc.block_tile_coords(T, H, W, 8)
+    ny, nx = -(-H // 8), -(-W // 8)
+    assert (got[:, 0] >= 0).all() and (got[:, 0] < T).all()
+    assert (got[:, 1] < ny).all() and (got[:, 2] < nx).all() and (got >= 0).all()
+    assert (np.diff(got[:, 0]) >= 0).all()
+    order = orc.fractal_order(T, H, W, 8)
+    for i in (0, len(got) // 3, len(got) - 1):
+        r = int(order[64 * i])
+        assert got[i].tolist() == [r // (H * W), (r % (H * W)) // W // 8, (r % W) // 8]
+
+
 # ------------------------------------------------ fixed-budget comparator
 
 @pytest.mark.parametrize("case", _read_golden("topk_select_cases.txt"))

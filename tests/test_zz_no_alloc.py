@@ -41,7 +41,7 @@ def _same_mask(a: nabla.Mask, b: nabla.Mask) -> None:
 def test_noalloc_mask_equals_workspace_mask_on_two_calls():
     w = synth.WORKLOADS[3].scaled(H=2)                 # 720p frames, 2 heads, STA on
     inputs = [synth.make_inputs(w), synth.make_inputs(w.scaled(seed=77))]
-    coords = inputs[0]["coords"].cuda()
+    coords = nabla.sta_block_coords(w.T, w.Hl, w.Wl, w.P).cuda()
     for x, thr in zip(inputs, (0.8, 0.5)):
         q, k = x["q"].cuda(), x["k"].cuda()
         ref = nabla.build_mask(q, k, thr, sta_coords=coords, sta_window=w.sta_window)
@@ -68,3 +68,25 @@ def test_noalloc_rejects_shapes_beyond_the_static_scratch():
     assert st == 2
     msg = nabla.lib().nabla_last_error().decode()
     assert "static scratch" in msg and str(32 << 20) in msg
+
+
+def test_noalloc_status_reads_back_a_timeout_and_recovers():
+    """The score GEMM's bounded waits report into the static scratch's status
+    word, which nabla_build_mask_noalloc_status reads back: 0 after a normal
+    call; with a 1 ns wait limit the first wait that is not already satisfied
+    runs out and the word reads 4 (0 if every wait happened to be satisfied at
+    once); the next call with the default limit is correct again."""
+    x = synth.make_random_qkv(1, 4, 4096, 128, "bf16", seed=9)
+    q, k = x["q"].cuda(), x["k"].cuda()
+    ref = nabla.build_mask(q, k, 0.7)
+    nabla.build_mask_noalloc(q, k, 0.7)
+    assert nabla.build_mask_noalloc_status() == 0
+    try:
+        nabla.set_wait_limit_ns(1)
+        nabla.build_mask_noalloc(q, k, 0.7)
+        assert nabla.build_mask_noalloc_status() in (0, 4)
+    finally:
+        nabla.set_wait_limit_ns(0)
+    got = nabla.build_mask_noalloc(q, k, 0.7)
+    assert nabla.build_mask_noalloc_status() == 0
+    _same_mask(got, ref)
