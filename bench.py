@@ -218,8 +218,10 @@ def run_reference(args) -> None:
 def measure_training(dev, warmup: int, steps: int) -> dict:
     """The training leg: mask (with the transposed lists), forward and backward
     at the pretraining shape (B=2, H=16, S=16,384, D=128, bf16, thr 0.8), each
-    timed with CUDA events on the launching stream.  Backward flops are the
-    algorithmic 10 * 64 * 64 * D per kept tile (five GEMMs)."""
+    timed with CUDA events on the launching stream.  The forward runs in
+    residual mode (o_res: the backward takes rowsum(dO * O) from o + o_res);
+    the plain forward (no residual) is timed beside it for its cost.  Backward
+    flops are the algorithmic 10 * 64 * 64 * D per kept tile (five GEMMs)."""
     import torch
 
     import block_sparse_attention_nabla_b200 as nabla
@@ -231,6 +233,7 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
     ws = nabla.workspace(q, want_bwd=True)
     mask = nabla.Mask.empty(B, H, S, dev, transpose=True)
     o, lse = torch.empty_like(q), torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    o_res = torch.empty_like(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream()
 
@@ -240,17 +243,20 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
         nabla.build_mask(q, k, w.thresholds[0], out=mask, ws=ws, transpose=True)
         if ev:
             ev[1].record(stream)
-        nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+        nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws, o_res=o_res)
         if ev:
             ev[2].record(stream)
-        nabla.attn_bwd(q, k, v, o, do, lse, mask, dq=dq, dk=dk, dv=dv, ws=ws)
+        nabla.attn_bwd(q, k, v, o, do, lse, mask, dq=dq, dk=dk, dv=dv, ws=ws, o_res=o_res)
         if ev:
             ev[3].record(stream)
+        nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+        if ev:
+            ev[4].record(stream)
 
     for _ in range(max(warmup, 1)):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     for i in range(steps):
         step(evs[i])
     torch.cuda.synchronize()
@@ -259,6 +265,7 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
     mask_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    fwd_plain_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
     kept = int(mask.cnt.to(torch.int64).sum().item())
     nb = mask.cnt.shape[-1]
     peaks = _peaks()
@@ -267,12 +274,14 @@ def measure_training(dev, warmup: int, steps: int) -> dict:
     return {"workload": f"{w.name}: B={B} H={H} S={S} D={D} bf16, thr {w.thresholds[0]}, fwd + bwd with dO",
             "kept_fraction": kept / (B * H * nb * nb), "kept_tiles": kept, "steps": steps,
             "mask_ms": mask_ms, "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops,
+            "fwd_mode": "residual (o_res written; P V with P in two bf16 terms)",
+            "fwd_plain_ms": fwd_plain_ms, "fwd_plain_tflops": kept * 4 * 64 * 64 * D / (fwd_plain_ms * 1e-3) / 1e12,
             "bwd_ms": bwd_ms, "bwd_tflops": bwd_tflops,
             "bwd_roofline": {"bound": "tensor", "kernels": "bwd_stats + dkdv_tc + dq_tc (attn_bwd_tc.cu)",
                              "achieved": bwd_tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
                              "frac": bwd_tflops / peaks["bf16_sus"],
                              "algorithmic": "kept tiles x 10*64*64*D flops per call (executed: 14*64*64*D)"},
-            "gpu_launches_per_step": 9}
+            "gpu_launches_per_step": 10}
 
 
 def builder_bytes(B: int, H: int, S: int, D: int, elem: int, kept_tiles: int) -> int:

@@ -82,8 +82,8 @@ def lib() -> ctypes.CDLL:
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
     L.nabla_build_mask_noalloc_status.argtypes = [ctypes.POINTER(I32), P]
     L.nabla_sta_block_coords.argtypes = [I32, I32, I32, I32, I32, P]
-    L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, SZ, P]
-    L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
+    L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, P, SZ, P]
+    L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_fractal_reorder.argtypes = [P, P, I32, I32, I32, I32, I32, SZ, I32, P]
     L.nabla_block_mass.argtypes = [SH, P, P, P, P, SZ, P]
     L.nabla_mask_recall.argtypes = [SH, P, P, P, P]
@@ -390,27 +390,34 @@ def fractal_reorder(x: torch.Tensor, T: int, H: int, W: int, P: int = 8, inverse
     return out
 
 
-def attn_fwd(q, k, v, mask: Mask, o=None, lse=None, ws=None):
-    """Block-sparse attention forward; returns (o, lse)."""
+def attn_fwd(q, k, v, mask: Mask, o=None, lse=None, ws=None, o_res=None):
+    """Block-sparse attention forward; returns (o, lse).  Pass o_res (a bf16
+    tensor shaped like q) to also get the rounding residual of o, for training:
+    attn_bwd then takes rowsum(dO * O) from o + o_res."""
     sh = _shape_of(q)
     _same(q, k, v)
     o = o if o is not None else torch.empty_like(q)
     lse = lse if lse is not None else torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     _same(q, o)
+    if o_res is not None:
+        _same(q, o_res)
     _check_f32(lse, tuple(q.shape[:3]), q.device, "lse")
     mask.check(sh.B, sh.H, sh.S, q.device)
     ws = ws if ws is not None else workspace(q)
     ms = mask.as_struct()
     _check(lib().nabla_attn_fwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                ctypes.byref(ms), o.data_ptr(), lse.data_ptr(), ws.data_ptr(),
+                                ctypes.byref(ms), o.data_ptr(), _ptr(o_res), lse.data_ptr(), ws.data_ptr(),
                                 ws.numel(), _stream()), "nabla_attn_fwd")
     return o, lse
 
 
-def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None, dq=None, dk=None, dv=None):
-    """Backward of attn_fwd under the same mask; returns (dq, dk, dv)."""
+def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None, dq=None, dk=None, dv=None, o_res=None):
+    """Backward of attn_fwd under the same mask; returns (dq, dk, dv).  o_res:
+    the forward's residual of o, if it wrote one."""
     sh = _shape_of(q)
     _same(q, k, v, o, do)
+    if o_res is not None:
+        _same(q, o_res)
     dq = dq if dq is not None else torch.empty_like(q)
     dk = dk if dk is not None else torch.empty_like(k)
     dv = dv if dv is not None else torch.empty_like(v)
@@ -420,7 +427,7 @@ def attn_bwd(q, k, v, o, do, lse, mask: Mask, ws=None, dq=None, dk=None, dv=None
     ws = ws if ws is not None else workspace(q, want_bwd=True)
     ms = mask.as_struct()
     _check(lib().nabla_attn_bwd(ctypes.byref(sh), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                o.data_ptr(), do.data_ptr(), lse.data_ptr(), ctypes.byref(ms),
+                                o.data_ptr(), _ptr(o_res), do.data_ptr(), lse.data_ptr(), ctypes.byref(ms),
                                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
                                 ws.numel(), _stream()), "nabla_attn_bwd")
     return dq, dk, dv

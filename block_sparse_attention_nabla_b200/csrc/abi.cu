@@ -288,7 +288,7 @@ nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint32_t* bits
 }
 
 nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
-                            const nabla_mask* mask, void* o, float* lse, void* workspace,
+                            const nabla_mask* mask, void* o, void* o_res, float* lse, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream) {
   g_last_error.clear();
   NABLA_TRY(check_shape(shape));
@@ -297,13 +297,18 @@ nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(check_tensor(k, "k"));
   NABLA_TRY(check_tensor(v, "v"));
   NABLA_TRY(check_tensor(o, "o"));
+  if (o_res) {
+    NABLA_TRY(check_tensor(o_res, "o_res"));
+    if (d.dtype != NABLA_BF16)
+      return fail(NABLA_ERR_INVALID_ARG, "o_res applies to bf16 only (an fp32 O needs no residual)");
+  }
   if (lse && !aligned(lse, 4)) return fail(NABLA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
   NABLA_TRY(check_mask_out(mask, true));
   NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
   cudaStream_t st = (cudaStream_t)stream;
   NABLA_TRY(reset_status(workspace, st));
   if (d.dtype == NABLA_BF16)
-    NABLA_CUDA(launch_attn_fwd_tc(d, q, k, v, mask->bits, mask->work, o, lse, (int32_t*)workspace, st),
+    NABLA_CUDA(launch_attn_fwd_tc(d, q, k, v, mask->bits, mask->work, o, o_res, lse, (int32_t*)workspace, st),
                "tensor-core attention forward");
   else
     NABLA_CUDA(launch_attn_fwd_simt(d, q, k, v, mask->cnt, mask->idx, o, lse, st),
@@ -312,7 +317,7 @@ nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void*
 }
 
 nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
-                            const void* o, const void* dout, const float* lse,
+                            const void* o, const void* o_res, const void* dout, const float* lse,
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream) {
   g_last_error.clear();
@@ -323,6 +328,11 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(check_tensor(v, "v"));
   NABLA_TRY(check_tensor(o, "o"));
   NABLA_TRY(check_tensor(dout, "dout"));
+  if (o_res) {
+    NABLA_TRY(check_tensor(o_res, "o_res"));
+    if (d.dtype != NABLA_BF16)
+      return fail(NABLA_ERR_INVALID_ARG, "o_res applies to bf16 only (an fp32 O needs no residual)");
+  }
   NABLA_TRY(check_tensor(dq, "dq"));
   NABLA_TRY(check_tensor(dk, "dk"));
   NABLA_TRY(check_tensor(dv, "dv"));
@@ -335,12 +345,12 @@ nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void*
   NABLA_TRY(reset_status(workspace, st));
   char* ws = (char*)workspace;
   if (d.dtype == NABLA_BF16 && d.D == 128)
-    NABLA_CUDA(launch_attn_bwd_tc(d, q, k, v, o, dout, lse, mask->bits, mask->cnt, mask->idx, mask->cnt_t,
+    NABLA_CUDA(launch_attn_bwd_tc(d, q, k, v, o, o_res, dout, lse, mask->bits, mask->cnt, mask->idx, mask->cnt_t,
                                   (float*)(ws + L.lse2p), (float*)(ws + L.deltap), dq, dk, dv,
                                   (int32_t*)ws, st),
                "tensor-core attention backward");
   else
-    NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
+    NABLA_CUDA(launch_attn_bwd_simt(d, q, k, v, o, o_res, dout, lse, mask->cnt, mask->idx, mask->cnt_t,
                                     mask->idx_t, (float*)(ws + L.delta), dq, dk, dv, st),
                "attention backward");
   return NABLA_OK;

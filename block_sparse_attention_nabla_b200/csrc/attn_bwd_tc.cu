@@ -774,6 +774,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // and Delta = 0 for the padding, so padded rows get P = 0.  One warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_stats_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ o_res,
                                                         const __nv_bfloat16* __restrict__ dout,
                                                         const float* __restrict__ lse, int S, int nb,
                                                         long long rows, float* __restrict__ lse2p,
@@ -792,7 +793,14 @@ __global__ void __launch_bounds__(256) bwd_stats_kernel(const __nv_bfloat16* __r
     for (int e = 0; e < E; e += 2) {
       const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + base + lane * E + e);
       const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(dout + base + lane * E + e);
-      const float2 fa = __bfloat1622float2(a), fc = __bfloat1622float2(c);
+      float2 fa = __bfloat1622float2(a);
+      const float2 fc = __bfloat1622float2(c);
+      if (o_res) {
+        // O + its rounding residual: the forward's fp32 O to about 2^-16
+        const float2 fr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o_res + base + lane * E + e));
+        fa.x += fr.x;
+        fa.y += fr.y;
+      }
       acc = fmaf(fa.x, fc.x, acc);
       acc = fmaf(fa.y, fc.y, acc);
     }
@@ -808,13 +816,14 @@ __global__ void __launch_bounds__(256) bwd_stats_kernel(const __nv_bfloat16* __r
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
+                               const void* o_res, const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
                                const int32_t* idx, const int32_t* cnt_t, float* lse2p, float* deltap, void* dq,
                                void* dk, void* dv, int32_t* ws_header, cudaStream_t st) {
   if (d.dtype != NABLA_BF16 || d.D != 128) return cudaErrorInvalidValue;
   const long long rows = d.BH() * d.nb * 64;
   bwd_stats_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, d.S, d.nb, rows, lse2p, deltap);
+      (const __nv_bfloat16*)o, (const __nv_bfloat16*)o_res, (const __nv_bfloat16*)dout, lse, d.S, d.nb, rows,
+      lse2p, deltap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tdo;

@@ -33,6 +33,14 @@
 //               only when the running max grows by more than 2^8 (exact after
 //               the final division); finally O / l and LSE.
 // TMEM columns: [0, 64) S0 / P0, [64, 128) S1 / P1, [128, 128 + D) O.
+//
+// Residual mode (a caller that trains passes o_res): the softmax threads also
+// write P_lo = bf16(P - bf16(P)) into the upper 32 columns of the S buffer, the
+// issuer adds O += P_lo V after O += P V, and the epilogue writes, beside the
+// bf16 O, its rounding residual bf16(O - bf16(O)).  O + o_res then carries the
+// softmax-weighted sum at about 2^-16 relative instead of 2^-9, which the
+// backward needs for Delta = rowsum(dO * O) in rows whose softmax is nearly
+// one-hot (there dS = P (dP - Delta) cancels).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -136,12 +144,13 @@ struct WalkIter {
   }
 };
 
-template <int D>
+template <int D, bool kRes>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ bits,
                   const int32_t* __restrict__ work, int n_units, int S, int nb, int W, int npairs,
-                  float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                  float scale_log2, __nv_bfloat16* __restrict__ out, __nv_bfloat16* __restrict__ out_res,
+                  float* __restrict__ lse,
                   int32_t* __restrict__ unit_ctr, int32_t* __restrict__ status, uint64_t limit_ns) {
   using L = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -305,6 +314,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const uint64_t bdesc = desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
           mma_ts(tmem + kOCol, tmem + sb * 64 + kk * 8, bdesc, idesc_o, (h > unit_first || kk > 0) ? 1u : 0u);
         }
+        if constexpr (kRes) {
+          // O += P_lo V: the bf16 remainder of P, kept in the S buffer's
+          // upper 32 columns, so that O carries P at about 2^-16 relative
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
+            mma_ts(tmem + kOCol, tmem + sb * 64 + 32 + kk * 8, bdesc, idesc_o, 1u);
+          }
+        }
         mma_commit(b.v_empty + vs);
         mma_commit(b.o_done);
         return true;
@@ -384,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // block j only writes P = 0.
         const bool mine = (flags & my_flag) != 0;
         uint32_t pk[32];
+        uint32_t plo[kRes ? 32 : 1];
         float corr = 1.f;
         bool rescale = false;
         if (mine) {
@@ -428,6 +447,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (c & 1) acc2b = fadd2(acc2b, f2pack(p0, p1));
             else acc2 = fadd2(acc2, f2pack(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
+            if constexpr (kRes) {
+              // p minus its bf16 value is exact in fp32; its bf16 rounding
+              // leaves about 2^-9 of that, i.e. 2^-17 of p
+              const float h0 = __uint_as_float(pk[c] << 16), h1 = __uint_as_float(pk[c] & 0xffff0000u);
+              plo[c] = pack_bf16x2(p0 - h0, p1 - h1);
+            }
           }
           float s0, s1, s2, s3;
           f2unpack(acc2, s0, s1);
@@ -436,8 +461,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          if constexpr (kRes) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) plo[c] = 0u;
+          }
         }
         tmem_st32(lane_base + sb * 64, pk);
+        if constexpr (kRes) tmem_st32(lane_base + sb * 64 + 32, plo);
         if (__any_sync(0xffffffffu, rescale)) {
           // O must hold the sum over tiles < g before it is scaled.  S of
           // tile g completed, and it was issued after P V of tile g - 2, so
@@ -495,6 +525,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = pkd[e];
         }
+        if constexpr (kRes) {
+          // the rounding residual O - bf16(O), itself rounded to bf16
+          uint4 rkd[4];
+          uint32_t* rw = reinterpret_cast<uint32_t*>(rkd);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float o0 = __uint_as_float(ov[2 * c]) * inv, o1 = __uint_as_float(ov[2 * c + 1]) * inv;
+            rw[c] = pack_bf16x2(o0 - __uint_as_float(pw[c] << 16), o1 - __uint_as_float(pw[c] & 0xffff0000u));
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(out_res + ((long long)bh * S + qrow) * D + c0);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = rkd[e];
+          }
+        }
       }
       if (valid && lse) lse[(long long)bh * S + qrow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
@@ -516,34 +561,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(status, 0, (int32_t)NABLA_ERR_TIMEOUT);
 }
 
-template <int D>
+template <int D, bool kRes>
 cudaError_t run(const Dims& d, const void* q, const void* k, const void* v, const uint32_t* bits,
-                const int32_t* work, void* o, float* lse, int32_t* ws_header, cudaStream_t st) {
+                const int32_t* work, void* o, void* o_res, float* lse, int32_t* ws_header, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (!make_map_bf16(&tq, q, d, 128) || !make_map_bf16(&tk, k, d, 64) || !make_map_bf16(&tv, v, d, 64))
     return cudaErrorInvalidValue;
   const int n_units = (int)(d.BH() * d.npairs);
   const int grid = std::min(n_units, kCtasPerSm * sm_count());
-  auto kern = fwd_tc_kernel<D>;
+  auto kern = fwd_tc_kernel<D, kRes>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)FwdLayout<D>::bytes);
   if (e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   kern<<<grid, kThreads, FwdLayout<D>::bytes, st>>>(tq, tk, tv, bits, work, n_units, d.S, d.nb, d.W,
-                                                    d.npairs, scale_log2, (__nv_bfloat16*)o, lse,
-                                                    ws_header + kWsUnitCounter, ws_header + kWsStatus,
-                                                    wait_limit_ns());
+                                                    d.npairs, scale_log2, (__nv_bfloat16*)o,
+                                                    (__nv_bfloat16*)o_res, lse, ws_header + kWsUnitCounter,
+                                                    ws_header + kWsStatus, wait_limit_ns());
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
-                               const uint32_t* bits, const int32_t* work, void* o, float* lse,
+                               const uint32_t* bits, const int32_t* work, void* o, void* o_res, float* lse,
                                int32_t* ws_header, cudaStream_t st) {
   if (d.dtype != NABLA_BF16) return cudaErrorInvalidValue;
-  if (d.D == 128) return run<128>(d, q, k, v, bits, work, o, lse, ws_header, st);
-  return run<64>(d, q, k, v, bits, work, o, lse, ws_header, st);
+  if (o_res) {
+    if (d.D == 128) return run<128, true>(d, q, k, v, bits, work, o, o_res, lse, ws_header, st);
+    return run<64, true>(d, q, k, v, bits, work, o, o_res, lse, ws_header, st);
+  }
+  if (d.D == 128) return run<128, false>(d, q, k, v, bits, work, o, nullptr, lse, ws_header, st);
+  return run<64, false>(d, q, k, v, bits, work, o, nullptr, lse, ws_header, st);
 }
 
 }  // namespace nabla

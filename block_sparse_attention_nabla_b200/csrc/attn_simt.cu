@@ -113,15 +113,21 @@ __global__ void __launch_bounds__(256) fwd_kernel(const T* __restrict__ q, const
   }
 }
 
-// Delta_r = sum_d dO[r][d] * O[r][d], one warp per row.
+// Delta_r = sum_d dO[r][d] * O[r][d], one warp per row; O plus its rounding
+// residual when the forward wrote one (bf16 only, o_res may be NULL).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, const T* __restrict__ dout,
-                                                    float* __restrict__ delta, long long rows) {
+__global__ void __launch_bounds__(256) delta_kernel(const T* __restrict__ o, const T* __restrict__ o_res,
+                                                    const T* __restrict__ dout, float* __restrict__ delta,
+                                                    long long rows) {
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   float s = 0.f;
-  for (int d = lane; d < D; d += 32) s = fmaf(to_f(o[row * D + d]), to_f(dout[row * D + d]), s);
+  for (int d = lane; d < D; d += 32) {
+    float od = to_f(o[row * D + d]);
+    if (o_res) od += to_f(o_res[row * D + d]);
+    s = fmaf(od, to_f(dout[row * D + d]), s);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) delta[row] = s;
@@ -284,13 +290,13 @@ cudaError_t fwd_t(const Dims& d, const void* q, const void* k, const void* v, co
 
 template <typename T, int D>
 cudaError_t bwd_t(const Dims& d, const void* q, const void* k, const void* v, const void* o,
-                  const void* dout, const float* lse, const int32_t* cnt, const int32_t* idx,
+                  const void* o_res, const void* dout, const float* lse, const int32_t* cnt, const int32_t* idx,
                   const int32_t* cnt_t, const int32_t* idx_t, float* delta, void* dq, void* dk,
                   void* dv, cudaStream_t st) {
   const float scale = 1.0f / sqrtf((float)D);
   const long long rows = d.BH() * d.S;
-  delta_kernel<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>((const T*)o, (const T*)dout,
-                                                                           delta, rows);
+  delta_kernel<T, D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>((const T*)o, (const T*)o_res,
+                                                                           (const T*)dout, delta, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(float) * (4 * 64 * (D + 1) + 2 * 64 * 65 + 128);
@@ -319,18 +325,18 @@ cudaError_t launch_attn_fwd_simt(const Dims& d, const void* q, const void* k, co
 }
 
 cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
-                                 const void* o, const void* dout, const float* lse,
+                                 const void* o, const void* o_res, const void* dout, const float* lse,
                                  const int32_t* cnt, const int32_t* idx, const int32_t* cnt_t,
                                  const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
                                  cudaStream_t st) {
   if (d.dtype == NABLA_FP32) {
     if (d.D == 128)
-      return bwd_t<float, 128>(d, q, k, v, o, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
-    return bwd_t<float, 64>(d, q, k, v, o, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
+      return bwd_t<float, 128>(d, q, k, v, o, o_res, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
+    return bwd_t<float, 64>(d, q, k, v, o, o_res, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
   }
   if (d.D == 128)
-    return bwd_t<__nv_bfloat16, 128>(d, q, k, v, o, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
-  return bwd_t<__nv_bfloat16, 64>(d, q, k, v, o, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
+    return bwd_t<__nv_bfloat16, 128>(d, q, k, v, o, o_res, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
+  return bwd_t<__nv_bfloat16, 64>(d, q, k, v, o, o_res, dout, lse, cnt, idx, cnt_t, idx_t, delta, dq, dk, dv, st);
 }
 
 }  // namespace nabla

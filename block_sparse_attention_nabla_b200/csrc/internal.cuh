@@ -113,7 +113,7 @@ cudaError_t launch_attn_fwd_simt(const Dims& d, const void* q, const void* k, co
                                  const int32_t* cnt, const int32_t* idx, void* o, float* lse,
                                  cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
-                                 const void* o, const void* dout, const float* lse,
+                                 const void* o, const void* o_res, const void* dout, const float* lse,
                                  const int32_t* cnt, const int32_t* idx, const int32_t* cnt_t,
                                  const int32_t* idx_t, float* delta, void* dq, void* dk, void* dv,
                                  cudaStream_t st);
@@ -123,13 +123,14 @@ cudaError_t launch_mask_recall(const Dims& d, const float* mass, const uint32_t*
                                cudaStream_t st);
 cudaError_t launch_fractal_reorder(const void* x, void* y, int B, int T, int H, int W, int P,
                                    size_t row_bytes, int inverse, cudaStream_t st);
+// o_res: NULL, or [B, H, S, D] bf16 for the rounding residual of O (residual mode).
 cudaError_t launch_attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v,
-                               const uint32_t* bits, const int32_t* work, void* o, float* lse,
+                               const uint32_t* bits, const int32_t* work, void* o, void* o_res, float* lse,
                                int32_t* ws_header, cudaStream_t st);
 
 // bf16, D = 128 only.  lse2p / deltap: workspace [B*H][nb*64] fp32 each.
 cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
+                               const void* o_res, const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
                                const int32_t* idx, const int32_t* cnt_t, float* lse2p, float* deltap, void* dq,
                                void* dk, void* dv, int32_t* ws_header, cudaStream_t st);
 

@@ -50,7 +50,7 @@ extern "C" {
 #define NABLA_API
 #endif
 
-#define NABLA_ABI_VERSION 1
+#define NABLA_ABI_VERSION 2
 #define NABLA_BLOCK 64
 
 typedef struct CUstream_st* nabla_stream_t; /* same type as cudaStream_t */
@@ -234,24 +234,35 @@ NABLA_API nabla_status nabla_mask_from_bits(const nabla_shape* shape, const uint
  * tiles of `mask` (bits, cnt, idx and work must all describe the same mask:
  * the bf16 path walks bits and work, the fp32 path cnt and idx) and outside
  * the sequence.
- *   o    [B, H, S, D] output, shape->dtype.
- *   lse  float [B, H, S]: natural-log log-sum-exp of the scaled logits
- *        (Q K^T / sqrt(D)) over the attended keys, needed by the backward.
- *        May be NULL.  A row with no kept block gets o = 0, lse = -inf.
+ *   o      [B, H, S, D] output, shape->dtype.
+ *   o_res  NULL, or (bf16 only) [B, H, S, D] bf16, 16-byte aligned: the
+ *          rounding residual of o, bf16(O - bf16(O)), for training.  With it
+ *          the tensor cores also multiply V by the bf16 remainder of the
+ *          softmax weights P (P itself enters the product in bf16), so that
+ *          o + o_res carries the attention output to about 2^-16 relative
+ *          instead of 2^-9; nabla_attn_bwd uses it for
+ *          Delta = rowsum(dO * O), which rows with a nearly one-hot softmax
+ *          need (there dS = P (dP - Delta) cancels).  Costs one more P V
+ *          product per tile.  NABLA_ERR_INVALID_ARG for fp32 (no residual).
+ *   lse    float [B, H, S]: natural-log log-sum-exp of the scaled logits
+ *          (Q K^T / sqrt(D)) over the attended keys, needed by the backward.
+ *          May be NULL.  A row with no kept block gets o = 0 (and o_res = 0),
+ *          lse = -inf.
  * bf16 runs on the tensor cores (tcgen05, fp32 accumulation in TMEM); fp32 runs
  * in fp32 on the CUDA cores. */
 NABLA_API nabla_status nabla_attn_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
-                            const nabla_mask* mask, void* o, float* lse, void* workspace,
+                            const nabla_mask* mask, void* o, void* o_res, float* lse, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 
 /* Backward of nabla_attn_fwd with the mask held constant (no gradient flows
  * into the mask builder).  o and lse are the forward's outputs, dout the
- * upstream gradient; mask needs bits, cnt, idx, cnt_t and idx_t, all of the
+ * upstream gradient; o_res is NULL or the forward's o_res (bf16 only): with it
+ * Delta = rowsum(dO * (o + o_res)), else rowsum(dO * o); mask needs bits, cnt, idx, cnt_t and idx_t, all of the
  * same mask (the bf16 path walks cnt / idx for dQ and bits / cnt_t for dK and
  * dV; the fp32 path the four lists).  Writes dq, dk, dv [B, H, S, D] in
  * shape->dtype.  The result is deterministic (no atomics). */
 NABLA_API nabla_status nabla_attn_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
-                            const void* o, const void* dout, const float* lse,
+                            const void* o, const void* o_res, const void* dout, const float* lse,
                             const nabla_mask* mask, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 

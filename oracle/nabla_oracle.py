@@ -34,9 +34,6 @@ Readings where the paper is silent (each with its reason):
 * STA window: |dt| <= wT // 2, |dy| <= wH // 2, |dx| <= wW // 2 in tile units,
   truncated at the grid edge (no shifting of the window);
 * the mask is a constant of the backward pass (no gradient through pooling);
-* optionally (o_format="bf16") the backward takes rowsum(dO * O) with O
-  rounded to bfloat16, the output a bf16 forward stores and hands on, instead
-  of the exact O of the textbook gradient;
 * edge patches of a frame whose sides are not multiples of P keep their valid
   tokens, row-major.
 
@@ -260,20 +257,21 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, o_format: str | None = None):
+def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, ds_bound: bool = False):
     """Gradients of masked_attention with the mask held constant: with
     P = softmax(Q K_sel^T / sqrt(D)) per query block,
       dV_sel += P^T dO,  dP = dO V_sel^T,  dS = P * (dP - rowsum(P * dP)),
       dQ = dS K_sel / sqrt(D),  dK_sel += dS^T Q / sqrt(D).
-    rowsum(P * dP) equals rowsum(dO * O).  o_format="bf16" takes that row sum
-    with O rounded to bfloat16 (round to nearest even) first: the output a
-    forward stores in bf16, which is all a backward that is handed O can use;
-    the default is the exact (textbook) gradient.
-    Returns (dQ, dK, dV) fp64 [B, H, S, D]."""
+    rowsum(P * dP) equals rowsum(dO * O).
+    Returns (dQ, dK, dV) fp64 [B, H, S, D].  ds_bound=True also returns
+    (bQ, bK): every gradient entry's sum of term magnitudes through dS,
+    bQ = |dS| |K_sel| / sqrt(D) and bK_sel += |dS|^T |Q| / sqrt(D), the scale
+    of the error that rounding dS before these products can cause."""
     Q, K, V, dO = as_f64(Q), as_f64(K), as_f64(V), as_f64(dO)
     B, H, S, D = Q.shape
     nb = num_blocks(S, N)
     dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    bQ, bK = np.zeros_like(Q), np.zeros_like(K)
     scale = 1.0 / np.sqrt(D)
     for b in range(B):
         for h in range(H):
@@ -288,14 +286,15 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, o_format: s
                 g = dO[b, h, rows]
                 dV[b, h, keys] += P.T @ g
                 dP = g @ V[b, h, keys].T
-                if o_format == "bf16":
-                    O_rows = round_bf16(P @ V[b, h, keys])
-                    delta = (g * O_rows).sum(axis=-1, keepdims=True)
-                else:
-                    delta = (P * dP).sum(axis=-1, keepdims=True)
+                delta = (P * dP).sum(axis=-1, keepdims=True)
                 dS = P * (dP - delta)
                 dQ[b, h, rows] = dS @ K[b, h, keys] * scale
                 dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
+                if ds_bound:
+                    bQ[b, h, rows] = np.abs(dS) @ np.abs(K[b, h, keys]) * scale
+                    bK[b, h, keys] += np.abs(dS).T @ np.abs(Q[b, h, rows]) * scale
+    if ds_bound:
+        return dQ, dK, dV, bQ, bK
     return dQ, dK, dV
 
 

@@ -49,7 +49,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_abi_version(L):
-    assert L.nabla_abi_version() == 1
+    assert L.nabla_abi_version() == 2
 
 
 def test_workspace_size_formula(L):
@@ -108,19 +108,25 @@ def test_build_mask_argument_errors(L):
 def test_attention_argument_errors(L):
     sh, m = shape(), mask_struct()
     fwd = lambda **kw: L.nabla_attn_fwd(ctypes.byref(kw.get("sh", sh)), kw.get("q", FAKE), FAKE, FAKE,
-                                        ctypes.byref(kw.get("m", m)), kw.get("o", FAKE),
+                                        ctypes.byref(kw.get("m", m)), kw.get("o", FAKE), kw.get("o_res", None),
                                         kw.get("lse", FAKE), kw.get("ws", FAKE), kw.get("wsb", 1 << 40), None)
     assert fwd(o=None) == INVALID
+    assert fwd(o_res=FAKE + 8) == INVALID                # misaligned residual
+    assert fwd(o_res=FAKE, sh=shape(dtype=1)) == INVALID  # fp32 has no residual
+    assert b"o_res" in L.nabla_last_error()
     assert fwd(lse=FAKE + 2) == INVALID
     assert fwd(sh=shape(D=32)) == UNSUPPORTED
     assert fwd(wsb=10) == WORKSPACE
-    bwd = lambda **kw: L.nabla_attn_bwd(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+    bwd = lambda **kw: L.nabla_attn_bwd(ctypes.byref(kw.get("sh", sh)), FAKE, FAKE, FAKE, FAKE,
+                                        kw.get("o_res", None), FAKE, FAKE,
                                         ctypes.byref(kw.get("m", m)), FAKE, FAKE, kw.get("dv", FAKE),
                                         FAKE, kw.get("wsb", 1 << 40), None)
     assert bwd() == INVALID                              # forward-only mask: no transposed lists
     assert b"cnt_t" in L.nabla_last_error()
     full = mask_struct(cnt_t=FAKE, idx_t=FAKE)
     assert bwd(m=full, dv=None) == INVALID
+    assert bwd(m=full, o_res=FAKE + 4) == INVALID
+    assert bwd(m=full, o_res=FAKE, sh=shape(dtype=1)) == INVALID
     assert bwd(m=full, wsb=1000) == WORKSPACE
     # the tensor-core dK / dV walks the bitmask columns: bits are required
     assert bwd(m=mask_struct(cnt_t=FAKE, idx_t=FAKE, bits=None)) == INVALID

@@ -121,12 +121,13 @@ def test_fwd_uses_gpu_built_mask_end_to_end():
 
 # ---------------------------------------------------------------- backward
 
-def _bwd_parity(x, M, kind, heads=None):
+def _bwd_parity(x, M, kind, heads=None, residual=False):
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
-    o, lse = nabla.attn_fwd(q, k, v, mask)
+    o_res = torch.empty_like(q) if residual else None
+    o, lse = nabla.attn_fwd(q, k, v, mask, o_res=o_res)
     ws = nabla.workspace(q, want_bwd=True)
-    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws)
+    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws, o_res=o_res)
     torch.cuda.synchronize()
     assert nabla.workspace_status(ws) == 0
     for (b, h) in ([(b, h) for b in range(q.shape[0]) for h in range(q.shape[1])] if heads is None else heads):
@@ -144,11 +145,12 @@ def test_bwd_tiny_fp32():
     _bwd_parity(x, M, "fp32")
 
 
+@pytest.mark.parametrize("residual", [False, True])
 @pytest.mark.parametrize("S,D", [(1000, 128), (414, 64), (130, 128)])
-def test_bwd_small_bf16(S, D):
+def test_bwd_small_bf16(S, D, residual):
     x = synth.make_random_qkv(1, 2, S, D, "bf16", seed=S, with_grad=True)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
-    _bwd_parity(x, M, "bf16")
+    _bwd_parity(x, M, "bf16", residual=residual)
 
 
 @pytest.mark.parametrize("S,D", [(1000, 128), (130, 64)])
@@ -158,11 +160,12 @@ def test_bwd_small_fp32(S, D):
     _bwd_parity(x, M, "fp32")
 
 
-def test_bwd_pretraining_workload_two_heads():
+@pytest.mark.parametrize("residual", [False, True])
+def test_bwd_pretraining_workload_two_heads(residual):
     w = synth.WORKLOADS[4]
     x = synth.make_inputs(w)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], w.thresholds[0])
-    _bwd_parity(x, M, "bf16", heads=[(0, 0), (1, 15)])
+    _bwd_parity(x, M, "bf16", heads=[(0, 0), (1, 15)], residual=residual)
 
 
 @pytest.mark.parametrize("B,H,S,seed", [(1, 2, 1000, 21), (2, 3, 2000, 22), (1, 1, 64, 23)])
@@ -179,7 +182,37 @@ def test_bwd_external_mask_empty_rows_columns_and_odd_lists(B, H, S, seed):
         M[:, :, :, 2] = False           # a key block nobody attends to
         M[:, :, 3, :] = False
         M[:, :, 3, nb - 1] = True       # one kept block: a lone (odd) step, ragged tail keys
-    _bwd_parity(x, M, "bf16")
+    _bwd_parity(x, M, "bf16", residual=True)
+
+
+@pytest.mark.parametrize("S,D", [(1000, 128), (414, 64)])
+def test_forward_residual_carries_o_beyond_bf16(S, D):
+    """Residual mode of the forward: o alone still meets the bf16 output bar,
+    and o + o_res matches the fp64 oracle's O to about 2^-13 relative (P V with
+    P in two bf16 terms; the residual of O rounded to bf16), where bf16 alone
+    is 2^-9.  Rows of a block that keeps nothing get o = o_res = 0."""
+    x = synth.make_random_qkv(1, 2, S, D, "bf16", seed=3 * S + D)
+    M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
+    M[0, 1, 2, :] = False                               # an empty query block
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
+    ws = nabla.workspace(q)
+    o_res = torch.full_like(q, 7.0)
+    o, lse = nabla.attn_fwd(q, k, v, mask, ws=ws, o_res=o_res)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    O, L = orc.masked_attention(x["q"], x["k"], x["v"], M)
+    gu.assert_close(o, O, "bf16", "o in residual mode")
+    full = orc.as_f64(o) + orc.as_f64(o_res)
+    err = np.abs(full - O)
+    assert (err <= 2e-5 + 2.0 ** -13 * np.abs(O)).all(), float((err - 2.0 ** -13 * np.abs(O)).max())
+    assert orc.mean_rel(full, O) < 2e-5
+    assert (orc.as_f64(o_res)[0, 1, 128:192] == 0).all()
+    assert np.abs(lse.cpu().numpy()[np.isfinite(L)] - L[np.isfinite(L)]).max() < 1e-3
+    # the plain forward's o agrees with the residual mode's o to a bf16 ulp
+    o2, _ = nabla.attn_fwd(q, k, v, mask, ws=ws)
+    torch.cuda.synchronize()
+    assert np.abs(orc.as_f64(o2) - orc.as_f64(o)).max() <= 2.0 ** -7 * max(1.0, float(np.abs(O).max()))
 
 
 # ------------------------------------------------------ bounded waits

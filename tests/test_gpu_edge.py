@@ -53,32 +53,39 @@ def test_sta_window_wider_than_the_grid_keeps_everything():
 
 @pytest.mark.parametrize("scale", [2.0, 8.0])
 def test_extreme_logits_backward(scale):
+    """Steep softmax rows (Q and K scaled by 2 and 8): dS = P (dP - Delta)
+    cancels for the dominant key, so Delta = rowsum(dO * O) must come from an
+    O accurate well beyond bf16.  The forward's residual mode supplies it (P
+    enters P V as two bf16 terms and O's rounding residual is written), and the
+    backward takes Delta from o + o_res.  Gradients are held to the usual
+    gradient bar; at scale 8 the elementwise bar also allows what the bf16
+    rounding of the dS operand of the dQ and dK products can cause, 2^-8 times
+    the entry's sum of term magnitudes through dS (|dS| |K| / sqrt(D) for dQ,
+    |dS|^T |Q| / sqrt(D) for dK): with keys of magnitude ~25 that exceeds the
+    flat 2e-2 for any kernel that multiplies dS in bf16 on the tensor cores."""
     x = synth.make_random_qkv(1, 2, 1000, 128, "bf16", seed=31, with_grad=True)
     for n in ("q", "k"):
         x[n] = (x[n].float() * scale).to(torch.bfloat16)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], 0.8)
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     mask = gu.mask_on_gpu(M, tuple(q.shape), q.dtype)
-    o, lse = nabla.attn_fwd(q, k, v, mask)
+    o_res = torch.empty_like(q)
+    o, lse = nabla.attn_fwd(q, k, v, mask, o_res=o_res)
     ws = nabla.workspace(q, want_bwd=True)
-    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws)
+    dq, dk, dv = nabla.attn_bwd(q, k, v, o, do, lse, mask, ws=ws, o_res=o_res)
     torch.cuda.synchronize()
     assert nabla.workspace_status(ws) == 0
-    ref = orc.masked_attention_bwd(x["q"], x["k"], x["v"], x["do"], M)
-    # Steep rows: dS = P (dP - rowsum(dO * O)) cancels for the dominant key.
-    # The forward multiplies V by P in bf16 (a P of 1 - eps becomes 1), so the
-    # O the backward is handed is off by up to 2^-9 |v|, and dS enters the
-    # dQ / dK products in bf16: both reach dQ amplified by the cancellation
-    # (at the configured workloads the usual bar holds; see the other tests).
-    # Bound for this regime: 1 % of the largest gradient, and a mean relative
-    # error of 1e-2 at scale 2 and 2.5e-2 at scale 8, where many rows are
-    # one-hot and their gradients (~1e-11) sit far below the bf16 noise.
-    mean_bar = 1e-2 if scale <= 2.0 else 2.5e-2
-    for got, r, name in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
-        g = orc.as_f64(got)
-        assert np.isfinite(g).all(), name
-        assert np.abs(g - r).max() <= 1e-2 * np.abs(r).max(), (name, np.abs(g - r).max(), np.abs(r).max())
-        assert orc.mean_rel(g, r) <= mean_bar, (name, orc.mean_rel(g, r))
+    dQ, dK, dV, bQ, bK = orc.masked_attention_bwd(x["q"], x["k"], x["v"], x["do"], M, ds_bound=True)
+    if scale <= 2.0:
+        for got, r, name in zip((dq, dk, dv), (dQ, dK, dV), ("dQ", "dK", "dV")):
+            gu.assert_close(got, r, "bf16", f"{name} scale {scale}", grad=True)
+    else:
+        for got, r, bnd, name in zip((dq, dk, dv), (dQ, dK, dV), (bQ, bK, 0.0), ("dQ", "dK", "dV")):
+            g = orc.as_f64(got)
+            assert np.isfinite(g).all(), name
+            excess = np.abs(g - r) - gu.GRAD_REL * np.abs(r) - gu.GRAD_REL * bnd
+            assert excess.max() <= gu.TOL["bf16"]["max_abs"], (name, float(excess.max()))
+            assert orc.mean_rel(g, r) <= gu.TOL["bf16"]["mean_rel"], (name, orc.mean_rel(g, r))
 
 
 def test_extreme_logits_block_mass():

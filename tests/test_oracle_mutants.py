@@ -95,10 +95,11 @@ def _attn_transposed_mask(Q, K, V, M, N=64):
     return _ORIG_ATTN(Q, K, V, np.swapaxes(M, -1, -2), N)
 
 
-def _bwd_no_rowsum(Q, K, V, dO, M, N=64):
+def _bwd_no_rowsum(Q, K, V, dO, M, N=64, ds_bound=False):
     Q, K, V, dO = (orc.as_f64(x) for x in (Q, K, V, dO))
     B, H, S, D = Q.shape
     dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    bQ, bK = np.zeros_like(Q), np.zeros_like(K)
     for b in range(B):
         for h in range(H):
             for i in range(orc.num_blocks(S, N)):
@@ -111,7 +112,9 @@ def _bwd_no_rowsum(Q, K, V, dO, M, N=64):
                 dS = P * (dO[b, h, rows] @ V[b, h, keys].T)
                 dQ[b, h, rows] = dS @ K[b, h, keys] / np.sqrt(D)
                 dK[b, h, keys] += dS.T @ Q[b, h, rows] / np.sqrt(D)
-    return dQ, dK, dV
+                bQ[b, h, rows] = np.abs(dS) @ np.abs(K[b, h, keys]) / np.sqrt(D)
+                bK[b, h, keys] += np.abs(dS).T @ np.abs(Q[b, h, rows]) / np.sqrt(D)
+    return (dQ, dK, dV, bQ, bK) if ds_bound else (dQ, dK, dV)
 
 
 def _fractal_variant(col_major_tokens=False, col_major_patches=False, edges_last=False):

@@ -452,25 +452,25 @@ def test_round_bf16_ties_to_even_and_matches_torch():
     assert np.array_equal(orc.round_bf16(y), ref)
 
 
-def test_backward_with_bf16_output_reduces_to_exact_when_o_is_bf16():
-    # every key carries the same bf16 value row v, so O = v exactly and the
-    # row sum taken with the rounded O equals the exact one
-    rng = np.random.default_rng(4)
+def test_backward_ds_bound_matches_autograd_of_the_logits():
+    """The magnitude sums through dS: dS is the gradient of the loss
+    sum(dO * O) with respect to the scaled logits (masked keys at -inf), which
+    torch autograd gives independently; then bQ = |dS| |K| / sqrt(D) and
+    bK = |dS|^T |Q| / sqrt(D) per (b, h)."""
+    rng = np.random.default_rng(12)
     S, D = 150, 16
-    Q = rng.standard_normal((1, 1, S, D))
-    K = rng.standard_normal((1, 1, S, D))
-    v = orc.round_bf16(rng.standard_normal(D))
-    V = np.broadcast_to(v, (1, 1, S, D)).copy()
-    dO = rng.standard_normal((1, 1, S, D))
+    Q, K, V, dO = (rng.standard_normal((1, 1, S, D)) for _ in range(4))
     nb = orc.num_blocks(S)
     M = rng.random((1, 1, nb, nb)) < 0.6
     M[0, 0, np.arange(nb), np.arange(nb)] = True
-    exact = orc.masked_attention_bwd(Q, K, V, dO, M)
-    rounded = orc.masked_attention_bwd(Q, K, V, dO, M, o_format="bf16")
-    for a, b in zip(exact, rounded):
-        assert np.abs(a - b).max() < 1e-12
-    # with generic values the rounded-O row sum does change the gradient
-    V2 = rng.standard_normal((1, 1, S, D))
-    e2 = orc.masked_attention_bwd(Q, K, V2, dO, M)[0]
-    r2 = orc.masked_attention_bwd(Q, K, V2, dO, M, o_format="bf16")[0]
-    assert np.abs(e2 - r2).max() > 1e-6
+    dQ, dK, dV, bQ, bK = orc.masked_attention_bwd(Q, K, V, dO, M, ds_bound=True)
+    assert np.abs(dQ - orc.masked_attention_bwd(Q, K, V, dO, M)[0]).max() == 0.0
+    tok = np.kron(M[0, 0], np.ones((64, 64), dtype=bool))[:S, :S]
+    lg = torch.tensor(Q[0, 0] @ K[0, 0].T / math.sqrt(D), requires_grad=True)
+    P = torch.softmax(lg.masked_fill(torch.from_numpy(~tok), float("-inf")), dim=-1)
+    (P @ torch.from_numpy(V[0, 0]) * torch.from_numpy(dO[0, 0])).sum().backward()
+    dS = np.abs(lg.grad.numpy())
+    assert np.allclose(bQ[0, 0], dS @ np.abs(K[0, 0]) / math.sqrt(D), rtol=1e-10, atol=1e-12)
+    assert np.allclose(bK[0, 0], dS.T @ np.abs(Q[0, 0]) / math.sqrt(D), rtol=1e-10, atol=1e-12)
+    # the bound dominates the gradient itself (triangle inequality)
+    assert (np.abs(dQ) <= bQ + 1e-12).all() and (np.abs(dK) <= bK + 1e-12).all()
