@@ -181,7 +181,8 @@ static nabla_status build_mask_impl(const nabla_shape* shape, const void* q, con
   float* klo = (float*)(ws + L.klo);
   float* logits = (float*)(ws + L.logits);
   NABLA_TRY(reset_status(workspace, st));
-  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, st), "pooling kernel");
+  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, (int32_t*)workspace + kWsStatus, st),
+             "pooling kernel");
   NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, (int32_t*)workspace + kWsStatus, st),
              "score GEMM kernel");
   NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, topk ? 1.f : thr, sta, out->bits, out->cnt, out->idx,

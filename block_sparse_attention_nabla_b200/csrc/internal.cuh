@@ -92,8 +92,9 @@ nabla_status check_selection(float thr, int32_t topk, const nabla_sta* sta);
 // ---------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 
+// status: the workspace status word (a bounded wait that ran out sets NABLA_ERR_TIMEOUT).
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st);
+                        float* qhi, float* qlo, float* khi, float* klo, int32_t* status, cudaStream_t st);
 cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
                               const float* klo, float* L, int ldl, int32_t* status, cudaStream_t st);
 // topk > 0 selects the fixed-budget rule (the topk largest entries per row)

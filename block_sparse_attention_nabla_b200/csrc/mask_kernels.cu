@@ -2,9 +2,8 @@
 // "∇NABLA: Neighborhood Adaptive Block-Level Attention" (§3.1.2), the STA
 // union of §3.1.3, and the index structures the attention kernels walk.
 //
-//   pool_kernel        block averaging of Q and K (reads Q and K once; the
-//                      HBM-bound part of the builder)
-//   select_kernel      reduced scores Qa Ka^T / sqrt(D), row softmax, CDF
+//   select_kernel      row softmax of the reduced scores Qa Ka^T / sqrt(D)
+//                      (pooling: pool.cu; scores: score_tc.cu), CDF
 //                      binarisation, STA OR, bitmask + compact index lists
 //   lists_kernel       bitmask -> compact index lists (external masks)
 //   transpose_kernel   per key block, the query blocks that attend to it
@@ -19,31 +18,6 @@ namespace nabla {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ void add_chunk(const uint4& u, float (&acc)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __bfloat1622float2(h[e]);
-    acc[2 * e] += f.x;
-    acc[2 * e + 1] += f.y;
-  }
-}
-
-__device__ __forceinline__ void add_chunk(const uint4& u, float (&acc)[4]) {
-  acc[0] += __uint_as_float(u.x);
-  acc[1] += __uint_as_float(u.y);
-  acc[2] += __uint_as_float(u.z);
-  acc[3] += __uint_as_float(u.w);
-}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -67,78 +41,6 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
-}
-
-// ------------------------------------------------------------------ pooling
-// One warp per 64-token block of Q or K, no CTA-wide barriers: each lane owns
-// one 16-byte column chunk and sums its rows in fp64 from 16-byte loads, eight
-// loads in flight per lane; lanes that hold the same chunk for different rows
-// are combined by shuffles.  The means are written in fp64 (the selection
-// ranks near-equal entries by fp64 logits) and as a pair of fp32 values
-// hi + lo with hi the nearest tf32 value (operands of the tensor-core score
-// GEMM).  The tail block divides by its number of valid tokens.
-template <typename T, int D>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                   double* __restrict__ qa, double* __restrict__ ka,
-                                                   float* __restrict__ qhi, float* __restrict__ qlo,
-                                                   float* __restrict__ khi, float* __restrict__ klo,
-                                                   int S, int nb, long long per_tensor) {
-  constexpr int VE = 16 / sizeof(T);  // elements per 16-byte chunk
-  constexpr int CH = D / VE;          // chunks per row (8, 16 or 32)
-  constexpr int RPI = 32 / CH;        // rows covered by one warp-wide load
-  constexpr int NL = kBlock / RPI;    // loads per lane for a full block
-  constexpr int UNR = NL < 8 ? NL : 8;
-  const int lane = threadIdx.x & 31;
-  const int c = lane % CH, r0 = lane / CH;
-  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); item < 2 * per_tensor;
-       item += nwarps) {
-    const bool isk = item >= per_tensor;
-    const long long it = isk ? item - per_tensor : item;  // (b * H + h) * nb + i
-    const long long bh = it / nb;
-    const int i = (int)(it - bh * nb);
-    const T* src = (isk ? k : q) + (bh * S + (long long)i * kBlock) * D + c * VE;
-    const int valid = min(kBlock, S - i * kBlock);
-    double acc[VE];
-#pragma unroll
-    for (int e = 0; e < VE; ++e) acc[e] = 0.0;
-#pragma unroll
-    for (int p0 = 0; p0 < NL; p0 += UNR) {
-      uint4 v[UNR];
-#pragma unroll
-      for (int p = 0; p < UNR; ++p) {
-        const int r = r0 + (p0 + p) * RPI;
-        v[p] = r < valid ? ld_stream(src + (long long)r * D) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int p = 0; p < UNR; ++p) {
-        float f[VE];
-#pragma unroll
-        for (int e = 0; e < VE; ++e) f[e] = 0.f;
-        add_chunk(v[p], f);
-#pragma unroll
-        for (int e = 0; e < VE; ++e) acc[e] += (double)f[e];
-      }
-    }
-#pragma unroll
-    for (int off = CH; off < 32; off <<= 1)
-#pragma unroll
-      for (int e = 0; e < VE; ++e) acc[e] += __shfl_xor_sync(kFull, acc[e], off);
-    if (lane < CH) {
-      double* dst = (isk ? ka : qa) + it * D + c * VE;
-      float* dhi = (isk ? khi : qhi) + it * D + c * VE;
-      float* dlo = (isk ? klo : qlo) + it * D + c * VE;
-#pragma unroll
-      for (int e = 0; e < VE; ++e) {
-        const double mean = acc[e] / (double)valid;
-        const float f = (float)mean;
-        const float h = sm100::to_tf32(f);
-        dst[e] = mean;
-        dhi[e] = h;
-        dlo[e] = f - h;
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------------ select
@@ -612,52 +514,7 @@ cudaError_t set_smem(Kern k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-int num_sms();
-
-// Grid of at most `want` CTAs that all fit on the GPU at once.
-template <typename Kern>
-int resident_grid(Kern kern, int threads, long long want) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
-    per_sm = 1;
-  return (int)std::min<long long>(want, (long long)num_sms() * per_sm);
-}
-
-int num_sms() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
-
-
 }  // namespace
-
-cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        float* qhi, float* qlo, float* khi, float* klo, cudaStream_t st) {
-  const long long per = d.BH() * d.nb;
-  const long long warps = 2 * per;
-  // One wave of resident CTAs walking the blocks (grid-stride), instead of
-  // more CTAs than fit at once and a partial last wave.
-  auto launch = [&](auto kern, const auto* qq, const auto* kk) {
-    const int grid = resident_grid(kern, 256, (warps + 7) / 8);
-    kern<<<grid, 256, 0, st>>>(qq, kk, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, per);
-  };
-  if (d.dtype == NABLA_BF16) {
-    const auto* qq = (const __nv_bfloat16*)q;
-    const auto* kk = (const __nv_bfloat16*)k;
-    if (d.D == 128) launch(pool_kernel<__nv_bfloat16, 128>, qq, kk);
-    else launch(pool_kernel<__nv_bfloat16, 64>, qq, kk);
-  } else {
-    if (d.D == 128) launch(pool_kernel<float, 128>, (const float*)q, (const float*)k);
-    else launch(pool_kernel<float, 64>, (const float*)q, (const float*)k);
-  }
-  return cudaGetLastError();
-}
 
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,

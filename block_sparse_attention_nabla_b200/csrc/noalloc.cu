@@ -13,7 +13,7 @@
 // loads modules lazily), which commits the 32 MiB on that device; callers make
 // that first call, or nabla_build_mask_noalloc_status, at start-up, before they
 // reserve the rest of the device memory.  The status word at the start of the
-// array reports a bounded wait that ran out in the score GEMM, and
+// array reports a bounded wait that ran out in the pooling or the score GEMM, and
 // nabla_build_mask_noalloc_status reads it back.  Every call shares the array
 // and it keeps the last call's contents, so calls whose work overlaps on the
 // GPU (different streams, or different host threads on one device) race on
@@ -101,7 +101,8 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);  // the status word starts at zero
   if (e == cudaSuccess)
     e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), (float*)(ws + L.qhi),
-                    (float*)(ws + L.qlo), (float*)(ws + L.khi), (float*)(ws + L.klo), st);
+                    (float*)(ws + L.qlo), (float*)(ws + L.khi), (float*)(ws + L.klo), (int32_t*)ws + kWsStatus,
+                    st);
   if (e == cudaSuccess)
     e = launch_score_gemm(d, (const float*)(ws + L.qhi), (const float*)(ws + L.qlo),
                           (const float*)(ws + L.khi), (const float*)(ws + L.klo), (float*)(ws + L.logits),
