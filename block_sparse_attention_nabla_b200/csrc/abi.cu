@@ -180,13 +180,14 @@ static nabla_status build_mask_impl(const nabla_shape* shape, const void* q, con
   float* khi = (float*)(ws + L.khi);
   float* klo = (float*)(ws + L.klo);
   float* logits = (float*)(ws + L.logits);
+  int32_t* status = (int32_t*)workspace + kWsStatus;
+  int32_t* counters = (int32_t*)(ws + L.counters);
   NABLA_TRY(reset_status(workspace, st));
-  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, (int32_t*)workspace + kWsStatus, st),
-             "pooling kernel");
-  NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, (int32_t*)workspace + kWsStatus, st),
-             "score GEMM kernel");
+  NABLA_CUDA(cudaMemsetAsync(counters, 0, (size_t)d.BH() * 2 * sizeof(int32_t), st), "clear builder counters");
+  NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, counters, status, st), "pooling kernel");
+  NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, counters, status, st), "score GEMM kernel");
   NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, topk ? 1.f : thr, sta, out->bits, out->cnt, out->idx,
-                           st, topk),
+                           counters, status, st, topk),
              "select kernel");
   return emit_derived(d, out->bits, out, st);
 }

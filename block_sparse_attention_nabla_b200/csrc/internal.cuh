@@ -28,6 +28,8 @@ inline Dims make_dims(const nabla_shape& s) {
 }
 
 // Workspace layout: a 256-byte header (status word, scheduler counters), the
+// per-(b, h) progress counters through which the builder's kernels hand heads
+// on to each other, the
 // pooled Qa / Ka in fp64 and as tf32 hi / lo pairs ([B, H, nb, D] each), the
 // reduced logits L (fp32 [B, H, nb, ldl], ldl = nb rounded up to 4) and, for
 // the backward, the per-row Delta = rowsum(dO * O) (fp32 [B, H, S]) and the
@@ -35,6 +37,7 @@ inline Dims make_dims(const nabla_shape& s) {
 // [B, H, nb * 64] each).
 struct WsLayout {
   size_t header = 0;
+  size_t counters = 0;  // int32 [B * H][2]: pooled items, score tiles (the builder's hand-off), zeroed per call
   size_t qa = 0, ka = 0, qhi = 0, qlo = 0, khi = 0, klo = 0, logits = 0, delta = 0, lse2p = 0, deltap = 0;
   int ldl = 0;
   size_t total = 0;
@@ -45,6 +48,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline WsLayout ws_layout(const Dims& d, bool want_bwd) {
   WsLayout w;
   size_t off = 256;
+  w.counters = off; off = align256(off + (size_t)d.BH() * 2 * sizeof(int32_t));
   size_t pooled = (size_t)d.BH() * d.nb * d.D * sizeof(double);
   w.qa = off; off = align256(off + pooled);
   w.ka = off; off = align256(off + pooled);
@@ -92,16 +96,29 @@ nabla_status check_selection(float thr, int32_t topk, const nabla_sta* sta);
 // ---------------------------------------------------------------- launchers
 // Each returns the cudaError_t of its launches (cudaSuccess if all enqueued).
 
-// status: the workspace status word (a bounded wait that ran out sets NABLA_ERR_TIMEOUT).
+// The mask builder is a chain of three kernels launched back to back on one
+// stream: pooling, the score GEMM and the selection.  Each of the last two is
+// launched with programmatic stream serialization, so it starts while its
+// predecessor still runs, and takes a head (b, h) only once the predecessor
+// has counted all of that head's work done in `counters` (int32 [B * H][2],
+// zeroed before the pooling: [0] pooled items, [1] score tiles).  status: the
+// workspace status word (a bounded wait that ran out sets NABLA_ERR_TIMEOUT).
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
-                        float* qhi, float* qlo, float* khi, float* klo, int32_t* status, cudaStream_t st);
+                        float* qhi, float* qlo, float* khi, float* klo, int32_t* counters, int32_t* status,
+                        cudaStream_t st);
 cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
-                              const float* klo, float* L, int ldl, int32_t* status, cudaStream_t st);
+                              const float* klo, float* L, int ldl, int32_t* counters, int32_t* status,
+                              cudaStream_t st);
 // topk > 0 selects the fixed-budget rule (the topk largest entries per row)
 // instead of the CDF rule with thr.
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          cudaStream_t st, int topk = 0);
+                          const int32_t* counters, int32_t* status, cudaStream_t st, int topk = 0);
+// Targets of the counters: every pooled item is counted once by each of the
+// pooling kernel's D / 32 consumer warps, every score tile once by each of the
+// GEMM's four epilogue warps.
+inline int pool_target(const Dims& d) { return 2 * d.nb * (d.D / 32); }
+inline int score_target(const Dims& d) { const int T = (d.nb + 127) / 128; return 4 * T * T; }
 // STA-only bitmask (every sample and head): the sliding-tile window alone.
 cudaError_t launch_sta_bits(const Dims& d, const nabla_sta& sta, uint32_t* bits, cudaStream_t st);
 cudaError_t launch_lists_from_bits(const Dims& d, const uint32_t* bits, int32_t* cnt,

@@ -328,11 +328,17 @@ __device__ __forceinline__ void select_row(const SelectCtx& c, float* Lr, int ro
   if (lane == 0) *cntp = running;
 }
 
+// Launched behind the score GEMM with programmatic stream serialization: the
+// warp of a row starts once the GEMM has counted all tiles of the row's head
+// (and the pooling all its blocks; a bounded wait that runs out records
+// NABLA_ERR_TIMEOUT and the row is built from whatever is there).
 template <int D, int NPL>
 __global__ void __launch_bounds__(256) select_rows_kernel(
     const float* __restrict__ L, int ldl, const double* __restrict__ qa, const double* __restrict__ ka,
     long long rows, int nb, int W, float thr, int topk, const int32_t* __restrict__ coords, int hT, int hH,
-    int hW, uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx) {
+    int hW, uint32_t* __restrict__ bits, int32_t* __restrict__ cnt, int32_t* __restrict__ idx,
+    const int32_t* __restrict__ counters, int pool_goal, int score_goal, int32_t* __restrict__ status,
+    uint64_t limit_ns) {
   __shared__ int cand_j[8][kMaxCand];
   __shared__ float cand_e[8][kMaxCand];
   __shared__ double cand_lg[8][kMaxCand];
@@ -340,6 +346,12 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   const long long grow = (long long)blockIdx.x * 8 + warp;  // (b * H + h) * nb + i
   if (grow >= rows) return;
   const long long bh = grow / nb;
+  if (lane == 0) {
+    const bool ok = sm100::wait_counter(counters + 2 * bh + 1, score_goal, nullptr, limit_ns) &&
+                    sm100::wait_counter(counters + 2 * bh, pool_goal, nullptr, limit_ns);
+    if (!ok) atomicCAS(status, 0, (int32_t)NABLA_ERR_TIMEOUT);
+  }
+  __syncwarp();
   const int row = (int)(grow - bh * nb);
   SelectCtx ctx{qa + bh * nb * D, ka + bh * nb * D, nb, W, thr, topk, coords, hT, hH, hW, cand_j, cand_e, cand_lg};
   float* Lr = const_cast<float*>(L) + grow * ldl;
@@ -349,9 +361,11 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
 }
 
 template <int D>
-void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl, const double* qa,
-                        const double* ka, long long rows, int nb, int W, float thr, int topk, const int32_t* coords,
-                        int hT, int hH, int hW, uint32_t* bits, int32_t* cnt, int32_t* idx) {
+cudaError_t launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl, const double* qa,
+                               const double* ka, long long rows, int nb, int W, float thr, int topk,
+                               const int32_t* coords, int hT, int hH, int hW, uint32_t* bits, int32_t* cnt,
+                               int32_t* idx, const int32_t* counters, int pool_goal, int score_goal,
+                               int32_t* status) {
   // registers per lane hold ceil(nb / 32) values, rounded up to a few sizes
   auto k = W <= 8 ? select_rows_kernel<D, 8>
          : W <= 16 ? select_rows_kernel<D, 16>
@@ -359,7 +373,24 @@ void launch_select_rows(unsigned grid, cudaStream_t st, const float* L, int ldl,
          : W <= 40 ? select_rows_kernel<D, 40>
          : W <= 64 ? select_rows_kernel<D, 64>
                    : select_rows_kernel<D, 0>;
-  k<<<grid, 256, 0, st>>>(L, ldl, qa, ka, rows, nb, W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  {
+    // the SM keeps its largest shared-memory configuration, so the builder's
+    // kernels can be resident side by side
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+  }
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, L, ldl, qa, ka, rows, nb, W, thr, topk, coords, hT, hH, hW, bits, cnt, idx,
+                            counters, pool_goal, score_goal, status, wait_limit_ns());
 }
 
 // ----------------------------------------------------------- STA-only masks
@@ -518,17 +549,17 @@ cudaError_t set_smem(Kern k, size_t bytes) {
 
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          cudaStream_t st, int topk) {
+                          const int32_t* counters, int32_t* status, cudaStream_t st, int topk) {
   const long long rows = d.BH() * d.nb;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   const bool use_sta = sta && sta->block_coords;
   const int32_t* coords = use_sta ? sta->block_coords : nullptr;
   const int hT = use_sta ? sta->wT / 2 : 0, hH = use_sta ? sta->wH / 2 : 0, hW = use_sta ? sta->wW / 2 : 0;
   if (d.D == 128)
-    launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
-  else
-    launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt, idx);
-  return cudaGetLastError();
+    return launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits,
+                                   cnt, idx, counters, pool_target(d), score_target(d), status);
+  return launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt,
+                                idx, counters, pool_target(d), score_target(d), status);
 }
 
 cudaError_t launch_sta_bits(const Dims& d, const nabla_sta& sta, uint32_t* bits, cudaStream_t st) {

@@ -88,7 +88,7 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (L.total > kNoAllocScratchBytes) {
     record_error(NABLA_ERR_UNSUPPORTED,
                  "this shape needs %zu bytes of scratch; the static scratch of "
-                 "nabla_build_mask_noalloc holds %zu (B * H * nb * (32 D + 4 nb) bytes, nb = ceil(S / 64), must fit); "
+                 "nabla_build_mask_noalloc holds %zu (B * H * (nb * (32 D + 4 nb) + 8) bytes, nb = ceil(S / 64), plus about 2 KB, must fit); "
                  "use nabla_build_mask with a workspace",
                  L.total, kNoAllocScratchBytes);
     return NABLA_ERR_UNSUPPORTED;
@@ -98,18 +98,20 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (st0 != NABLA_OK) return st0;
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)scratch;
+  int32_t* status = (int32_t*)ws + kWsStatus;
+  int32_t* counters = (int32_t*)(ws + L.counters);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);  // the status word starts at zero
+  if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, (size_t)d.BH() * 2 * sizeof(int32_t), st);
   if (e == cudaSuccess)
     e = launch_pool(d, q, k, (double*)(ws + L.qa), (double*)(ws + L.ka), (float*)(ws + L.qhi),
-                    (float*)(ws + L.qlo), (float*)(ws + L.khi), (float*)(ws + L.klo), (int32_t*)ws + kWsStatus,
-                    st);
+                    (float*)(ws + L.qlo), (float*)(ws + L.khi), (float*)(ws + L.klo), counters, status, st);
   if (e == cudaSuccess)
     e = launch_score_gemm(d, (const float*)(ws + L.qhi), (const float*)(ws + L.qlo),
                           (const float*)(ws + L.khi), (const float*)(ws + L.klo), (float*)(ws + L.logits),
-                          L.ldl, (int32_t*)ws + kWsStatus, st);
+                          L.ldl, counters, status, st);
   if (e == cudaSuccess)
     e = launch_select(d, (const float*)(ws + L.logits), L.ldl, (const double*)(ws + L.qa),
-                      (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, st);
+                      (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, counters, status, st);
   if (e == cudaSuccess && out->cnt_t) e = launch_transpose_lists(d, out->bits, out->cnt_t, out->idx_t, st);
   if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);
   if (e != cudaSuccess) {

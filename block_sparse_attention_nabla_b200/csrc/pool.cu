@@ -12,10 +12,16 @@
 // what a warp-per-block loop with register loads could not sustain.
 //
 // Items are (b, h, tensor, block) in head-major order, dealt round-robin to a
-// persistent grid.  Outputs per block: the mean in fp64 (the selection ranks
-// near-equal entries by fp64 logits) and as a pair of fp32 values hi + lo with
-// hi the nearest tf32 value (operands of the tensor-core score GEMM).  A
-// partial last block divides by its number of valid tokens.
+// persistent grid of all the CTAs that fit (three per SM, each with two
+// consumer groups taking alternate ring slots).  Outputs per block: the mean
+// in fp64 (the selection ranks near-equal entries by fp64 logits) and as a
+// pair of fp32 values hi + lo with hi the nearest tf32 value (operands of the
+// tensor-core score GEMM).  A partial last block divides by its number of
+// valid tokens.  Each consumer warp adds, once per head, the number of that
+// head's items it has written to the head's counter (a release).  The score
+// GEMM is launched behind this kernel with programmatic stream serialization:
+// its CTAs take SMs as this kernel's CTAs leave them and wait on the counter
+// of each head before they read its pooled vectors.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -27,6 +33,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kPoolStages = 4;
+// Consumer groups: group g reduces the items it = g, g + kGroups, ... of its
+// CTA (stage it % kPoolStages), so several blocks are summed at once and the
+// conversions and fp64 adds of one block hide the latency of another's.
+constexpr int kGroups = 2;
 constexpr uint64_t kPoolDrainNs = 1000000000ull;
 
 template <typename T, int D>
@@ -35,7 +45,7 @@ struct PoolLayout {
   static constexpr uint32_t bar_off = kPoolStages * kStageBytes;   // full[S], empty[S]
   static constexpr uint32_t misc_off = bar_off + 2 * kPoolStages * 8;
   static constexpr uint32_t bytes = misc_off + 16;
-  static constexpr int kThreads = 32 + D;                           // producer warp + one thread per column
+  static constexpr int kThreads = 32 + kGroups * D;                 // producer warp + groups of one thread per column
 };
 
 __device__ __forceinline__ float to_float(float x) { return x; }
@@ -46,7 +56,7 @@ __global__ void __launch_bounds__(PoolLayout<T, D>::kThreads)
     pool_bulk_kernel(const T* __restrict__ q, const T* __restrict__ k, double* __restrict__ qa,
                      double* __restrict__ ka, float* __restrict__ qhi, float* __restrict__ qlo,
                      float* __restrict__ khi, float* __restrict__ klo, int S, int nb, long long n_items,
-                     int32_t* __restrict__ status, uint64_t limit_ns) {
+                     int32_t* __restrict__ counters, int32_t* __restrict__ status, uint64_t limit_ns) {
   using L = PoolLayout<T, D>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = (uint64_t*)(smem + L::bar_off);
@@ -56,12 +66,13 @@ __global__ void __launch_bounds__(PoolLayout<T, D>::kThreads)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPoolStages; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, D);  // every consumer thread releases the slot
+      mbar_init(empty + s, D);  // every thread of the group that reads it releases the slot
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_launch_dependents();
   const long long per_bh = 2ll * nb;  // Q blocks then K blocks of one (b, h)
 
   if (warp == 0) {
@@ -86,13 +97,31 @@ __global__ void __launch_bounds__(PoolLayout<T, D>::kThreads)
         mbar_wait(full + (j % kPoolStages), (uint32_t)((j / kPoolStages) & 1), nullptr, kPoolDrainNs);
     }
   } else {
-    const int col = threadIdx.x - 32;
-    long long it = 0;
-    for (long long item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+    const int ct = threadIdx.x - 32;
+    const int grp = ct / D, col = ct - grp * D;
+    long long it = grp;
+    long long cur_bh = -1;
+    int done_items = 0;  // items of head cur_bh this warp has written
+    // publish this warp's finished items of head cur_bh: every lane's stores
+    // are ordered before lane 0's release
+    auto publish = [&]() {
+      if (done_items > 0) {
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(counters + 2 * cur_bh, done_items);
+      }
+      done_items = 0;
+    };
+    for (long long item = blockIdx.x + (long long)grp * gridDim.x; item < n_items;
+         item += (long long)kGroups * gridDim.x, it += kGroups) {
       const uint32_t s = (uint32_t)(it % kPoolStages);
       const bool ok = mbar_wait(full + s, (uint32_t)((it / kPoolStages) & 1), abort_flag, limit_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       const long long bh = item / per_bh;
+      if (bh != cur_bh) {
+        publish();
+        cur_bh = bh;
+      }
       const int r = (int)(item - bh * per_bh);
       const bool isk = r >= nb;
       const int i = isk ? r - nb : r;
@@ -116,7 +145,9 @@ __global__ void __launch_bounds__(PoolLayout<T, D>::kThreads)
       (isk ? ka : qa)[o] = mean;
       (isk ? khi : qhi)[o] = h;
       (isk ? klo : qlo)[o] = f - h;
+      ++done_items;
     }
+    publish();
   }
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(status, 0, (int32_t)NABLA_ERR_TIMEOUT);
@@ -124,36 +155,41 @@ __global__ void __launch_bounds__(PoolLayout<T, D>::kThreads)
 
 template <typename T, int D>
 cudaError_t run_pool(const Dims& d, const T* q, const T* k, double* qa, double* ka, float* qhi, float* qlo,
-                     float* khi, float* klo, int32_t* status, cudaStream_t st) {
+                     float* khi, float* klo, int32_t* counters, int32_t* status, cudaStream_t st) {
   using L = PoolLayout<T, D>;
   auto kern = pool_bulk_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
   if (e != cudaSuccess) return e;
+  // the largest shared-memory configuration, so that the builder's kernels fit side by side
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  // all the CTAs that fit at once: the pooling needs that many blocks in
+  // flight to stream Q and K at the HBM rate
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, L::kThreads, L::bytes) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   const long long n_items = 2 * d.BH() * d.nb;
   const int grid = (int)std::min<long long>(n_items, (long long)sm_count() * per_sm);
-  kern<<<grid, L::kThreads, L::bytes, st>>>(q, k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, n_items, status,
-                                            wait_limit_ns());
+  kern<<<grid, L::kThreads, L::bytes, st>>>(q, k, qa, ka, qhi, qlo, khi, klo, d.S, d.nb, n_items, counters,
+                                            status, wait_limit_ns());
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka, float* qhi,
-                        float* qlo, float* khi, float* klo, int32_t* status, cudaStream_t st) {
+                        float* qlo, float* khi, float* klo, int32_t* counters, int32_t* status, cudaStream_t st) {
   if (d.dtype == NABLA_BF16) {
     const auto* qq = (const __nv_bfloat16*)q;
     const auto* kk = (const __nv_bfloat16*)k;
-    if (d.D == 128) return run_pool<__nv_bfloat16, 128>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, status, st);
-    return run_pool<__nv_bfloat16, 64>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, status, st);
+    if (d.D == 128) return run_pool<__nv_bfloat16, 128>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, counters, status, st);
+    return run_pool<__nv_bfloat16, 64>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, counters, status, st);
   }
   const auto* qq = (const float*)q;
   const auto* kk = (const float*)k;
-  if (d.D == 128) return run_pool<float, 128>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, status, st);
-  return run_pool<float, 64>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, status, st);
+  if (d.D == 128) return run_pool<float, 128>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, counters, status, st);
+  return run_pool<float, 64>(d, qq, kk, qa, ka, qhi, qlo, khi, klo, counters, status, st);
 }
 
 }  // namespace nabla

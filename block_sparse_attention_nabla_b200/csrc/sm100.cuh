@@ -69,6 +69,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return true;
 }
 
+// ------------------------------------------- grid-level hand-off (PDL chain)
+// Lets the kernel launched after this one on the stream with programmatic
+// stream serialization start now (it synchronises through counters instead).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Orders this thread's earlier (generic-proxy) observations of global memory
+// before its later async-proxy (TMA) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded wait until *ctr >= target (another kernel's progress counter).
+// Returns false once limit_ns nanoseconds pass, or at once if *abort is set.
+__device__ __forceinline__ bool wait_counter(const int32_t* ctr, int target, volatile int* abort,
+                                             uint64_t limit_ns) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_gpu(ctr) < target) {
+    if (abort && *abort) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      if (abort) *abort = 1;
+      return false;
+    }
+    __nanosleep(256);
+  }
+  return true;
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

@@ -150,7 +150,7 @@ NABLA_API nabla_status nabla_build_mask_topk(const nabla_shape* shape, const voi
  *   builder's scratch (status word, pooled Qa / Ka, reduced logits) lives in a
  *   32 MiB static device array inside the library, held by every GPU that
  *   loads it until the process exits.  Shapes whose scratch exceeds it
- *   (B * H * nb * (32 D + 4 nb) bytes plus about 2 KB must fit in 32 MiB,
+ *   (B * H * (nb * (32 D + 4 nb) + 8) bytes plus about 2 KB must fit in 32 MiB,
  *   nb = ceil(S / 64)) are rejected with
  *   NABLA_ERR_UNSUPPORTED and a message naming both sizes.
  *   The first call on a device looks up the array's device address with that

@@ -23,6 +23,8 @@ Models:
   earlier MMAs are done, so each issuer is an in-order engine), the
   elementwise group and its epilogue, TMA copies landing at any time.
 
+* ``score_gemm`` -- score_tc.cu: operand stage ring, two TMEM accumulators
+  handed between the issuer and the epilogue.
 * ``fwd_pipeline`` -- attn_fwd_tc.cu after the unit ring: Q / K producer, V
   producer, the MMA issuer, the softmax group with its O rescale and
   epilogue.  Units without tiles do not signal O (mutation
@@ -456,3 +458,90 @@ def fwd_pipeline(units: list, seed: int, KS: int = 3, VS: int = 2, mutation: str
 
     roles = {"qk_producer": qk_producer(), "v_producer": v_producer(), "mma": mma(), "softmax": softmax()}
     _run(roles, bars, engines, execute, rnd)
+
+
+def score_gemm(n_tiles: int, seed: int, S: int = 2, n_sub: int = 4, mutation: str | None = None) -> None:
+    """score_tc.cu: the producer streams n_sub operand sub-chunks per tile
+    through S stages (full / empty), the issuer accumulates each tile into one
+    of two TMEM accumulators (acc_full after its last sub-chunk; before reusing
+    an accumulator it waits acc_empty of the tile two back), and the epilogue
+    drains them in tile order and releases each one once read.  Mutations:
+    "no_stage_wait" (the producer refills a stage without waiting empty),
+    "no_acc_wait" (the issuer reuses an accumulator without waiting acc_empty),
+    "early_release" (the epilogue releases an accumulator before reading it)."""
+    rnd = random.Random(seed)
+    bars = {}
+    for s in range(S):
+        bars[f"full{s}"] = _Bar(1)
+        bars[f"empty{s}"] = _Bar(1)
+    for b in range(2):
+        bars[f"acc_full{b}"] = _Bar(1)
+        bars[f"acc_empty{b}"] = _Bar(1)
+    bars["tick"] = _Bar(1)
+    st = {"stage": [None] * S, "acc": [None, None], "chunks": [0, 0], "reading": [False, False], "drained": []}
+    engines = {"tma": [], "mma": []}
+
+    def producer():
+        g = 0
+        for t in range(n_tiles):
+            for s in range(n_sub):
+                k, use = g % S, g // S
+                if use > 0 and mutation != "no_stage_wait":
+                    yield ("wait", f"empty{k}", use - 1)
+                engines["tma"].append(("load", k, (t, s)))
+                g += 1
+
+    def issuer():
+        g = 0
+        for lt in range(n_tiles):
+            ab = lt & 1
+            if lt >= 2 and mutation != "no_acc_wait":
+                yield ("wait", f"acc_empty{ab}", (lt >> 1) - 1)
+            for s in range(n_sub):
+                k = g % S
+                yield ("wait", f"full{k}", g // S)
+                engines["mma"].append(("mma", k, (lt, s), ab))
+                engines["mma"].append(("commit", f"empty{k}"))
+                g += 1
+            engines["mma"].append(("commit", f"acc_full{ab}"))
+
+    def epilogue():
+        for lt in range(n_tiles):
+            ab = lt & 1
+            yield ("wait", f"acc_full{ab}", lt >> 1)
+            if mutation == "early_release":
+                yield ("arrive", f"acc_empty{ab}")
+            if st["acc"][ab] != lt or st["chunks"][ab] != n_sub:
+                raise ProtocolError(f"epilogue of tile {lt} found {st['acc'][ab]} with {st['chunks'][ab]} chunks")
+            st["reading"][ab] = True
+            yield ("arrive", "tick")                  # the TMEM loads take a while
+            if st["acc"][ab] != lt or st["chunks"][ab] != n_sub:
+                raise ProtocolError(f"accumulator {ab} overwritten while tile {lt} was read")
+            st["reading"][ab] = False
+            st["drained"].append(lt)
+            if mutation != "early_release":
+                yield ("arrive", f"acc_empty{ab}")
+
+    def execute(e, op):
+        if op[0] == "load":
+            st["stage"][op[1]] = op[2]
+            bars[f"full{op[1]}"].arrive()
+        elif op[0] == "mma":
+            _, k, want, ab = op
+            if st["stage"][k] != want:
+                raise ProtocolError(f"MMA of {want} read stage {k} holding {st['stage'][k]}")
+            lt, s = want
+            if s == 0:
+                if st["reading"][ab]:
+                    raise ProtocolError(f"tile {lt} started accumulator {ab} during the previous tile's read")
+                st["acc"][ab], st["chunks"][ab] = lt, 1
+            else:
+                if st["acc"][ab] != lt or st["chunks"][ab] != s:
+                    raise ProtocolError(f"tile {lt} sub-chunk {s} found accumulator {ab} = {st['acc'][ab]}")
+                st["chunks"][ab] += 1
+        else:
+            bars[op[1]].arrive()
+
+    _run({"producer": producer(), "issuer": issuer(), "epilogue": epilogue()}, bars, engines, execute, rnd)
+    if st["drained"] != list(range(n_tiles)):
+        raise ProtocolError(f"tiles drained {st['drained']}")

@@ -59,7 +59,8 @@ def test_workspace_size_formula(L):
         nb = -(-S // 64)
         pooled = align(B * H * nb * D * 8)
         ldl = (nb + 3) // 4 * 4
-        fwd = 256 + 2 * pooled + 4 * align(B * H * nb * D * 4) + align(B * H * nb * ldl * 4)
+        counters = align(B * H * 2 * 4)      # per-(b, h) hand-off counters of the builder's kernels
+        fwd = 256 + counters + 2 * pooled + 4 * align(B * H * nb * D * 4) + align(B * H * nb * ldl * 4)
         assert L.nabla_workspace_size(ctypes.byref(shape(B, H, S, D)), 0) == fwd
         # backward: Delta [B, H, S] and the block-padded LSE2 / Delta [B, H, nb * 64]
         bwd = align(B * H * S * 4) + 2 * align(B * H * nb * 64 * 4)

@@ -69,3 +69,24 @@ def test_forward_pipeline_protocol_holds():
 @pytest.mark.parametrize("mutation", ["no_q_wait", "no_v_wait", "no_k_wait", "rescale_lag", "o_final_for_empty_units"])
 def test_forward_pipeline_mutants_are_caught(mutation):
     assert _fwd_traces(300, mutation) > 0
+
+
+def _gemm_traces(n, S, mutation=None):
+    rng = random.Random(5)
+    failures = 0
+    for seed in range(n):
+        try:
+            pm.score_gemm(rng.randint(0, 9), seed, S=S, n_sub=rng.choice([2, 4]), mutation=mutation)
+        except pm.ProtocolError:
+            failures += 1
+    return failures
+
+
+@pytest.mark.parametrize("S", [2, 3])
+def test_score_gemm_protocol_holds(S):
+    assert _gemm_traces(1500, S) == 0
+
+
+@pytest.mark.parametrize("mutation", ["no_stage_wait", "no_acc_wait", "early_release"])
+def test_score_gemm_mutants_are_caught(mutation):
+    assert _gemm_traces(600, 2, mutation) > 0
