@@ -12,16 +12,15 @@
 // what a warp-per-block loop with register loads could not sustain.
 //
 // Items are (b, h, tensor, block) in head-major order, dealt round-robin to a
-// persistent grid of all the CTAs that fit (three per SM, each with two
-// consumer groups taking alternate ring slots).  Outputs per block: the mean
-// in fp64 (the selection ranks near-equal entries by fp64 logits) and as a
-// pair of fp32 values hi + lo with hi the nearest tf32 value (operands of the
-// tensor-core score GEMM).  A partial last block divides by its number of
-// valid tokens.  Each consumer warp adds, once per head, the number of that
-// head's items it has written to the head's counter (a release).  The score
-// GEMM is launched behind this kernel with programmatic stream serialization:
-// its CTAs take SMs as this kernel's CTAs leave them and wait on the counter
-// of each head before they read its pooled vectors.
+// persistent grid of all the CTAs that fit (three per SM).  Outputs per
+// block: the mean in fp64 (the selection ranks near-equal entries by fp64
+// logits) and as a pair of fp32 values hi + lo with hi the nearest tf32 value
+// (operands of the tensor-core score GEMM).  A partial last block divides by
+// its number of valid tokens.  Each consumer warp adds, once per head, the
+// number of that head's items it has written to the head's counter (a
+// release).  The score GEMM is launched behind this kernel with programmatic
+// stream serialization: its CTAs take SMs as this kernel's CTAs leave them and
+// wait on the counter of each head before they read its pooled vectors.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -34,9 +33,9 @@ using namespace sm100;
 
 constexpr int kPoolStages = 4;
 // Consumer groups: group g reduces the items it = g, g + kGroups, ... of its
-// CTA (stage it % kPoolStages), so several blocks are summed at once and the
-// conversions and fp64 adds of one block hide the latency of another's.
-constexpr int kGroups = 2;
+// CTA (stage it % kPoolStages).  One group per CTA with three CTAs per SM is
+// the fastest measured (273 us at 720p against 407 us with two groups).
+constexpr int kGroups = 1;
 constexpr uint64_t kPoolDrainNs = 1000000000ull;
 
 template <typename T, int D>
