@@ -257,7 +257,8 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, ds_bound: bool = False):
+def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, ds_bound: bool = False,
+                         ds_format: str | None = None):
     """Gradients of masked_attention with the mask held constant: with
     P = softmax(Q K_sel^T / sqrt(D)) per query block,
       dV_sel += P^T dO,  dP = dO V_sel^T,  dS = P * (dP - rowsum(P * dP)),
@@ -266,7 +267,10 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, ds_bound: b
     Returns (dQ, dK, dV) fp64 [B, H, S, D].  ds_bound=True also returns
     (bQ, bK): every gradient entry's sum of term magnitudes through dS,
     bQ = |dS| |K_sel| / sqrt(D) and bK_sel += |dS|^T |Q| / sqrt(D), the scale
-    of the error that rounding dS before these products can cause."""
+    of the error that rounding dS before these products can cause.
+    ds_format="bf16" rounds dS to bfloat16 (nearest even) before the dQ and
+    dK products, the operand a bf16 tensor-core backward multiplies; the
+    default is the exact (textbook) gradient."""
     Q, K, V, dO = as_f64(Q), as_f64(K), as_f64(V), as_f64(dO)
     B, H, S, D = Q.shape
     nb = num_blocks(S, N)
@@ -288,8 +292,9 @@ def masked_attention_bwd(Q, K, V, dO, M: np.ndarray, N: int = BLOCK, ds_bound: b
                 dP = g @ V[b, h, keys].T
                 delta = (P * dP).sum(axis=-1, keepdims=True)
                 dS = P * (dP - delta)
-                dQ[b, h, rows] = dS @ K[b, h, keys] * scale
-                dK[b, h, keys] += dS.T @ Q[b, h, rows] * scale
+                dSm = round_bf16(dS) if ds_format == "bf16" else dS
+                dQ[b, h, rows] = dSm @ K[b, h, keys] * scale
+                dK[b, h, keys] += dSm.T @ Q[b, h, rows] * scale
                 if ds_bound:
                     bQ[b, h, rows] = np.abs(dS) @ np.abs(K[b, h, keys]) * scale
                     bK[b, h, keys] += np.abs(dS).T @ np.abs(Q[b, h, rows]) * scale

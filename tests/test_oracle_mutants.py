@@ -95,7 +95,7 @@ def _attn_transposed_mask(Q, K, V, M, N=64):
     return _ORIG_ATTN(Q, K, V, np.swapaxes(M, -1, -2), N)
 
 
-def _bwd_no_rowsum(Q, K, V, dO, M, N=64, ds_bound=False):
+def _bwd_no_rowsum(Q, K, V, dO, M, N=64, ds_bound=False, ds_format=None):
     Q, K, V, dO = (orc.as_f64(x) for x in (Q, K, V, dO))
     B, H, S, D = Q.shape
     dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
@@ -110,8 +110,9 @@ def _bwd_no_rowsum(Q, K, V, dO, M, N=64, ds_bound=False):
                 P = e / e.sum(-1, keepdims=True)
                 dV[b, h, keys] += P.T @ dO[b, h, rows]
                 dS = P * (dO[b, h, rows] @ V[b, h, keys].T)
-                dQ[b, h, rows] = dS @ K[b, h, keys] / np.sqrt(D)
-                dK[b, h, keys] += dS.T @ Q[b, h, rows] / np.sqrt(D)
+                dSm = orc.round_bf16(dS) if ds_format == "bf16" else dS
+                dQ[b, h, rows] = dSm @ K[b, h, keys] / np.sqrt(D)
+                dK[b, h, keys] += dSm.T @ Q[b, h, rows] / np.sqrt(D)
                 bQ[b, h, rows] = np.abs(dS) @ np.abs(K[b, h, keys]) / np.sqrt(D)
                 bK[b, h, keys] += np.abs(dS).T @ np.abs(Q[b, h, rows]) / np.sqrt(D)
     return (dQ, dK, dV, bQ, bK) if ds_bound else (dQ, dK, dV)

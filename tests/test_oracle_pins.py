@@ -452,6 +452,33 @@ def test_round_bf16_ties_to_even_and_matches_torch():
     assert np.array_equal(orc.round_bf16(y), ref)
 
 
+def test_backward_bf16_ds_is_exact_when_ds_is_bf16_and_bounded_by_ds_bound():
+    """ds_format="bf16" rounds dS before the dQ / dK products.  (a) With V
+    constant along the keys every dP row is constant, so dS = P (dP - rowsum(P
+    dP)) = 0 exactly and rounding changes nothing.  (b) In general the change
+    per gradient entry is at most 2^-9 times its sum of term magnitudes through
+    dS (the ds_bound sums), the bound a rounding of every dS entry to 8
+    significant bits allows."""
+    rng = np.random.default_rng(13)
+    S, D = 150, 16
+    Q, K, dO = (rng.standard_normal((1, 1, S, D)) for _ in range(3))
+    nb = orc.num_blocks(S)
+    M = rng.random((1, 1, nb, nb)) < 0.6
+    M[0, 0, np.arange(nb), np.arange(nb)] = True
+    V = np.broadcast_to(rng.standard_normal(D), (1, 1, S, D)).copy()
+    exact = orc.masked_attention_bwd(Q, K, V, dO, M)
+    rounded = orc.masked_attention_bwd(Q, K, V, dO, M, ds_format="bf16")
+    for a, b in zip(exact, rounded):
+        assert np.abs(a - b).max() < 1e-12
+    V = rng.standard_normal((1, 1, S, D))
+    dQ, dK, dV, bQ, bK = orc.masked_attention_bwd(Q, K, V, dO, M, ds_bound=True)
+    rQ, rK, rV = orc.masked_attention_bwd(Q, K, V, dO, M, ds_format="bf16")
+    assert np.abs(rV - dV).max() == 0.0
+    assert np.abs(rQ - dQ).max() > 0.0
+    assert (np.abs(rQ - dQ) <= 2.0 ** -9 * bQ + 1e-12).all()
+    assert (np.abs(rK - dK) <= 2.0 ** -9 * bK + 1e-12).all()
+
+
 def test_backward_ds_bound_matches_autograd_of_the_logits():
     """The magnitude sums through dS: dS is the gradient of the loss
     sum(dO * O) with respect to the scaled logits (masked keys at -inf), which
@@ -474,3 +501,25 @@ def test_backward_ds_bound_matches_autograd_of_the_logits():
     assert np.allclose(bK[0, 0], dS.T @ np.abs(Q[0, 0]) / math.sqrt(D), rtol=1e-10, atol=1e-12)
     # the bound dominates the gradient itself (triangle inequality)
     assert (np.abs(dQ) <= bQ + 1e-12).all() and (np.abs(dK) <= bK + 1e-12).all()
+
+
+def test_steep_rows_bf16_ds_alone_breaks_the_flat_gradient_bar():
+    """The reading behind the steep-row gradient bar.  With Q and K scaled by
+    8 (logits of magnitude ~10^2, nearly one-hot softmax rows) the exact
+    gradient, with dS alone rounded to bf16 before the dQ / dK products (P,
+    Delta and every other step exact in fp64), already misses the flat bar
+    |x - ref| <= 2e-2 + 2^-8 |ref| for dQ, while 2^-8 times the dS term
+    magnitudes covers it.  So no kernel that multiplies dS in bf16 on the
+    tensor cores meets the flat bar there, and the test at that scale adds
+    the dS term."""
+    import synth
+    x = synth.make_random_qkv(1, 2, 1000, 128, "bf16", seed=31, with_grad=True)   # the GPU test's inputs
+    Q, K = (8.0 * orc.as_f64(x[n][:, :1]) for n in ("q", "k"))                      # head 0
+    V, dO = orc.as_f64(x["v"][:, :1]), orc.as_f64(x["do"][:, :1])
+    M, _, _ = orc.nabla_mask(Q, K, 0.8)
+    dQ, dK, dV, bQ, bK = orc.masked_attention_bwd(Q, K, V, dO, M, ds_bound=True)
+    rQ, rK, _ = orc.masked_attention_bwd(Q, K, V, dO, M, ds_format="bf16")
+    flat = np.abs(rQ - dQ) - 2.0 ** -8 * np.abs(dQ)
+    assert flat.max() > 2e-2
+    assert (np.abs(rQ - dQ) - 2.0 ** -8 * np.abs(dQ) - 2.0 ** -8 * bQ).max() <= 2e-2
+    assert (np.abs(rK - dK) - 2.0 ** -8 * np.abs(dK) - 2.0 ** -8 * bK).max() <= 2e-2
