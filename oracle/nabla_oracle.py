@@ -192,6 +192,27 @@ def bits_to_mask(bits: np.ndarray, nb: int) -> np.ndarray:
     return (b & 1).astype(bool).reshape(bits.shape[:-1] + (-1,))[..., :nb]
 
 
+# ----------------------------------------------------------------- projection
+
+def qkv_project(X, Wt, H: int, D: int):
+    """Eq. 1 (§2.1): Q = X W_Q, K = X W_K, V = X W_V, for every sample.
+
+    X [B, S, C] holds the tokens' hidden states.  The multi-head reading: W_Q
+    is C x (H D), and head h of Q takes its columns h D .. h D + D - 1.  Wt
+    [3, H D, C] holds the transposes W_Q^T, W_K^T, W_V^T (one row per output
+    feature, n = h D + d), the way a linear layer stores its weight.
+    Returns Q, K, V as fp64 [B, H, S, D]."""
+    X, Wt = as_f64(X), as_f64(Wt)
+    B, S, C = X.shape
+    if Wt.shape != (3, H * D, C):
+        raise ValueError(f"Wt must be [3, {H * D}, {C}], got {list(Wt.shape)}")
+    out = []
+    for m in range(3):
+        Y = np.matmul(X, Wt[m].T)                              # [B, S, H D] = X W
+        out.append(Y.reshape(B, S, H, D).transpose(0, 2, 1, 3))  # head h: columns h D + d
+    return tuple(np.ascontiguousarray(y) for y in out)
+
+
 # ------------------------------------------------------------------ attention
 
 def _allowed_keys(M_row: np.ndarray, S: int, N: int = BLOCK) -> np.ndarray:

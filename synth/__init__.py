@@ -218,3 +218,25 @@ def line_coords(nb: int, T: int = 1, ny: int = 1) -> torch.Tensor:
     i = np.arange(nb)
     c = np.stack([i // (ny * nx), (i // nx) % ny, i % nx], 1).astype(np.int32)
     return torch.from_numpy(c)
+
+
+def make_projection_inputs(B: int, S: int, C: int, H: int, D: int, seed: int,
+                           sigma: float = 0.5, device: str = "cpu") -> dict:
+    """Hidden states and weights for the Eq. 1 projection Q = X W_Q (and K, V).
+
+    X [B, S, C] bf16: eps ~ N(0, 1) per token plus one mean vector per 64-token
+    block ~ N(0, sigma^2 I_C), so the projected Q and K carry block structure
+    for the mask builder to find.  Wt [3, H D, C] bf16: the transposed W_Q,
+    W_K, W_V (one row per output feature), entries ~ N(0, 1 / C), which keeps
+    the projected values at unit scale.  device="cuda" draws the same kind of
+    values on the GPU (a different stream of random numbers) for sizes the
+    host would take long to fill."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    nb = num_blocks(S)
+    m = torch.randn(B, nb, C, generator=g, device=device) * sigma
+    tok_block = torch.arange(S, device=device) // BLOCK
+    X = torch.empty(B, S, C, dtype=torch.bfloat16, device=device)
+    for b in range(B):
+        X[b] = (torch.randn(S, C, generator=g, device=device) + m[b][tok_block]).to(torch.bfloat16)
+    Wt = (torch.randn(3, H * D, C, generator=g, device=device) / math.sqrt(C)).to(torch.bfloat16)
+    return {"x": X, "wt": Wt, "S": S, "nb": nb}

@@ -3,8 +3,10 @@ in test_oracle_pins.py catch every one of them: a wrong sort direction, a
 strict comparison, an exclusive cumulative sum, thr for 1 - thr, a missing
 order restoration, a tail block divided by 64, transposed or unscaled scores,
 softmax over the wrong axis, a wrong STA half-width, a transposed block mask,
-a dropped term in the backward pass, and a fractal order with tokens or
-patches taken column-major or edge patches moved to the end of the frame."""
+a dropped term in the backward pass, a fractal order with tokens or
+patches taken column-major or edge patches moved to the end of the frame, and
+an Eq. 1 projection with heads and dimensions swapped, one weight for Q, K and
+V, or the stored weight read untransposed."""
 import numpy as np
 import pytest
 
@@ -185,7 +187,27 @@ def _coords_variant(last_token=False, xy_swapped=False):
     return f
 
 
+def _project_variant(heads_inner=False, one_weight=False, untransposed=False):
+    def f(X, Wt, H, D):
+        X, Wt = orc.as_f64(X), orc.as_f64(Wt)
+        B, S, C = X.shape
+        out = []
+        for m in range(3):
+            w = Wt[0] if one_weight else Wt[m]
+            w = w.reshape(C, H * D) if untransposed else w.T
+            Y = np.matmul(X, w)
+            if heads_inner:
+                out.append(Y.reshape(B, S, D, H).transpose(0, 3, 1, 2))
+            else:
+                out.append(Y.reshape(B, S, H, D).transpose(0, 2, 1, 3))
+        return tuple(out)
+    return f
+
+
 MUTANTS = {
+    "projection_heads_inner": ("qkv_project", _project_variant(heads_inner=True)),
+    "projection_one_weight_for_qkv": ("qkv_project", _project_variant(one_weight=True)),
+    "projection_weight_not_transposed": ("qkv_project", _project_variant(untransposed=True)),
     "descending_sort": ("cdf_binarize", _cdf_variant(descending=True)),
     "strict_compare": ("cdf_binarize", _cdf_variant(strict=True)),
     "exclusive_cumsum": ("cdf_binarize", _cdf_variant(exclusive=True)),

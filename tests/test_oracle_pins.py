@@ -149,6 +149,64 @@ def test_nabla_mask_on_block_constant_inputs():
     assert M[0, 0].tolist() == [[True, True], [False, True]]
 
 
+# ------------------------------------------------ Eq. 1 projection (§2.1)
+
+def test_qkv_project_brute_force_tiny():
+    # Eq. 1 written out with Python loops: Q[b, h, s, d] = sum_c X[b, s, c] W_Q[c, h D + d]
+    rng = np.random.default_rng(11)
+    B, S, C, H, D = 2, 5, 3, 2, 3
+    X = rng.integers(-4, 5, size=(B, S, C)).astype(float)
+    W = rng.integers(-4, 5, size=(3, C, H * D)).astype(float)   # W_Q, W_K, W_V as in Eq. 1
+    Wt = np.ascontiguousarray(np.swapaxes(W, 1, 2))              # stored transposed
+    got = orc.qkv_project(X, Wt, H, D)
+    for m in range(3):
+        want = np.zeros((B, H, S, D))
+        for b in range(B):
+            for h in range(H):
+                for s in range(S):
+                    for d in range(D):
+                        want[b, h, s, d] = sum(X[b, s, c] * W[m, c, h * D + d] for c in range(C))
+        assert got[m].shape == (B, H, S, D)
+        assert np.array_equal(got[m], want)
+
+
+def test_qkv_project_one_hot_closed_form():
+    # A token that is the one-hot vector f e_c picks row c of W, scaled by f:
+    # Q[b, h, s, d] = f W_Q[c, h D + d].  With W^T[m, n, c] = 1000 m + 10 n + c
+    # every output names its own (m, n = h D + d, c).
+    B, S, C, H, D = 2, 7, 4, 2, 3
+    X = np.zeros((B, S, C))
+    f = np.zeros((B, S))
+    for b in range(B):
+        for s in range(S):
+            f[b, s] = 1 + s + 10 * b
+            X[b, s, (s + b) % C] = f[b, s]
+    Wt = np.fromfunction(lambda m, n, c: 1000 * m + 10 * n + c, (3, H * D, C))
+    out = orc.qkv_project(X, Wt, H, D)
+    for m in range(3):
+        for b in range(B):
+            for h in range(H):
+                for s in range(S):
+                    for d in range(D):
+                        want = f[b, s] * (1000 * m + 10 * (h * D + d) + (s + b) % C)
+                        assert out[m][b, h, s, d] == want
+
+
+def test_block_pooling_commutes_with_the_projection():
+    # the block mean is linear, so pooling the projected tokens equals
+    # projecting the pooled tokens (ragged tail included); exact here
+    # because every value is a small multiple of 1/8
+    rng = np.random.default_rng(5)
+    B, S, C, H, D = 1, 150, 6, 2, 4
+    X = rng.integers(-8, 9, size=(B, S, C)) / 8.0
+    Wt = rng.integers(-8, 9, size=(3, H * D, C)) / 8.0
+    Q, K, V = orc.qkv_project(X, Wt, H, D)
+    Xa = orc.block_pool(X)                                       # [B, nb, C]
+    Qa, Ka, Va = orc.qkv_project(Xa, Wt, H, D)                   # [B, H, nb, D]
+    assert np.allclose(orc.block_pool(Q), Qa, rtol=0, atol=1e-12)
+    assert np.allclose(orc.block_pool(K), Ka, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------------- STA
 
 @pytest.mark.parametrize("case", _read_golden("sta_table1.txt"))
