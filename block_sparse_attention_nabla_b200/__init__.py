@@ -21,7 +21,8 @@ import torch
 __all__ = ["NablaError", "Mask", "build_mask", "mask_from_bits", "attn_fwd", "attn_bwd",
            "workspace", "workspace_size", "workspace_status", "set_wait_limit_ns", "lib",
            "selftest_wait_timeout", "build_mask_noalloc", "build_mask_noalloc_status", "fractal_reorder",
-           "build_mask_topk", "block_mass", "mask_recall", "sta_block_coords",
+           "build_mask_topk", "block_mass", "mask_recall", "sta_block_coords", "qkv_project",
+           "build_mask_pooled",
            "BLOCK", "BF16", "FP32"]
 
 BLOCK = 64
@@ -31,7 +32,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnabla.so
 
 # Exported symbols, in the order include/nabla.h declares them.
 SYMBOLS = ["nabla_workspace_size", "nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc",
-           "nabla_build_mask_noalloc_status", "nabla_build_sta_mask", "nabla_sta_block_coords",
+           "nabla_build_mask_noalloc_status", "nabla_qkv_project", "nabla_build_mask_pooled",
+           "nabla_build_sta_mask", "nabla_sta_block_coords",
            "nabla_mask_from_bits", "nabla_attn_fwd",
            "nabla_attn_bwd", "nabla_block_mass", "nabla_mask_recall", "nabla_fractal_reorder", "nabla_selftest_wait_timeout", "nabla_workspace_status",
            "nabla_set_wait_limit_ns",
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.nabla_build_mask_noalloc.argtypes = [SH, P, P, ctypes.c_float, ST, MK, P]
     L.nabla_build_mask_noalloc_status.argtypes = [ctypes.POINTER(I32), P]
     L.nabla_sta_block_coords.argtypes = [I32, I32, I32, I32, I32, P]
+    L.nabla_qkv_project.argtypes = [SH, I32, P, P, P, P, P, P, SZ, P]
+    L.nabla_build_mask_pooled.argtypes = [SH, ctypes.c_float, ST, MK, P, SZ, P]
     L.nabla_attn_fwd.argtypes = [SH, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_attn_bwd.argtypes = [SH, P, P, P, P, P, P, P, MK, P, P, P, P, SZ, P]
     L.nabla_fractal_reorder.argtypes = [P, P, I32, I32, I32, I32, I32, SZ, I32, P]
@@ -93,7 +97,8 @@ def lib() -> ctypes.CDLL:
     L.nabla_last_error.argtypes, L.nabla_last_error.restype = [], ctypes.c_char_p
     L.nabla_abi_version.argtypes, L.nabla_abi_version.restype = [], I32
     for name in ("nabla_build_mask", "nabla_build_mask_topk", "nabla_build_mask_noalloc", "nabla_mask_from_bits",
-                 "nabla_build_mask_noalloc_status", "nabla_build_sta_mask", "nabla_sta_block_coords",
+                 "nabla_build_mask_noalloc_status", "nabla_qkv_project", "nabla_build_mask_pooled",
+                 "nabla_build_sta_mask", "nabla_sta_block_coords",
                  "nabla_attn_fwd", "nabla_attn_bwd", "nabla_fractal_reorder", "nabla_block_mass",
                  "nabla_mask_recall",
                  "nabla_workspace_status", "nabla_selftest_wait_timeout"):
@@ -292,6 +297,54 @@ def build_mask_noalloc_status() -> int:
     _check(lib().nabla_build_mask_noalloc_status(ctypes.byref(out), _stream()),
            "nabla_build_mask_noalloc_status")
     return out.value
+
+
+def qkv_project(x: torch.Tensor, wt: torch.Tensor, H: int, D: int, q: torch.Tensor | None = None,
+                k: torch.Tensor | None = None, v: torch.Tensor | None = None,
+                ws: torch.Tensor | None = None):
+    """Eq. 1: Q = X W_Q, K = X W_K, V = X W_V from hidden states x [B, S, C]
+    and the transposed weights wt [3, H * D, C] (bf16 CUDA tensors), with the
+    block means of Q and K written into the workspace on the way.  Returns
+    (q, k, v, ws); build_mask_pooled(q.shape, thr, ws) then builds the mask
+    from those means without reading q and k."""
+    if x.dim() != 3 or wt.dim() != 3:
+        raise NablaError("x must be [B, S, C] and wt [3, H * D, C]")
+    B, S, C = x.shape
+    if tuple(wt.shape) != (3, H * D, C):
+        raise NablaError(f"wt must be [3, {H * D}, {C}], got {list(wt.shape)}")
+    for t, name in ((x, "x"), (wt, "wt")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise NablaError(f"{name} must be a contiguous bf16 CUDA tensor")
+    outs = []
+    for t in (q, k, v):
+        t = torch.empty(B, H, S, D, dtype=torch.bfloat16, device=x.device) if t is None else t
+        if tuple(t.shape) != (B, H, S, D) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise NablaError(f"q, k, v must be contiguous bf16 [{B}, {H}, {S}, {D}]")
+        outs.append(t)
+    sh = _shape_of(outs[0])
+    ws = workspace(outs[0]) if ws is None else ws
+    _check(lib().nabla_qkv_project(ctypes.byref(sh), int(C), x.data_ptr(), wt.data_ptr(), outs[0].data_ptr(),
+                                   outs[1].data_ptr(), outs[2].data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+           "nabla_qkv_project")
+    return outs[0], outs[1], outs[2], ws
+
+
+def build_mask_pooled(q_shape, thr: float, ws: torch.Tensor, sta_coords: torch.Tensor | None = None,
+                      sta_window: tuple | None = None, out: Mask | None = None, transpose: bool = True,
+                      dtype=torch.bfloat16) -> Mask:
+    """build_mask from the block means qkv_project left in ws (no read of Q, K)."""
+    B, H, S, D = (int(x) for x in q_shape)
+    if dtype not in _DTYPES:
+        raise NablaError("dtype must be bfloat16 or float32")
+    sh = _Shape(B, H, S, D, BLOCK, _DTYPES[dtype])
+    out = out or Mask.empty(B, H, S, ws.device, transpose)
+    out.check(B, H, S, ws.device)
+    sta = _sta_struct(sta_coords, sta_window, S)
+    ms = out.as_struct()
+    _check(lib().nabla_build_mask_pooled(ctypes.byref(sh), ctypes.c_float(thr),
+                                         ctypes.byref(sta) if sta is not None else None, ctypes.byref(ms),
+                                         ws.data_ptr(), ws.numel(), _stream()), "nabla_build_mask_pooled")
+    return out
 
 
 def sta_block_coords(T: int, H: int, W: int, P: int = 8, S: int | None = None) -> torch.Tensor:

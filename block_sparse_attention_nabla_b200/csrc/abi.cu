@@ -185,9 +185,10 @@ static nabla_status build_mask_impl(const nabla_shape* shape, const void* q, con
   NABLA_TRY(reset_status(workspace, st));
   NABLA_CUDA(cudaMemsetAsync(counters, 0, (size_t)d.BH() * 2 * sizeof(int32_t), st), "clear builder counters");
   NABLA_CUDA(launch_pool(d, q, k, qa, ka, qhi, qlo, khi, klo, counters, status, st), "pooling kernel");
-  NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, counters, status, st), "score GEMM kernel");
+  NABLA_CUDA(launch_score_gemm(d, qhi, qlo, khi, klo, logits, L.ldl, counters, pool_target(d), status, st),
+             "score GEMM kernel");
   NABLA_CUDA(launch_select(d, logits, L.ldl, qa, ka, topk ? 1.f : thr, sta, out->bits, out->cnt, out->idx,
-                           counters, status, st, topk),
+                           counters, pool_target(d), status, st, topk),
              "select kernel");
   return emit_derived(d, out->bits, out, st);
 }
@@ -205,6 +206,60 @@ nabla_status nabla_build_mask_topk(const nabla_shape* shape, const void* q, cons
   g_last_error.clear();
   if (topk < 1) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
   return build_mask_impl(shape, q, k, 1.f, topk, sta, out, workspace, workspace_bytes, stream);
+}
+
+nabla_status nabla_qkv_project(const nabla_shape* shape, int32_t C, const void* x, const void* wt, void* q,
+                               void* k, void* v, void* workspace, size_t workspace_bytes, nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  if (d.dtype != NABLA_BF16)
+    return fail(NABLA_ERR_UNSUPPORTED, "nabla_qkv_project runs on the tensor cores: bf16 only");
+  if (C < 8 || C % 8 != 0) return fail(NABLA_ERR_INVALID_ARG, "C must be a positive multiple of 8 (got %d)", C);
+  if (C > (1 << 20)) return fail(NABLA_ERR_UNSUPPORTED, "C = %d is above the limit of 1048576", C);
+  NABLA_TRY(check_tensor(x, "x"));
+  NABLA_TRY(check_tensor(wt, "wt"));
+  NABLA_TRY(check_tensor(q, "q"));
+  NABLA_TRY(check_tensor(k, "k"));
+  NABLA_TRY(check_tensor(v, "v"));
+  NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsLayout L = ws_layout(d, false);
+  char* ws = (char*)workspace;
+  NABLA_TRY(reset_status(workspace, st));
+  NABLA_CUDA(launch_qkv_project(d, C, x, wt, q, k, v, (double*)(ws + L.qa), (double*)(ws + L.ka),
+                                (float*)(ws + L.qhi), (float*)(ws + L.qlo), (float*)(ws + L.khi),
+                                (float*)(ws + L.klo), (int32_t*)workspace + kWsStatus, st),
+             "projection kernel");
+  return NABLA_OK;
+}
+
+nabla_status nabla_build_mask_pooled(const nabla_shape* shape, float thr, const nabla_sta* sta,
+                                     const nabla_mask* out, void* workspace, size_t workspace_bytes,
+                                     nabla_stream_t stream) {
+  g_last_error.clear();
+  NABLA_TRY(check_shape(shape));
+  const Dims d = make_dims(*shape);
+  NABLA_TRY(check_selection(thr, 0, sta));
+  NABLA_TRY(check_mask_out(out, true));
+  NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsLayout L = ws_layout(d, false);
+  char* ws = (char*)workspace;
+  int32_t* status = (int32_t*)workspace + kWsStatus;
+  int32_t* counters = (int32_t*)(ws + L.counters);
+  // the pooled vectors are in place: the score GEMM and the selection wait
+  // for no pooling (goal 0), only the selection for the GEMM's tiles
+  NABLA_CUDA(cudaMemsetAsync(counters, 0, (size_t)d.BH() * 2 * sizeof(int32_t), st), "clear builder counters");
+  NABLA_CUDA(launch_score_gemm(d, (const float*)(ws + L.qhi), (const float*)(ws + L.qlo),
+                               (const float*)(ws + L.khi), (const float*)(ws + L.klo), (float*)(ws + L.logits),
+                               L.ldl, counters, 0, status, st),
+             "score GEMM kernel");
+  NABLA_CUDA(launch_select(d, (const float*)(ws + L.logits), L.ldl, (const double*)(ws + L.qa),
+                           (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, counters, 0, status,
+                           st),
+             "select kernel");
+  return emit_derived(d, out->bits, out, st);
 }
 
 nabla_status nabla_fractal_reorder(const void* x, void* y, int32_t B, int32_t T, int32_t H, int32_t W,

@@ -78,6 +78,10 @@ uint64_t wait_limit_ns();
 // [B, H, nb, D] fp32 array, box {32, 128, 1}, 128-byte swizzle.
 bool make_map_bf16(CUtensorMap* map, const void* base, const Dims& d, int box_rows);
 bool make_map_pooled_f32(CUtensorMap* map, const float* base, const Dims& d);
+// make_map_bf16_rows: 3-D view {inner, rows, outer} of a contiguous bf16 array
+// (inner a multiple of 8), box {64, box_rows, 1}, 128-byte swizzle; elements
+// outside the array read as zero.
+bool make_map_bf16_rows(CUtensorMap* map, const void* base, int inner, long long rows, int outer, int box_rows);
 int sm_count();
 
 // Records the message nabla_last_error() returns in the calling thread (an
@@ -106,14 +110,18 @@ nabla_status check_selection(float thr, int32_t topk, const nabla_sta* sta);
 cudaError_t launch_pool(const Dims& d, const void* q, const void* k, double* qa, double* ka,
                         float* qhi, float* qlo, float* khi, float* klo, int32_t* counters, int32_t* status,
                         cudaStream_t st);
+// pool_goal: the count of pooled items that marks a head ready, pool_target(d)
+// behind the pooling kernel, 0 when the pooled vectors are already in place
+// (written by the Eq. 1 projection before the build).
 cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
-                              const float* klo, float* L, int ldl, int32_t* counters, int32_t* status,
-                              cudaStream_t st);
+                              const float* klo, float* L, int ldl, int32_t* counters, int pool_goal,
+                              int32_t* status, cudaStream_t st);
 // topk > 0 selects the fixed-budget rule (the topk largest entries per row)
 // instead of the CDF rule with thr.
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          const int32_t* counters, int32_t* status, cudaStream_t st, int topk = 0);
+                          const int32_t* counters, int pool_goal, int32_t* status, cudaStream_t st,
+                          int topk = 0);
 // Targets of the counters: every pooled item is counted once by each of the
 // pooling kernel's D / 32 consumer warps, every score tile once by each of the
 // GEMM's four epilogue warps.
@@ -151,6 +159,14 @@ cudaError_t launch_attn_bwd_tc(const Dims& d, const void* q, const void* k, cons
                                const void* o_res, const void* dout, const float* lse, const uint32_t* bits, const int32_t* cnt,
                                const int32_t* idx, const int32_t* cnt_t, float* lse2p, float* deltap, void* dq,
                                void* dk, void* dv, int32_t* ws_header, cudaStream_t st);
+
+// Eq. 1 projection with the block pooling fused (qkv_tc.cu): x [B, S, C] and
+// wt [3, H D, C] bf16 (C a multiple of 8); q, k, v [B, H, S, D] bf16; the
+// pooled Q and K into the builder's workspace arrays (same values as
+// launch_pool computes from q and k).
+cudaError_t launch_qkv_project(const Dims& d, int C, const void* x, const void* wt, void* q, void* k, void* v,
+                               double* qa, double* ka, float* qhi, float* qlo, float* khi, float* klo,
+                               int32_t* status, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 

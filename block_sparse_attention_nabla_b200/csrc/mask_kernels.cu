@@ -549,7 +549,8 @@ cudaError_t set_smem(Kern k, size_t bytes) {
 
 cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* qa, const double* ka,
                           float thr, const nabla_sta* sta, uint32_t* bits, int32_t* cnt, int32_t* idx,
-                          const int32_t* counters, int32_t* status, cudaStream_t st, int topk) {
+                          const int32_t* counters, int pool_goal, int32_t* status, cudaStream_t st,
+                          int topk) {
   const long long rows = d.BH() * d.nb;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   const bool use_sta = sta && sta->block_coords;
@@ -557,9 +558,9 @@ cudaError_t launch_select(const Dims& d, const float* L, int ldl, const double* 
   const int hT = use_sta ? sta->wT / 2 : 0, hH = use_sta ? sta->wH / 2 : 0, hW = use_sta ? sta->wW / 2 : 0;
   if (d.D == 128)
     return launch_select_rows<128>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits,
-                                   cnt, idx, counters, pool_target(d), score_target(d), status);
+                                   cnt, idx, counters, pool_goal, score_target(d), status);
   return launch_select_rows<64>(grid, st, L, ldl, qa, ka, rows, d.nb, d.W, thr, topk, coords, hT, hH, hW, bits, cnt,
-                                idx, counters, pool_target(d), score_target(d), status);
+                                idx, counters, pool_goal, score_target(d), status);
 }
 
 cudaError_t launch_sta_bits(const Dims& d, const nabla_sta& sta, uint32_t* bits, cudaStream_t st) {

@@ -108,10 +108,11 @@ extern "C" NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* sh
   if (e == cudaSuccess)
     e = launch_score_gemm(d, (const float*)(ws + L.qhi), (const float*)(ws + L.qlo),
                           (const float*)(ws + L.khi), (const float*)(ws + L.klo), (float*)(ws + L.logits),
-                          L.ldl, counters, status, st);
+                          L.ldl, counters, pool_target(d), status, st);
   if (e == cudaSuccess)
     e = launch_select(d, (const float*)(ws + L.logits), L.ldl, (const double*)(ws + L.qa),
-                      (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, counters, status, st);
+                      (const double*)(ws + L.ka), thr, sta, out->bits, out->cnt, out->idx, counters,
+                      pool_target(d), status, st);
   if (e == cudaSuccess && out->cnt_t) e = launch_transpose_lists(d, out->bits, out->cnt_t, out->idx_t, st);
   if (e == cudaSuccess) e = launch_work_list(d, out->bits, out->work, st);
   if (e != cudaSuccess) {

@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_gemm_kernel(
 
 template <int D>
 cudaError_t run(const Dims& d, const float* qhi, const float* qlo, const float* khi, const float* klo,
-                float* L, int ldl, int32_t* counters, int32_t* status, cudaStream_t st) {
+                float* L, int ldl, int32_t* counters, int pool_goal, int32_t* status, cudaStream_t st) {
   CUtensorMap a, b, c, e;
   if (!make_map_pooled_f32(&a, qhi, d) || !make_map_pooled_f32(&b, qlo, d) ||
       !make_map_pooled_f32(&c, khi, d) || !make_map_pooled_f32(&e, klo, d))
@@ -270,16 +270,16 @@ cudaError_t run(const Dims& d, const float* qhi, const float* qlo, const float* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a, b, c, e, L, d.nb, ldl, T, n_tiles, 1.0f / sqrtf((float)d.D), counters,
-                            pool_target(d), status, wait_limit_ns());
+                            pool_goal, status, wait_limit_ns());
 }
 
 }  // namespace
 
 cudaError_t launch_score_gemm(const Dims& d, const float* qhi, const float* qlo, const float* khi,
-                              const float* klo, float* L, int ldl, int32_t* counters, int32_t* status,
-                              cudaStream_t st) {
-  if (d.D == 128) return run<128>(d, qhi, qlo, khi, klo, L, ldl, counters, status, st);
-  return run<64>(d, qhi, qlo, khi, klo, L, ldl, counters, status, st);
+                              const float* klo, float* L, int ldl, int32_t* counters, int pool_goal,
+                              int32_t* status, cudaStream_t st) {
+  if (d.D == 128) return run<128>(d, qhi, qlo, khi, klo, L, ldl, counters, pool_goal, status, st);
+  return run<64>(d, qhi, qlo, khi, klo, L, ldl, counters, pool_goal, status, st);
 }
 
 }  // namespace nabla

@@ -50,7 +50,7 @@ extern "C" {
 #define NABLA_API
 #endif
 
-#define NABLA_ABI_VERSION 2
+#define NABLA_ABI_VERSION 3
 #define NABLA_BLOCK 64
 
 typedef struct CUstream_st* nabla_stream_t; /* same type as cudaStream_t */
@@ -120,8 +120,9 @@ NABLA_API size_t nabla_workspace_size(const nabla_shape* shape, int32_t want_bwd
  *          value are all kept).
  *   sta    NULL or sta->block_coords NULL: no STA union.
  *   out    bits, cnt, idx, work are required; cnt_t/idx_t are filled if not NULL.
- * Pooling, scores and selection run in fp32 (the pooled vectors are fp32
- * means of the inputs). */
+ * The pooled vectors are fp64 means of the inputs; the reduced scores use
+ * them as tf32 hi / lo pairs accumulated in fp32, and entries whose fp32
+ * values fall into the cut-off's 2^-7-wide bucket are ranked by fp64 logits. */
 NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const void* q, const void* k, float thr,
                               const nabla_sta* sta, const nabla_mask* out, void* workspace,
                               size_t workspace_bytes, nabla_stream_t stream);
@@ -179,6 +180,49 @@ NABLA_API nabla_status nabla_build_mask_noalloc(const nabla_shape* shape, const 
  * paper has no counterpart.  Errors: NABLA_ERR_INVALID_ARG for a NULL
  * host_status, NABLA_ERR_CUDA if the copy fails. */
 NABLA_API nabla_status nabla_build_mask_noalloc_status(int32_t* host_status, nabla_stream_t stream);
+
+/* Eq. 1 (§2.1), Q = X W_Q, K = X W_K, V = X W_V, on the tensor cores, with the
+ * block averaging of Algorithm 1 (§3.1.2) fused into the same kernel: while it
+ * writes Q and K it also writes their 64-token block means, so that
+ * nabla_build_mask_pooled builds the mask without reading Q and K again.
+ *   shape  as for nabla_build_mask; dtype must be NABLA_BF16.  Head h of Q is
+ *          columns h D .. h D + D - 1 of X W_Q (likewise K and V).
+ *   C      hidden size: the columns of X and the rows of W_Q; >= 8 and a
+ *          multiple of 8 (rows of 16-byte multiples), at most 1,048,576.
+ *   x      device, [B, S, C] bf16, token-major hidden states, read only.
+ *   wt     device, [3, H * D, C] bf16: W_Q^T, W_K^T, W_V^T, one row of C
+ *          weights per output feature n = h D + d (the layout of a linear
+ *          layer's weight), read only.
+ *   q, k, v  device, [B, H, S, D] bf16, written: the fp32-accumulated products
+ *          rounded to the nearest bf16 (ties to even).  They must not overlap
+ *          x, wt, each other or the workspace.
+ *   workspace, workspace_bytes  the mask builder's workspace (at least
+ *          nabla_workspace_size(shape, 0) bytes, 256-byte aligned): receives
+ *          the block means of the stored Q and K, the same values the
+ *          builder's own pooling computes from them; its status word is
+ *          cleared first and records NABLA_ERR_TIMEOUT if a bounded wait of
+ *          the kernel ran out.
+ * All pointers 16-byte aligned.  Asynchronous on `stream`; allocates nothing.
+ * Errors: NABLA_ERR_INVALID_ARG for an invalid shape, a NULL or misaligned
+ * pointer or a bad C; NABLA_ERR_UNSUPPORTED for fp32 inputs, a block size, D
+ * or sequence length this build does not handle, or C above the limit;
+ * NABLA_ERR_WORKSPACE for a workspace that is too small or misaligned;
+ * NABLA_ERR_CUDA if the launch fails. */
+NABLA_API nabla_status nabla_qkv_project(const nabla_shape* shape, int32_t C, const void* x, const void* wt,
+                                         void* q, void* k, void* v, void* workspace, size_t workspace_bytes,
+                                         nabla_stream_t stream);
+
+/* nabla_build_mask starting from the block means that nabla_qkv_project left
+ * in the workspace: the reduced scores, selection, STA union and lists of
+ * Algorithm 1 without reading Q and K.  thr, sta, out and the results as for
+ * nabla_build_mask (bit-identical masks for the same Q and K).  The workspace
+ * must be the one the projection wrote for this shape, on the same stream (or
+ * ordered after it), with no other call using it in between; its status word
+ * is not cleared, so a timeout of the projection stays visible to
+ * nabla_workspace_status.  Allocates nothing.  Errors as nabla_build_mask. */
+NABLA_API nabla_status nabla_build_mask_pooled(const nabla_shape* shape, float thr, const nabla_sta* sta,
+                                               const nabla_mask* out, void* workspace, size_t workspace_bytes,
+                                               nabla_stream_t stream);
 
 /* Sliding-tile (STA) mask alone, without the NABLA selection: the STA
  * configurations of Table 1 (§4.1) and the neighbourhood mask of §2.2 (Eq. 5).

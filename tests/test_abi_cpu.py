@@ -42,14 +42,14 @@ def mask_struct(**kw):
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 18
+    assert len(names) == 20
     assert sorted(nabla.SYMBOLS) == names
     for n in names:
         assert hasattr(L, n), n
 
 
 def test_abi_version(L):
-    assert L.nabla_abi_version() == 2
+    assert L.nabla_abi_version() == 3
 
 
 def test_workspace_size_formula(L):
@@ -104,6 +104,38 @@ def test_build_mask_argument_errors(L):
     assert _build(L, ws_bytes=100) == WORKSPACE
     assert b"needed" in L.nabla_last_error()
     assert _build(L, ws=FAKE + 16) == WORKSPACE         # workspace must be 256-byte aligned
+
+
+def test_projection_argument_errors(L):
+    def proj(sh=None, C=256, x=FAKE, wt=FAKE, q=FAKE, k=FAKE, v=FAKE, ws=FAKE, ws_bytes=1 << 40):
+        return L.nabla_qkv_project(ctypes.byref(sh or shape()), C, x, wt, q, k, v, ws, ws_bytes, None)
+    assert proj(C=0) == INVALID
+    assert proj(C=100) == INVALID                        # not a multiple of 8
+    assert b"multiple of 8" in L.nabla_last_error()
+    assert proj(C=(1 << 20) + 8) == UNSUPPORTED
+    assert proj(sh=shape(dtype=1)) == UNSUPPORTED        # the projection runs on the tensor cores: bf16
+    assert b"bf16" in L.nabla_last_error()
+    assert proj(sh=shape(D=96)) == UNSUPPORTED
+    assert proj(x=None) == INVALID
+    assert b"x is NULL" in L.nabla_last_error()
+    assert proj(wt=FAKE + 8) == INVALID
+    assert proj(v=None) == INVALID
+    assert proj(ws=None) == WORKSPACE
+    assert proj(ws_bytes=1000) == WORKSPACE
+
+
+def test_pooled_build_argument_errors(L):
+    def build(sh=None, thr=0.5, sta=None, m=None, ws=FAKE, ws_bytes=1 << 40):
+        return L.nabla_build_mask_pooled(ctypes.byref(sh or shape()), ctypes.c_float(thr),
+                                         ctypes.byref(sta) if sta is not None else None,
+                                         ctypes.byref(m or mask_struct()), ws, ws_bytes, None)
+    assert build(thr=0.0) == INVALID
+    assert build(thr=1.5) == INVALID
+    assert build(m=mask_struct(bits=None)) == INVALID
+    assert build(sta=nabla._Sta(FAKE, 0, 3, 3)) == INVALID
+    assert build(sh=shape(D=96)) == UNSUPPORTED
+    assert build(ws=None) == WORKSPACE
+    assert build(ws_bytes=100) == WORKSPACE
 
 
 def test_attention_argument_errors(L):
