@@ -600,6 +600,63 @@ def measure_reorder(nabla, dev, warmup: int, steps: int) -> dict:
             "kernel": "reorder_kernel (reorder.cu)", **res}
 
 
+def measure_projection(nabla, dev, warmup: int, steps: int, heads: int | None = None) -> dict:
+    """Eq. 1 projection with the block pooling fused (NEXT-4): Q, K, V = X W
+    at the 720p shape (B=1, S=75,600, C=5120, H=40, D=128) from hidden states
+    with per-block means and N(0, 1/C) weights drawn on the GPU.  Reports the
+    fused kernel (tensor-bound: 2 S C (3 H D) flops; timed alone, so against
+    the burst bf16 peak), a library GEMM of the same product for context, and
+    the mask build from the fused means against the build that pools Q and K
+    itself.  heads (profiling only) keeps C and S and projects onto fewer heads."""
+    import torch
+    import synth
+    B, H, S, D, C = 1, heads or 40, 75600, 128, 5120
+    d = synth.make_projection_inputs(B, S, C, H, D, seed=3, device=dev)
+    x, wt = d["x"], d["wt"]
+    q, k, v, ws = nabla.qkv_project(x, wt, H, D)
+    mask = nabla.build_mask_pooled(q.shape, THR, ws, transpose=False)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(max(warmup, 1)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    flops = 2.0 * B * S * C * 3 * H * D
+    proj_ms = timed(lambda: nabla.qkv_project(x, wt, H, D, q, k, v, ws), steps)
+    if nabla.workspace_status(ws) != 0:
+        raise SystemExit("device status word reports a timeout in the projection leg")
+    pooled_ms = timed(lambda: nabla.build_mask_pooled(q.shape, THR, ws, out=mask, transpose=False), steps)
+    ws2 = nabla.workspace(q)
+    direct_ms = timed(lambda: nabla.build_mask(q, k, THR, out=mask, ws=ws2, transpose=False), steps)
+    out = torch.empty(B * S, 3 * H * D, dtype=torch.bfloat16, device=dev)
+    lib_ms = timed(lambda: torch.matmul(x.reshape(B * S, C), wt.reshape(3 * H * D, C).t(), out=out), steps)
+    if nabla.workspace_status(ws) != 0 or nabla.workspace_status(ws2) != 0:
+        raise SystemExit("device status word reports a timeout in the projection leg")
+    peaks = _peaks()
+    tflops = flops / (proj_ms * 1e-3) / 1e12
+    res = {"workload": f"X [{B}, {S}, {C}] x W [{C}, 3 x {H * D}] bf16 -> Q, K, V [{B}, {H}, {S}, {D}] "
+                       f"+ block means of Q, K; thr {THR} for the builds",
+           "kernel": "qkv_project_kernel (qkv_tc.cu)", "ms": proj_ms, "tflops": tflops,
+           "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                        "frac": tflops / peaks["bf16"],
+                        "peak_note": f"{peaks['source']} burst bf16 (kernel timed alone)",
+                        "algorithmic": "2 * B * S * C * 3 * H * D flops per launch"},
+           "library_gemm_ms": lib_ms, "library_gemm_tflops": flops / (lib_ms * 1e-3) / 1e12,
+           "library_gemm_note": "torch.matmul (cuBLAS) of the same product into [B*S, 3*H*D], no pooling",
+           "mask_build_from_fused_means_ms": pooled_ms, "mask_build_from_q_k_ms": direct_ms}
+    del x, wt, q, k, v, ws, ws2, out, mask
+    torch.cuda.empty_cache()
+    return res
+
+
 def _config(w, n) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.H} S={w.S} D={w.D} bf16, {w.T}x{w.Hl}x{w.Wl} tokens, "
                         f"thr {THR}, no STA",
@@ -629,6 +686,8 @@ def main() -> None:
                     help="run only the two threshold sweeps and print their JSON (not a bench line)")
     ap.add_argument("--only-fidelity", action="store_true",
                     help="run only the block-fidelity leg and print its object (profiling; not a bench line)")
+    ap.add_argument("--only-projection", action="store_true",
+                    help="run only the fused projection leg and print its object (profiling; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the head count (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
@@ -668,6 +727,11 @@ def main() -> None:
         del qs, ks, vs
         print(json.dumps({"sweep": first, "sweep_sigma06": measure_sweep_sigma06(
             nabla, dev0, max(1, args.warmup), max(1, args.steps))}), flush=True)
+        return
+    if args.only_projection:
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_projection(nabla, torch.device("cuda", 0), max(1, args.warmup),
+                                            max(1, args.steps), args.heads)), flush=True)
         return
     if args.only_fidelity:
         torch.cuda.set_device(0)
@@ -765,6 +829,10 @@ def main() -> None:
     if world == 1 and not args.no_sweep:
         reorder = measure_reorder(nabla, dev, 3, 10)
 
+    projection = None
+    if world == 1 and not args.no_sweep:
+        projection = measure_projection(nabla, dev, 3, 10)
+
     fidelity = None
     if world == 1 and not args.no_sweep:
         fidelity = measure_fidelity(nabla, q, k)
@@ -816,6 +884,7 @@ def main() -> None:
             "sweep_sigma06": sweep06,
             "table1": table1,
             "fractal_reorder": reorder,
+            "projection": projection,
             "fidelity": fidelity,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks.summary(),

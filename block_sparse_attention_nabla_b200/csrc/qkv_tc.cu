@@ -16,9 +16,10 @@
 //
 // Persistent kernel, one CTA per SM, tiles of 128 tokens (two 64-token blocks
 // of one sample) x 256 output features, taken in a fixed round-robin share of
-// a grouped order (eight token tiles per group, all feature tiles of a group
-// before the next) so that the CTAs of one wave share their X and W tiles in
-// L2.  Warp 0 streams 64-feature slices of X and W^T (16 + 32 KB) through a
+// a grouped order (16 token tiles per group, all feature tiles of a group
+// before the next): the CTAs of one wave share their X and W tiles in L2
+// (at C = 5120 a wave holds 16 X tiles and about 9 W tiles, 45 MB, the
+// smallest such working set), and W is read from DRAM about once per group.  Warp 0 streams 64-feature slices of X and W^T (16 + 32 KB) through a
 // 4-stage TMA ring; warp 1 owns TMEM and issues four K = 16 MMAs per slice
 // (M = 128, N = 256, both operands K-major in shared memory, the shape that
 // runs at the full tensor rate) into one of two 256-column accumulators;
@@ -43,7 +44,7 @@ constexpr int kTileN = 256;                              // output features per 
 constexpr int kTileK = 64;                               // hidden features per stage (128-byte rows)
 constexpr int kStages = 4;
 constexpr int kThreads = 192;                            // producer, MMA issuer, 4 epilogue warps
-constexpr int kGroupM = 8;                               // token tiles per raster group
+constexpr int kGroupM = 16;                              // token tiles per raster group
 constexpr int kChunk = 64;                               // accumulator columns per epilogue pass
 constexpr uint32_t kABytes = kTileM * 128;               // X slice: 128 rows x 128 B
 constexpr uint32_t kBBytes = kTileN * 128;               // W^T slice: 256 rows x 128 B
