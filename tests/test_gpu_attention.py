@@ -80,11 +80,11 @@ def test_fwd_edge_masks(dtype):
     assert np.isneginf(lse.cpu().numpy()[empty]).all()
 
 
-@pytest.mark.parametrize("wid,heads", [(2, list(range(40))), (3, [0, 17, 39]), (7, [0, 17, 39])])
+@pytest.mark.parametrize("wid,heads", [(2, list(range(40))), (3, list(range(40))), (7, list(range(40)))])
 def test_fwd_full_size_sampled_rows(wid, heads):
     """Full-size forward (the benchmark's launch configuration) under the
-    oracle's mask, checked on sampled rows: every head of the 480p shape,
-    three heads of the 720p shapes."""
+    oracle's mask, checked on sampled rows of every head of the 480p and 720p
+    shapes."""
     w = synth.WORKLOADS[wid]
     x = synth.make_inputs(w)
     thr = w.thresholds[0]
@@ -161,12 +161,16 @@ def test_bwd_small_fp32(S, D):
     _bwd_parity(x, M, "fp32")
 
 
-@pytest.mark.parametrize("residual", [False, True])
-def test_bwd_pretraining_workload_two_heads(residual):
+@pytest.mark.parametrize("residual,heads", [
+    (False, [(0, 0), (1, 15)]),
+    # the training configuration (residual mode): eight heads over both samples
+    (True, [(b, h) for b in (0, 1) for h in (0, 5, 10, 15)]),
+])
+def test_bwd_pretraining_workload(residual, heads):
     w = synth.WORKLOADS[4]
     x = synth.make_inputs(w)
     M, C, _ = gu.oracle_mask(x["q"], x["k"], w.thresholds[0])
-    _bwd_parity(x, M, "bf16", heads=[(0, 0), (1, 15)], residual=residual)
+    _bwd_parity(x, M, "bf16", heads=heads, residual=residual)
 
 
 @pytest.mark.parametrize("B,H,S,seed", [(1, 2, 1000, 21), (2, 3, 2000, 22), (1, 1, 64, 23)])
