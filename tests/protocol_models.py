@@ -23,8 +23,12 @@ Models:
   earlier MMAs are done, so each issuer is an in-order engine), the
   elementwise group and its epilogue, TMA copies landing at any time.
 
-* ``score_gemm`` -- score_tc.cu: operand stage ring, two TMEM accumulators
-  handed between the issuer and the epilogue.
+* ``score_gemm`` -- score_tc.cu (and qkv_tc.cu, with four stages): operand
+  stage ring, two TMEM accumulators handed between the issuer and the
+  epilogue.
+* ``staging_ring`` -- qkv_tc.cu's epilogue: four warps stage each 64-column
+  chunk in one of two shared-memory tiles, meet at one named barrier per
+  chunk, then read the whole tile (row stores and block sums).
 * ``fwd_pipeline`` -- attn_fwd_tc.cu after the unit ring: Q / K producer, V
   producer, the MMA issuer, the softmax group with its O rescale and
   epilogue.  Units without tiles do not signal O (mutation
@@ -545,3 +549,34 @@ def score_gemm(n_tiles: int, seed: int, S: int = 2, n_sub: int = 4, mutation: st
     _run({"producer": producer(), "issuer": issuer(), "epilogue": epilogue()}, bars, engines, execute, rnd)
     if st["drained"] != list(range(n_tiles)):
         raise ProtocolError(f"tiles drained {st['drained']}")
+
+
+def staging_ring(n_chunks: int, seed: int, n_warps: int = 4, mutation: str | None = None) -> None:
+    """qkv_tc.cu's epilogue: for chunk c every warp writes its rows into
+    staging tile c % 2, arrives at the named barrier (one phase per chunk) and
+    waits for it, then reads rows of every warp.  A warp writes tile c % 2
+    again only at chunk c + 2, after the barrier of chunk c + 1, which no warp
+    reaches before it has finished reading chunk c.  Mutation "one_tile" stages
+    every chunk in the same tile."""
+    rnd = random.Random(seed)
+    bars = {"named": _Bar(n_warps)}
+    st = {"tile": [dict(), dict()], "readers": [set(), set()]}
+
+    def warp(w):
+        for c in range(n_chunks):
+            b = 0 if mutation == "one_tile" else c & 1
+            if st["readers"][b] - {w}:
+                raise ProtocolError(f"warp {w} writes tile {b} for chunk {c} while {st['readers'][b]} read it")
+            st["tile"][b][w] = c
+            yield ("arrive", "named")
+            yield ("wait", "named", c)
+            st["readers"][b].add(w)
+            for v in range(n_warps):
+                if st["tile"][b].get(v) != c:
+                    raise ProtocolError(f"warp {w} reads chunk {c} and finds warp {v}'s rows of {st['tile'][b].get(v)}")
+                yield ("arrive", f"tick{w}")          # the reads take a while
+            st["readers"][b].discard(w)
+
+    for w in range(n_warps):
+        bars[f"tick{w}"] = _Bar(1)
+    _run({f"warp{w}": warp(w) for w in range(n_warps)}, bars, {}, lambda e, op: None, rnd)

@@ -82,7 +82,7 @@ def _gemm_traces(n, S, mutation=None):
     return failures
 
 
-@pytest.mark.parametrize("S", [2, 3])
+@pytest.mark.parametrize("S", [2, 3, 4])
 def test_score_gemm_protocol_holds(S):
     assert _gemm_traces(1500, S) == 0
 
@@ -90,3 +90,18 @@ def test_score_gemm_protocol_holds(S):
 @pytest.mark.parametrize("mutation", ["no_stage_wait", "no_acc_wait", "early_release"])
 def test_score_gemm_mutants_are_caught(mutation):
     assert _gemm_traces(600, 2, mutation) > 0
+
+
+def test_staging_ring_protocol_holds():
+    for seed in range(800):
+        pm.staging_ring(6, seed)
+
+
+def test_staging_ring_single_tile_is_caught():
+    failures = 0
+    for seed in range(300):
+        try:
+            pm.staging_ring(6, seed, mutation="one_tile")
+        except pm.ProtocolError:
+            failures += 1
+    assert failures > 0
