@@ -42,12 +42,30 @@ THR = 0.8
 NCU_TRAFFIC = {
     # 4-head capture of the 720p shape at thr 0.8: 301.6 MB, scaled x10 to 40 heads
     "attn_fwd_tc.cu": ("bc42bc8e5f502ccf8f42ff8185e5efa74da747e0c6fee1a7d40adc9c6b74438a", 3.016e9),
+    # full-size capture of the projection leg (one pass): DRAM read 7.96 GB + write 2.50 GB
+    "qkv_tc.cu": ("2bf31b7e64ef472bc2670ca245436e66ceafb3494d6951646151ea3385f8ff90", 10.46e9),
 }
+# the mask builder's four launches, captured together at full size (one pass
+# each): pool 1.55 GB + 184 MB, score GEMM 98 + 165 MB, selection 323 + 95 MB,
+# work list 7 MB; keyed by the three sources they come from
+NCU_BUILDER_TRAFFIC = ({"pool.cu": "ca97bc086ac16466e6d5db392101528fccf729ca4dfb3b099cfc0c5a87fad7b6",
+                        "score_tc.cu": "21f70fb96eaedfe6a16ebc1c608ea74616280707caf240b4744f22c3cd28cc5a",
+                        "mask_kernels.cu": "b7a03e632ccf5e26dd4f61360ca8d46eab111746af8de1b68aff913884ac51aa"},
+                       2.422e9)
 
 
 def _sha(path: str) -> str:
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
+
+
+def _builder_traffic():
+    files, bytes_ = NCU_BUILDER_TRAFFIC
+    for f, h in files.items():
+        path = os.path.join(ROOT, "block_sparse_attention_nabla_b200", "csrc", f)
+        if not os.path.exists(path) or _sha(path) != h:
+            return None
+    return bytes_
 
 
 def _traffic(kernel_file: str):
@@ -648,6 +666,7 @@ def measure_projection(nabla, dev, warmup: int, steps: int, heads: int | None = 
            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16"], "unit": "TFLOP/s",
                         "frac": tflops / peaks["bf16"],
                         "peak_note": f"{peaks['source']} burst bf16 (kernel timed alone)",
+                        "traffic": _traffic("qkv_tc.cu") if H == 40 else None,
                         "algorithmic": "2 * B * S * C * 3 * H * D flops per launch"},
            "library_gemm_ms": lib_ms, "library_gemm_tflops": flops / (lib_ms * 1e-3) / 1e12,
            "library_gemm_note": "torch.matmul (cuBLAS) of the same product into [B*S, 3*H*D], no pooling",
@@ -875,7 +894,8 @@ def main() -> None:
             "mask_roofline": {"bound": "hbm", "kernels": "pool + score GEMM + select + work list",
                               "achieved": mask_gbs, "peak": peaks["hbm"], "unit": "GB/s",
                               "frac": mask_gbs / peaks["hbm"], "bytes_per_call": mask_bytes,
-                              "ms_per_call": mask_avg, "traffic": None,
+                              "ms_per_call": mask_avg,
+                              "traffic": _builder_traffic() if (H, S) == (40, 75600) else None,
                               "algorithmic": "Q + K read once; bitmask, counts, kept indices, work list written"},
             "e2e": e2e,
             "configs": configs,
