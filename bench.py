@@ -206,6 +206,73 @@ def cpu_baseline(x: dict, thr: float, budget_s: float = 12.0, heads_total: int |
             "host_cpus": os.cpu_count()}
 
 
+def cpu_baseline_legs(main_rate_tflops: float, sweep=None, table1=None) -> dict:
+    """The fp64 oracle, as it stands, timed beside the other legs on bounded
+    samples of their workloads (a few seconds each), each extrapolated to the
+    leg's full problem and labelled; part of the CPU-baseline leg."""
+    import numpy as np
+    import synth
+    from oracle import nabla_oracle as orc
+    out = {}
+    # backward at the pretraining shape: one (b, h) in full
+    w = synth.WORKLOADS[4]
+    x = synth.make_inputs(w, heads=[0])
+    sl = (slice(0, 1), slice(0, 1))
+    M, _, _ = orc.nabla_mask(x["q"][sl], x["k"][sl], w.thresholds[0])
+    t0 = time.perf_counter()
+    orc.masked_attention_bwd(x["q"][sl], x["k"][sl], x["v"][sl], x["do"][sl], M)
+    t = time.perf_counter() - t0
+    kept = int(M.sum())
+    out["training_backward"] = {
+        "tflops": kept * 10 * 64 * 64 * w.D / t / 1e12, "full_config_extrapolated_s": t * w.B * w.H,
+        "sample": f"(b, h) = (0, 0) of the pretraining shape: fp64 backward under its mask ({kept} kept tiles, "
+                  f"{t:.2f} s), scaled to {w.B * w.H} heads"}
+    # Eq. 1 projection with the pooling: 256 tokens of the 720p shape, C = 5120
+    S_s, S_full, C, H, D = 256, 75600, 5120, 40, 128
+    pi = synth.make_projection_inputs(1, S_s, C, H, D, seed=3)
+    t0 = time.perf_counter()
+    Q, K, V = orc.qkv_project(pi["x"], pi["wt"], H, D)
+    orc.block_pool(orc.round_bf16(Q)), orc.block_pool(orc.round_bf16(K))
+    t = time.perf_counter() - t0
+    out["projection"] = {
+        "tflops": 2.0 * S_s * C * 3 * H * D / t / 1e12, "full_config_extrapolated_s": t * S_full / S_s,
+        "sample": f"{S_s} tokens of X [1, {S_full}, {C}] x W [{C}, 3 x {H * D}] in fp64 with the block means "
+                  f"of Q and K ({t:.2f} s), scaled to {S_full} tokens"}
+    # fractal reorder: the 720p latent with 64 fp32 channels (256-byte rows),
+    # scaled by row bytes to the 5120 bf16 channels of the GPU leg
+    T, Hl, Wl, P, ch = 21, 45, 80, 8, 64
+    a = np.random.default_rng(0).standard_normal((1, T * Hl * Wl, ch)).astype(np.float32)
+    t0 = time.perf_counter()
+    orc.fractal_reorder(a, T, Hl, Wl, P)
+    t = time.perf_counter() - t0
+    out["fractal_reorder"] = {
+        "full_config_extrapolated_s": t * (5120 * 2) / (ch * 4),
+        "sample": f"[1, {T}x{Hl}x{Wl}, {ch}] fp32 rows gathered ({t:.3f} s), scaled by bytes to {5120} "
+                  f"bf16 channels"}
+    # block fidelity: four query blocks of head 0 at the 720p shape
+    w3 = synth.WORKLOADS[WORKLOAD_ID]
+    x3 = synth.make_inputs(w3, heads=[0])
+    blocks = [0, 300, 700, w3.nb - 1]
+    t0 = time.perf_counter()
+    orc.block_mass_rows(x3["q"], x3["k"], 0, 0, blocks)
+    t = time.perf_counter() - t0
+    out["block_fidelity"] = {
+        "full_config_extrapolated_s": t / len(blocks) * w3.nb * w3.H,
+        "sample": f"block mass of {len(blocks)} query blocks of head 0 ({t:.2f} s), scaled to "
+                  f"{w3.nb} blocks x {w3.H} heads"}
+    # the sweeps and Table 1 run the main leg's kernels on other masks: their
+    # oracle time follows from the main leg's oracle rate on kept tiles
+    def derived(rows):
+        return [{"thr": r.get("thr"), "method": r.get("method"),
+                 "oracle_s_extrapolated": r["attn_tflops"] * r["attn_ms"] * 1e-3 / main_rate_tflops}
+                for r in rows]
+    if sweep:
+        out["sweep"] = {"note": "kept-tile flops / the main leg's oracle rate", "cases": derived(sweep["cases"])}
+    if table1:
+        out["table1"] = {"note": "kept-tile flops / the main leg's oracle rate", "cases": derived(table1["cases"])}
+    return out
+
+
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -912,6 +979,7 @@ def main() -> None:
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR,
                                                 heads_total=B * H)
+            line["cpu_baseline"]["legs"] = cpu_baseline_legs(line["cpu_baseline"]["value"], sweep, table1)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
