@@ -223,6 +223,22 @@ nabla_status nabla_qkv_project(const nabla_shape* shape, int32_t C, const void* 
   NABLA_TRY(check_tensor(k, "k"));
   NABLA_TRY(check_tensor(v, "v"));
   NABLA_TRY(check_ws(d, false, workspace, workspace_bytes));
+  if ((long long)3 * d.H * d.D > (1ll << 31) - 1)
+    return fail(NABLA_ERR_UNSUPPORTED, "3 * H * D = %lld output features is above 2^31 - 1", 3ll * d.H * d.D);
+  {
+    // the outputs may overlap neither the inputs, each other nor the workspace
+    const unsigned long long nqkv = (unsigned long long)d.BH() * d.S * d.D * 2;
+    struct Range { const void* p; unsigned long long n; const char* name; } r[6] = {
+        {x, (unsigned long long)d.B * d.S * C * 2, "x"}, {wt, 3ull * d.H * d.D * C * 2, "wt"},
+        {q, nqkv, "q"}, {k, nqkv, "k"}, {v, nqkv, "v"}, {workspace, workspace_bytes, "workspace"}};
+    for (int i = 2; i < 5; ++i)
+      for (int j = 0; j < 6; ++j) {
+        if (j == i) continue;
+        const uintptr_t a = (uintptr_t)r[i].p, b = (uintptr_t)r[j].p;
+        if (a < b + r[j].n && b < a + r[i].n)
+          return fail(NABLA_ERR_INVALID_ARG, "%s overlaps %s", r[i].name, r[j].name);
+      }
+  }
   cudaStream_t st = (cudaStream_t)stream;
   const WsLayout L = ws_layout(d, false);
   char* ws = (char*)workspace;

@@ -204,8 +204,9 @@ NABLA_API nabla_status nabla_build_mask_noalloc_status(int32_t* host_status, nab
  *          the kernel ran out.
  * All pointers 16-byte aligned.  Asynchronous on `stream`; allocates nothing.
  * Errors: NABLA_ERR_INVALID_ARG for an invalid shape, a NULL or misaligned
- * pointer or a bad C; NABLA_ERR_UNSUPPORTED for fp32 inputs, a block size, D
- * or sequence length this build does not handle, or C above the limit;
+ * pointer, a bad C, or q, k or v overlapping another buffer of the call;
+ * NABLA_ERR_UNSUPPORTED for fp32 inputs, a block size, D or sequence length
+ * this build does not handle, C above the limit or 3 H D above 2^31 - 1;
  * NABLA_ERR_WORKSPACE for a workspace that is too small or misaligned;
  * NABLA_ERR_CUDA if the launch fails. */
 NABLA_API nabla_status nabla_qkv_project(const nabla_shape* shape, int32_t C, const void* x, const void* wt,

@@ -122,6 +122,12 @@ def test_projection_argument_errors(L):
     assert proj(v=None) == INVALID
     assert proj(ws=None) == WORKSPACE
     assert proj(ws_bytes=1000) == WORKSPACE
+    big = 1 << 36                                        # far apart: no overlap
+    assert proj(k=FAKE + 16, q=FAKE, v=FAKE + big, x=FAKE + 2 * big, wt=FAKE + 3 * big,
+                ws=FAKE + 4 * big) == INVALID            # q and k overlap
+    assert b"overlaps" in L.nabla_last_error()
+    assert proj(q=FAKE + big, k=FAKE + 2 * big, v=FAKE + 3 * big, x=FAKE + 3 * big + 256,
+                wt=FAKE + 5 * big, ws=FAKE + 6 * big) == INVALID   # v over x
 
 
 def test_pooled_build_argument_errors(L):
