@@ -76,9 +76,9 @@ def test_projection_matches_the_oracle(B, H, S, D, C):
 
 
 @pytest.mark.parametrize("sta", [False, True])
-@pytest.mark.parametrize("B,H,S,C,thr", [(1, 2, 4096, 256, 0.8), (2, 3, 1000, 192, 0.9), (1, 2, 130, 64, 0.5)])
-def test_pooled_build_equals_the_build_from_q_and_k(B, H, S, C, thr, sta):
-    D = 128
+@pytest.mark.parametrize("B,H,S,D,C,thr", [(1, 2, 4096, 128, 256, 0.8), (2, 3, 1000, 128, 192, 0.9),
+                                           (1, 2, 130, 128, 64, 0.5), (1, 5, 3000, 64, 320, 0.7)])
+def test_pooled_build_equals_the_build_from_q_and_k(B, H, S, D, C, thr, sta):
     d = synth.make_projection_inputs(B, S, C, H, D, seed=7 + S)
     x, wt = d["x"].cuda(), d["wt"].cuda()
     q, k, v, ws = nabla.qkv_project(x, wt, H, D)
