@@ -125,3 +125,29 @@ def test_projection_full_720p_shape():
         G = orc.bits_to_mask(gu.gpu_bits(pooled), nb)[:, h:h + 1]
         exempt = orc.band_mask(Cm, 0.8, gu.BAND)
         assert int(((G != M) & ~exempt).sum()) == 0, h
+
+
+def test_projection_with_tiny_wait_limit_stops_cleanly():
+    """With a 1 ns limit the projection's first wait that is not already
+    satisfied runs out: the kernel stops, lets its own copies and MMAs land,
+    frees TMEM and reports NABLA_ERR_TIMEOUT (0 if every wait happened to be
+    satisfied at once).  The next call with the default limit is correct, and
+    so is the mask built from its means."""
+    B, H, S, D, C = 1, 4, 2000, 128, 512
+    d = synth.make_projection_inputs(B, S, C, H, D, seed=41)
+    x, wt = d["x"].cuda(), d["wt"].cuda()
+    q, k, v, ws = nabla.qkv_project(x, wt, H, D)
+    torch.cuda.synchronize()
+    try:
+        nabla.set_wait_limit_ns(1)
+        nabla.qkv_project(x, wt, H, D, q, k, v, ws)
+        torch.cuda.synchronize()
+        assert nabla.workspace_status(ws) in (0, 4)
+    finally:
+        nabla.set_wait_limit_ns(0)
+    nabla.qkv_project(x, wt, H, D, q, k, v, ws)
+    pooled = nabla.build_mask_pooled(q.shape, 0.8, ws)
+    torch.cuda.synchronize()
+    assert nabla.workspace_status(ws) == 0
+    _check_projection([q.cpu(), k.cpu(), v.cpu()], d["x"], d["wt"], H, D)
+    _same_mask(pooled, nabla.build_mask(q, k, 0.8), transpose=True)
