@@ -11,7 +11,11 @@
  *      restore the original order; optionally OR-ed (§3.1.3) with the
  *      sliding-tile (STA) window mask of §2.2;
  *   2. block-sparse attention over the kept 64 x 64 tiles: Eq. 4 of §2.2,
- *      softmax(Q K^T / sqrt(D) + M) V with M in {-inf, 0}, and its backward.
+ *      softmax(Q K^T / sqrt(D) + M) V with M in {-inf, 0}, and its backward;
+ *   3. around them: Eq. 1's projection Q = X W_Q, K = X W_K, V = X W_V with
+ *      the block averaging fused into it, the §3.1.1 token reordering, the
+ *      STA-only masks and block coordinates, a fixed-budget Top-k selection
+ *      and a per-block fidelity check of the pooling proxy.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
