@@ -979,7 +979,10 @@ def main() -> None:
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline({n: x[n][:, :1] for n in ("q", "k", "v")}, THR,
                                                 heads_total=B * H)
-            line["cpu_baseline"]["legs"] = cpu_baseline_legs(line["cpu_baseline"]["value"], sweep, table1)
+            try:
+                line["cpu_baseline"]["legs"] = cpu_baseline_legs(line["cpu_baseline"]["value"], sweep, table1)
+            except Exception as e:  # a host-side sample must not cost the bench line
+                line["cpu_baseline"]["legs"] = {"error": f"{type(e).__name__}: {e}"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
