@@ -86,8 +86,11 @@ def _peaks() -> dict:
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """Samples nvidia-smi clocks and throttle reasons while the timed region
+    runs: nvidia-smi is started (and has printed its first line) before the
+    region, every line carries its timestamp, and the summary keeps the lines
+    that fall between mark_start() and mark_end()."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -95,16 +98,26 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.file = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+            deadline = time.time() + 5.0
+            while time.time() < deadline and os.path.getsize(self.file.name) == 0:
+                time.sleep(0.05)  # sampling is live before the region starts
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -117,25 +130,40 @@ class ClockSampler:
     def summary(self) -> dict:
         if self.proc is None or self.file is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        import datetime
         self.file.flush()
         rows = [l.split(",") for l in open(self.file.name).read().strip().splitlines() if l.strip()]
         os.unlink(self.file.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        parsed = []
         for r in rows:
             r = [x.strip() for x in r]
-            if len(r) < 9:
+            if len(r) < 10:
                 continue
+            ts = None
+            for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+                try:
+                    ts = datetime.datetime.strptime(r[0], fmt).timestamp()
+                    break
+                except ValueError:
+                    pass
             try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
+                parsed.append((ts, float(r[2]), float(r[3]), r[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, r[5:9]):
+        inside = [p for p in parsed if p[0] is not None and self.t0 is not None and self.t1 is not None
+                  and self.t0 - 0.05 <= p[0] <= self.t1 + 0.05]
+        use = inside or parsed
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for p in use:
+            for n, v in zip(names, p[3]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [p[1] for p in use]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(p[2] for p in use) if use else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                **({} if inside else {"note": "no sample fell inside the timed region; all samples used"})}
 
 
 def rank_workload(w, rank: int):
@@ -860,23 +888,27 @@ def main() -> None:
         if ev:
             ev[2].record(stream)
 
-    for _ in range(max(args.warmup, 0)):
-        step()
-    torch.cuda.synchronize()
-    if nabla.workspace_status(ws) != 0:
-        raise SystemExit("device status word reports a timeout in warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    # the clock sampler starts before the warm-up (so that its start-up adds no
+    # idle gap before the timed region) and keeps the samples of the region
     with ClockSampler(local) as clocks:
+        for _ in range(max(args.warmup, 0)):
+            step()
+        torch.cuda.synchronize()
+        if nabla.workspace_status(ws) != 0:
+            raise SystemExit("device status word reports a timeout in warm-up")
+
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks.mark_start()
         t_start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_end()
     if world > 1:
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
