@@ -37,6 +37,11 @@
  * - On any error the call enqueues nothing (argument errors) or stops enqueuing
  *   (launch errors), returns a status != NABLA_OK and records a message that
  *   nabla_last_error() returns in the calling thread.
+ * - A call enqueues only kernel launches and memsets on `stream`, so a sequence
+ *   of calls can be captured into a CUDA graph and replayed; make one eager
+ *   call of each entry point on the device first (it loads the library's
+ *   modules).  No kernel accumulates with floating-point atomics: repeated
+ *   calls on the same inputs give bit-identical results.
  */
 #ifndef NABLA_H
 #define NABLA_H

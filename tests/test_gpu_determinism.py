@@ -49,3 +49,44 @@ def test_projection_and_pooled_mask_are_bitwise_repeatable():
     for r in runs[1:]:
         for name, a, b in zip(("q", "k", "v", "bits", "work"), runs[0], r):
             assert torch.equal(a, b), name
+
+
+def test_mask_and_forward_replay_from_a_cuda_graph():
+    """The step (mask build + forward) is stream-ordered launches and memsets
+    only, so it can be captured into a CUDA graph once and replayed: each
+    replay equals the eager calls bit for bit (inputs updated in place between
+    replays, as a serving loop would)."""
+    w = synth.WORKLOADS[4]
+    x = synth.make_inputs(w, heads=[0, 9])
+    y = synth.make_inputs(w.scaled(seed=w.seed + 1), heads=[0, 9])
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    B, H, S, D = q.shape
+    ws = nabla.workspace(q)
+    mask = nabla.Mask.empty(B, H, S, q.device, transpose=False)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+
+    def step():
+        nabla.build_mask(q, k, 0.8, out=mask, ws=ws, transpose=False)
+        nabla.attn_fwd(q, k, v, mask, o=o, lse=lse, ws=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                                          # warm: modules loaded, attributes set
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for inputs in (y, x):
+        for name, t in zip("qkv", (q, k, v)):
+            t.copy_(inputs[name].cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        assert nabla.workspace_status(ws) == 0
+        got = (mask.bits.clone(), o.clone(), lse.clone())
+        step()                                          # eager, same inputs
+        torch.cuda.synchronize()
+        for name, a, b in zip(("bits", "o", "lse"), got, (mask.bits, o, lse)):
+            assert torch.equal(a, b), name
