@@ -37,11 +37,14 @@
  * - On any error the call enqueues nothing (argument errors) or stops enqueuing
  *   (launch errors), returns a status != NABLA_OK and records a message that
  *   nabla_last_error() returns in the calling thread.
- * - A call enqueues only kernel launches and memsets on `stream`, so a sequence
- *   of calls can be captured into a CUDA graph and replayed; make one eager
- *   call of each entry point on the device first (it loads the library's
- *   modules).  No kernel accumulates with floating-point atomics: repeated
- *   calls on the same inputs give bit-identical results.
+ * - The builders, attention, projection, reorder and fidelity calls enqueue
+ *   only kernel launches and memsets on `stream`, so a sequence of them can be
+ *   captured into a CUDA graph and replayed; make one eager call of each on
+ *   the device first (it loads the library's modules).  The status read-backs
+ *   (nabla_workspace_status, nabla_build_mask_noalloc_status) copy to the host
+ *   and synchronise, so they stay outside a capture.  No kernel accumulates
+ *   with floating-point atomics: repeated calls on the same inputs give
+ *   bit-identical results.
  */
 #ifndef NABLA_H
 #define NABLA_H
